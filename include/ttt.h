@@ -1,0 +1,154 @@
+/*
+ * ttt.h - C ABI of libttt_b200.so: forward pass of chunked test-time-training
+ * (TTT) layers with key->value binding, on one NVIDIA B200 (sm_100a).
+ *
+ * Three operations, each a per-(batch, head) scan over chunks of `chunk`
+ * tokens with fast weights W kept in fp32:
+ *
+ *  ttt_linear_fwd, loss = TTT_LOSS_MSE  (TTT-Linear, mini-batch GD)
+ *    "Test-Time Training (TTT)" summary, sections "TTT 정의", "예시 2: DeltaNet
+ *    유도", "TTT-Linear" and "병렬화: Mini-batch Gradient Descent": with
+ *    t' = t - (t mod chunk),
+ *      W_t = W_{t'} - sum_{i=t'}^{t} eta_i k_i^T (k_i W_{t'} - v_i),
+ *      y_t = q_t W_t          (row vectors; W is dk x dv).
+ *    Equivalently, per chunk (Q, K, V the chunk's rows, N = diag(eta),
+ *    tril keeps i <= t): Y = QW - tril(QK^T) N (KW - V);
+ *    W <- W - K^T N (KW - V).
+ *
+ *  ttt_linear_fwd, loss = TTT_LOSS_NEG_DOT  (inner-product loss)
+ *    Same page, sections "Linear Attention" and "예시 1: Linear Attention
+ *    유도": the gradient -k^T v does not depend on W, so the layer is causal
+ *    linear attention with per-token weights: S_t = S_{t-1} + eta_t k_t^T v_t,
+ *    y_t = q_t S_t, S_0 = W0; the result does not depend on `chunk`.
+ *    ("Test-Time Training with KV Binding Is Secretly Linear Attention",
+ *    abstract: TTT with KV binding as a learned linear-attention operator.)
+ *
+ *  lact_swiglu_fwd  (LaCT large-chunk SwiGLU fast weights)
+ *    "Test-Time Training Done Right" review, sections 3.2, 3.3 and 4 /
+ *    Figure 3: f(x) = W2 (silu(W1 x) * W3 x); per chunk c the loss
+ *    sum_i eta_i * (-f(k_i) . v_i) is differentiated at the current weights,
+ *    the gradients G1, G2, G3 are optionally orthogonalised by 5 Newton-Schulz
+ *    steps X <- aX + b(XX^T)X + c(XX^T)^2 X, (a,b,c) = (3.4445, -4.7750,
+ *    2.0315), from X0 = G / (||G||_F + 1e-7) (Muon), then W <- W - G and every
+ *    row of W1, W3 (over dk) and of W2 (over dh) is rescaled to the L2 norm it
+ *    had in the initial weights. causal=1: chunk c's queries see the weights
+ *    before chunk c's update (apply, then update); causal=0: update with
+ *    chunk c, then apply to chunk c.
+ *
+ * Conventions shared by every entry point
+ *  - Tensors are described by ttt_tensor: a device pointer, an element type,
+ *    and shape/stride in ELEMENTS (not bytes). Token tensors q, k, v, out are
+ *    4-d [B, H, T, d] with any strides whose last one is 1; eta is 3-d
+ *    [B, H, T] fp32 with any strides. Weight tensors are contiguous
+ *    (row-major) with the shapes given below.
+ *  - Alignment: every base pointer must be 16-byte aligned and every stride of
+ *    q, k, v, out times the element size must be a multiple of 16 bytes.
+ *  - Ownership: all memory is the caller's. The library keeps no pointer past
+ *    the call and never frees caller memory. Inputs are read-only; `out` and
+ *    the *_final tensors must not overlap any input.
+ *  - Asynchrony: work is enqueued on `stream` (a cudaStream_t passed as
+ *    void*; NULL = the legacy default stream) and the call returns without
+ *    waiting for it. Argument errors are detected on the host before anything
+ *    is launched and returned synchronously; nothing is written then.
+ *  - Device-side errors: kernels that wait on a barrier give up after a
+ *    bounded number of polls and record TTT_ERR_TIMEOUT in a device status
+ *    word instead of hanging; ttt_get_device_status() reads and clears it.
+ *  - Supported sizes: B, H, T >= 1 (T = 0 is accepted and does nothing
+ *    except copying W0 to W_final); chunk >= 1 (a shorter last chunk is
+ *    allowed); dk, dv in [1, 256] for fp32 tensors. bf16 kernels take
+ *    dk = dv in {64, 128} for TTT-Linear and d in {64, 128, 256},
+ *    dh a multiple of 128 up to 1024 for LaCT; other sizes return
+ *    TTT_ERR_UNSUPPORTED.
+ */
+#ifndef TTT_B200_H
+#define TTT_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TTT_OK = 0,
+  TTT_ERR_NULL = -1,        /* a required pointer is NULL */
+  TTT_ERR_SHAPE = -2,       /* sizes inconsistent across tensors, or ndim wrong */
+  TTT_ERR_DTYPE = -3,       /* element type not allowed for this tensor */
+  TTT_ERR_LAYOUT = -4,      /* stride or 16-byte alignment rule broken */
+  TTT_ERR_UNSUPPORTED = -5, /* valid request this build has no kernel for */
+  TTT_ERR_CUDA = -6,        /* a CUDA runtime call failed (launch, memory) */
+  TTT_ERR_TIMEOUT = -7,     /* a device-side bounded wait gave up */
+  TTT_ERR_ALLOC = -8,       /* stream-ordered scratch allocation failed */
+  TTT_ERR_ARG = -9          /* scalar argument out of range (chunk, enums) */
+} ttt_status;
+
+typedef enum { TTT_F32 = 0, TTT_BF16 = 1 } ttt_dtype;
+
+typedef enum { TTT_LOSS_MSE = 0, TTT_LOSS_NEG_DOT = 1 } ttt_loss;
+
+typedef enum { LACT_UPDATE_GD = 0, LACT_UPDATE_MUON = 1 } lact_update_rule;
+
+typedef struct {
+  void* data;          /* device pointer, 16-byte aligned */
+  int32_t dtype;       /* ttt_dtype */
+  int32_t ndim;        /* number of valid entries in shape/stride */
+  int64_t shape[4];
+  int64_t stride[4];   /* in elements */
+} ttt_tensor;
+
+/*
+ * TTT-Linear / inner-product layer forward.
+ *  q, k   [B,H,T,dk]  fp32 or bf16 (same type for q, k, v, out)
+ *  v      [B,H,T,dv]
+ *  eta    [B,H,T]     fp32, per-token learning rate
+ *  W0     [H,dk,dv] (shared over the batch) or [B,H,dk,dv], fp32, contiguous
+ *  chunk  mini-batch size b >= 1
+ *  loss   TTT_LOSS_MSE or TTT_LOSS_NEG_DOT
+ *  out    [B,H,T,dv]  same type as q
+ *  W_final NULL, or [B,H,dk,dv] fp32 contiguous: weights after the last token
+ */
+ttt_status ttt_linear_fwd(const ttt_tensor* q, const ttt_tensor* k, const ttt_tensor* v,
+                          const ttt_tensor* eta, const ttt_tensor* W0, int32_t chunk,
+                          int32_t loss, const ttt_tensor* out, const ttt_tensor* W_final,
+                          void* stream);
+
+/*
+ * LaCT SwiGLU layer forward.
+ *  q, k [B,H,T,dk] bf16 or fp32; v, out [B,H,T,dv] (dk == dv for bf16)
+ *  eta  [B,H,T] fp32
+ *  W1, W3 [H,dh,dk] or [B,H,dh,dk]; W2 [H,dv,dh] or [B,H,dv,dh]; fp32,
+ *         contiguous, read-only (the scan works on private copies)
+ *  chunk  >= 1; update_rule LACT_UPDATE_GD or LACT_UPDATE_MUON; causal 0/1
+ * Scratch is taken stream-ordered from the device's default memory pool
+ * (cudaMallocAsync / cudaFreeAsync on `stream`); failure -> TTT_ERR_ALLOC.
+ */
+ttt_status lact_swiglu_fwd(const ttt_tensor* q, const ttt_tensor* k, const ttt_tensor* v,
+                           const ttt_tensor* eta, const ttt_tensor* W1, const ttt_tensor* W2,
+                           const ttt_tensor* W3, int32_t chunk, int32_t update_rule,
+                           int32_t causal, const ttt_tensor* out, void* stream);
+
+/* As lact_swiglu_fwd, also writing the final fast weights (each NULLable):
+ * W1_final, W3_final [B,H,dh,dk], W2_final [B,H,dv,dh], fp32 contiguous. */
+ttt_status lact_swiglu_fwd_ex(const ttt_tensor* q, const ttt_tensor* k, const ttt_tensor* v,
+                              const ttt_tensor* eta, const ttt_tensor* W1, const ttt_tensor* W2,
+                              const ttt_tensor* W3, int32_t chunk, int32_t update_rule,
+                              int32_t causal, const ttt_tensor* out,
+                              const ttt_tensor* W1_final, const ttt_tensor* W2_final,
+                              const ttt_tensor* W3_final, void* stream);
+
+/* Static description of a status code (never NULL). */
+const char* ttt_status_string(int32_t status);
+
+/* Synchronises `stream`, returns the first device-side error recorded since
+ * the last call (TTT_OK if none) and clears it. */
+ttt_status ttt_get_device_status(void* stream);
+
+/* Library version, as major*10000 + minor*100 + patch. */
+int32_t ttt_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TTT_B200_H */

@@ -1,0 +1,315 @@
+// C ABI of libttt_b200: argument validation and dispatch (see include/ttt.h).
+#include <mutex>
+
+#include "common.cuh"
+#include "lact.cuh"
+
+namespace {
+
+__device__ int g_device_status;
+
+constexpr int kMaxDevices = 64;
+int* g_status_ptr[kMaxDevices] = {};
+std::mutex g_status_mu;
+
+// Device address of the status word on the current device (looked up once
+// per device; the symbol itself is a host-side handle, not an address).
+int* device_status_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_status_mu);
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+    g_status_ptr[dev] = static_cast<int*>(p);
+  }
+  return g_status_ptr[dev];
+}
+
+size_t elem_size(int32_t dtype) { return dtype == TTT_BF16 ? 2 : 4; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Byte range [lo, hi) touched by a strided tensor (non-negative strides).
+struct Extent {
+  uintptr_t lo, hi;
+};
+Extent extent(const ttt_tensor* t) {
+  uintptr_t base = reinterpret_cast<uintptr_t>(t->data);
+  int64_t last = 0;
+  for (int i = 0; i < t->ndim; ++i) last += (t->shape[i] - 1) * t->stride[i];
+  return {base, base + (uintptr_t)((last + 1) * (int64_t)elem_size(t->dtype))};
+}
+bool empty(const ttt_tensor* t) {
+  for (int i = 0; i < t->ndim; ++i)
+    if (t->shape[i] == 0) return true;
+  return false;
+}
+bool overlaps(const ttt_tensor* a, const ttt_tensor* b) {
+  if (!a || !b || empty(a) || empty(b)) return false;
+  Extent x = extent(a), y = extent(b);
+  return x.lo < y.hi && y.lo < x.hi;
+}
+
+bool contiguous(const ttt_tensor* t) {
+  int64_t s = 1;
+  for (int i = t->ndim - 1; i >= 0; --i) {
+    if (t->shape[i] != 1 && t->stride[i] != s) return false;
+    s *= t->shape[i];
+  }
+  return true;
+}
+
+ttt_status check_tokens(const ttt_tensor* t, int64_t B, int64_t H, int64_t T, int64_t d,
+                        int32_t dtype) {
+  if (!t->data && !(B * H * T * d == 0)) return TTT_ERR_NULL;
+  if (t->ndim != 4) return TTT_ERR_SHAPE;
+  if (t->shape[0] != B || t->shape[1] != H || t->shape[2] != T || t->shape[3] != d)
+    return TTT_ERR_SHAPE;
+  if (t->dtype != dtype) return TTT_ERR_DTYPE;
+  if (t->stride[3] != 1 && d > 1) return TTT_ERR_LAYOUT;
+  const int64_t es = (int64_t)elem_size(dtype);
+  for (int i = 0; i < 3; ++i) {
+    if (t->stride[i] < 0) return TTT_ERR_LAYOUT;
+    if ((t->stride[i] * es) % 16 != 0 && t->shape[i] > 1) return TTT_ERR_LAYOUT;
+  }
+  if (!aligned16(t->data)) return TTT_ERR_LAYOUT;
+  return TTT_OK;
+}
+
+ttt::TokView view(const ttt_tensor* t) { return {t->data, t->stride[0], t->stride[1], t->stride[2]}; }
+
+}  // namespace
+
+extern "C" {
+
+int32_t ttt_version(void) { return 100; }
+
+const char* ttt_status_string(int32_t s) {
+  switch (s) {
+    case TTT_OK: return "ok";
+    case TTT_ERR_NULL: return "a required pointer is NULL";
+    case TTT_ERR_SHAPE: return "tensor shapes are inconsistent or have the wrong rank";
+    case TTT_ERR_DTYPE: return "element type not allowed for this tensor";
+    case TTT_ERR_LAYOUT: return "stride or 16-byte alignment rule broken";
+    case TTT_ERR_UNSUPPORTED: return "no kernel in this build for these sizes/types";
+    case TTT_ERR_CUDA: return "a CUDA runtime call failed";
+    case TTT_ERR_TIMEOUT: return "a device-side bounded wait gave up";
+    case TTT_ERR_ALLOC: return "stream-ordered scratch allocation failed";
+    case TTT_ERR_ARG: return "scalar argument out of range";
+    default: return "unknown status";
+  }
+}
+
+ttt_status ttt_get_device_status(void* stream) {
+  int* p = device_status_ptr();
+  if (!p) return TTT_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return TTT_ERR_CUDA;
+  int v = 0, zero = 0;
+  if (cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return TTT_ERR_CUDA;
+  if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return TTT_ERR_CUDA;
+  if (v == ttt::DEV_TIMEOUT) return TTT_ERR_TIMEOUT;
+  if (v != ttt::DEV_OK) return TTT_ERR_CUDA;
+  return TTT_OK;
+}
+
+ttt_status ttt_linear_fwd(const ttt_tensor* q, const ttt_tensor* k, const ttt_tensor* v,
+                          const ttt_tensor* eta, const ttt_tensor* W0, int32_t chunk,
+                          int32_t loss, const ttt_tensor* out, const ttt_tensor* W_final,
+                          void* stream) {
+  if (!q || !k || !v || !eta || !W0 || !out) return TTT_ERR_NULL;
+  if (chunk < 1) return TTT_ERR_ARG;
+  if (loss != TTT_LOSS_MSE && loss != TTT_LOSS_NEG_DOT) return TTT_ERR_ARG;
+  if (q->ndim != 4 || v->ndim != 4) return TTT_ERR_SHAPE;
+  const int64_t B = q->shape[0], H = q->shape[1], T = q->shape[2], dk = q->shape[3];
+  const int64_t dv = v->shape[3];
+  if (B < 1 || H < 1 || T < 0 || dk < 1 || dv < 1) return TTT_ERR_SHAPE;
+  if (dk > 256 || dv > 256 || T > (int64_t)1 << 31 || B * H > (1 << 30)) return TTT_ERR_UNSUPPORTED;
+  const int32_t dt = q->dtype;
+  if (dt != TTT_F32 && dt != TTT_BF16) return TTT_ERR_DTYPE;
+  ttt_status st;
+  if ((st = check_tokens(q, B, H, T, dk, dt)) != TTT_OK) return st;
+  if ((st = check_tokens(k, B, H, T, dk, dt)) != TTT_OK) return st;
+  if ((st = check_tokens(v, B, H, T, dv, dt)) != TTT_OK) return st;
+  if ((st = check_tokens(out, B, H, T, dv, dt)) != TTT_OK) return st;
+  // eta [B,H,T] fp32, any non-negative strides
+  if (eta->ndim != 3 || eta->shape[0] != B || eta->shape[1] != H || eta->shape[2] != T)
+    return TTT_ERR_SHAPE;
+  if (eta->dtype != TTT_F32) return TTT_ERR_DTYPE;
+  if (!eta->data && T > 0) return TTT_ERR_NULL;
+  for (int i = 0; i < 3; ++i)
+    if (eta->stride[i] < 0) return TTT_ERR_LAYOUT;
+  if (!aligned16(eta->data)) return TTT_ERR_LAYOUT;
+  // W0 [H,dk,dv] or [B,H,dk,dv] fp32 contiguous
+  if (!W0->data) return TTT_ERR_NULL;
+  if (W0->dtype != TTT_F32) return TTT_ERR_DTYPE;
+  int64_t w0_sb = 0;
+  if (W0->ndim == 3) {
+    if (W0->shape[0] != H || W0->shape[1] != dk || W0->shape[2] != dv) return TTT_ERR_SHAPE;
+  } else if (W0->ndim == 4) {
+    if (W0->shape[0] != B || W0->shape[1] != H || W0->shape[2] != dk || W0->shape[3] != dv)
+      return TTT_ERR_SHAPE;
+    w0_sb = H * dk * dv;
+  } else {
+    return TTT_ERR_SHAPE;
+  }
+  if (!contiguous(W0) || !aligned16(W0->data)) return TTT_ERR_LAYOUT;
+  if (W_final) {
+    if (!W_final->data) return TTT_ERR_NULL;
+    if (W_final->dtype != TTT_F32) return TTT_ERR_DTYPE;
+    if (W_final->ndim != 4 || W_final->shape[0] != B || W_final->shape[1] != H ||
+        W_final->shape[2] != dk || W_final->shape[3] != dv)
+      return TTT_ERR_SHAPE;
+    if (!contiguous(W_final) || !aligned16(W_final->data)) return TTT_ERR_LAYOUT;
+  }
+  const ttt_tensor* ins[] = {q, k, v, eta, W0};
+  for (const ttt_tensor* in : ins)
+    if (overlaps(out, in) || overlaps(W_final, in)) return TTT_ERR_ARG;
+  if (overlaps(out, W_final)) return TTT_ERR_ARG;
+
+  ttt::LinearArgs a;
+  a.q = view(q);
+  a.k = view(k);
+  a.v = view(v);
+  a.eta = {static_cast<const float*>(eta->data), eta->stride[0], eta->stride[1], eta->stride[2]};
+  a.W0 = static_cast<const float*>(W0->data);
+  a.w0_sb = w0_sb;
+  a.out = {out->data, out->stride[0], out->stride[1], out->stride[2]};
+  a.W_final = W_final ? static_cast<float*>(W_final->data) : nullptr;
+  a.B = (int)B;
+  a.H = (int)H;
+  a.T = (int)T;
+  a.dk = (int)dk;
+  a.dv = (int)dv;
+  a.chunk = chunk;
+  a.loss = loss;
+  a.status = device_status_ptr();
+  if (!a.status) return TTT_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  cudaError_t e;
+  if (dt == TTT_F32) {
+    e = ttt::launch_ttt_linear_f32(a, s);
+  } else {
+    bool supported = false;
+    e = ttt::launch_ttt_linear_bf16(a, s, &supported);
+    if (!supported) return TTT_ERR_UNSUPPORTED;
+  }
+  return e == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
+}
+
+static ttt_status lact_check_weight(const ttt_tensor* W, int64_t B, int64_t H, int64_t r,
+                                    int64_t c, int64_t* sb) {
+  if (!W->data) return TTT_ERR_NULL;
+  if (W->dtype != TTT_F32) return TTT_ERR_DTYPE;
+  if (W->ndim == 3) {
+    if (W->shape[0] != H || W->shape[1] != r || W->shape[2] != c) return TTT_ERR_SHAPE;
+    *sb = 0;
+  } else if (W->ndim == 4) {
+    if (W->shape[0] != B || W->shape[1] != H || W->shape[2] != r || W->shape[3] != c)
+      return TTT_ERR_SHAPE;
+    *sb = H * r * c;
+  } else {
+    return TTT_ERR_SHAPE;
+  }
+  if (!contiguous(W) || !aligned16(W->data)) return TTT_ERR_LAYOUT;
+  return TTT_OK;
+}
+
+static ttt_status lact_check_final(const ttt_tensor* W, int64_t B, int64_t H, int64_t r,
+                                   int64_t c) {
+  if (!W) return TTT_OK;
+  if (!W->data) return TTT_ERR_NULL;
+  if (W->dtype != TTT_F32) return TTT_ERR_DTYPE;
+  if (W->ndim != 4 || W->shape[0] != B || W->shape[1] != H || W->shape[2] != r ||
+      W->shape[3] != c)
+    return TTT_ERR_SHAPE;
+  if (!contiguous(W) || !aligned16(W->data)) return TTT_ERR_LAYOUT;
+  return TTT_OK;
+}
+
+ttt_status lact_swiglu_fwd_ex(const ttt_tensor* q, const ttt_tensor* k, const ttt_tensor* v,
+                              const ttt_tensor* eta, const ttt_tensor* W1, const ttt_tensor* W2,
+                              const ttt_tensor* W3, int32_t chunk, int32_t update_rule,
+                              int32_t causal, const ttt_tensor* out,
+                              const ttt_tensor* W1_final, const ttt_tensor* W2_final,
+                              const ttt_tensor* W3_final, void* stream) {
+  if (!q || !k || !v || !eta || !W1 || !W2 || !W3 || !out) return TTT_ERR_NULL;
+  if (chunk < 1) return TTT_ERR_ARG;
+  if (update_rule != LACT_UPDATE_GD && update_rule != LACT_UPDATE_MUON) return TTT_ERR_ARG;
+  if (causal != 0 && causal != 1) return TTT_ERR_ARG;
+  if (q->ndim != 4 || v->ndim != 4 || W1->ndim < 3) return TTT_ERR_SHAPE;
+  const int64_t B = q->shape[0], H = q->shape[1], T = q->shape[2], dk = q->shape[3];
+  const int64_t dv = v->shape[3];
+  const int64_t dh = W1->shape[W1->ndim - 2];
+  if (B < 1 || H < 1 || T < 0 || dk < 1 || dv < 1 || dh < 1) return TTT_ERR_SHAPE;
+  const int32_t dt = q->dtype;
+  if (dt != TTT_F32 && dt != TTT_BF16) return TTT_ERR_DTYPE;
+  ttt_status st;
+  if ((st = check_tokens(q, B, H, T, dk, dt)) != TTT_OK) return st;
+  if ((st = check_tokens(k, B, H, T, dk, dt)) != TTT_OK) return st;
+  if ((st = check_tokens(v, B, H, T, dv, dt)) != TTT_OK) return st;
+  if ((st = check_tokens(out, B, H, T, dv, dt)) != TTT_OK) return st;
+  if (eta->ndim != 3 || eta->shape[0] != B || eta->shape[1] != H || eta->shape[2] != T)
+    return TTT_ERR_SHAPE;
+  if (eta->dtype != TTT_F32) return TTT_ERR_DTYPE;
+  if (!eta->data && T > 0) return TTT_ERR_NULL;
+  for (int i = 0; i < 3; ++i)
+    if (eta->stride[i] < 0) return TTT_ERR_LAYOUT;
+  if (!aligned16(eta->data)) return TTT_ERR_LAYOUT;
+  int64_t sb1, sb2, sb3;
+  if ((st = lact_check_weight(W1, B, H, dh, dk, &sb1)) != TTT_OK) return st;
+  if ((st = lact_check_weight(W2, B, H, dv, dh, &sb2)) != TTT_OK) return st;
+  if ((st = lact_check_weight(W3, B, H, dh, dk, &sb3)) != TTT_OK) return st;
+  if ((st = lact_check_final(W1_final, B, H, dh, dk)) != TTT_OK) return st;
+  if ((st = lact_check_final(W2_final, B, H, dv, dh)) != TTT_OK) return st;
+  if ((st = lact_check_final(W3_final, B, H, dh, dk)) != TTT_OK) return st;
+  const ttt_tensor* ins[] = {q, k, v, eta, W1, W2, W3};
+  const ttt_tensor* outs[] = {out, W1_final, W2_final, W3_final};
+  for (const ttt_tensor* o : outs) {
+    for (const ttt_tensor* in : ins)
+      if (overlaps(o, in)) return TTT_ERR_ARG;
+    for (const ttt_tensor* o2 : outs)
+      if (o != o2 && overlaps(o, o2)) return TTT_ERR_ARG;
+  }
+
+  ttt::LactArgs a;
+  a.q = view(q);
+  a.k = view(k);
+  a.v = view(v);
+  a.eta = {static_cast<const float*>(eta->data), eta->stride[0], eta->stride[1], eta->stride[2]};
+  a.W1 = static_cast<const float*>(W1->data);
+  a.W2 = static_cast<const float*>(W2->data);
+  a.W3 = static_cast<const float*>(W3->data);
+  a.w_sb[0] = sb1;
+  a.w_sb[1] = sb2;
+  a.w_sb[2] = sb3;
+  a.out = {out->data, out->stride[0], out->stride[1], out->stride[2]};
+  a.W1_final = W1_final ? static_cast<float*>(W1_final->data) : nullptr;
+  a.W2_final = W2_final ? static_cast<float*>(W2_final->data) : nullptr;
+  a.W3_final = W3_final ? static_cast<float*>(W3_final->data) : nullptr;
+  a.B = (int)B;
+  a.H = (int)H;
+  a.T = (int)T;
+  a.dk = (int)dk;
+  a.dv = (int)dv;
+  a.dh = (int)dh;
+  a.chunk = chunk;
+  a.update_rule = update_rule;
+  a.causal = causal;
+  a.dtype = dt;
+  a.status = device_status_ptr();
+  if (!a.status) return TTT_ERR_CUDA;
+  return ttt::lact_forward(a, static_cast<cudaStream_t>(stream));
+}
+
+ttt_status lact_swiglu_fwd(const ttt_tensor* q, const ttt_tensor* k, const ttt_tensor* v,
+                           const ttt_tensor* eta, const ttt_tensor* W1, const ttt_tensor* W2,
+                           const ttt_tensor* W3, int32_t chunk, int32_t update_rule,
+                           int32_t causal, const ttt_tensor* out, void* stream) {
+  return lact_swiglu_fwd_ex(q, k, v, eta, W1, W2, W3, chunk, update_rule, causal, out, nullptr,
+                            nullptr, nullptr, stream);
+}
+
+}  // extern "C"

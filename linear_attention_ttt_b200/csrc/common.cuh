@@ -1,0 +1,103 @@
+// Shared device/host helpers of libttt_b200 (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/ttt.h"
+
+namespace ttt {
+
+// Error codes a kernel can record in the device status word.
+enum : int { DEV_OK = 0, DEV_TIMEOUT = 1, DEV_BAD_ARGS = 2 };
+
+// Upper bound on polls of one barrier before a kernel gives up (far above any
+// legitimate wait: a poll is tens of ns, so this is on the order of seconds).
+constexpr uint32_t kMaxPolls = 1u << 26;
+
+__device__ __forceinline__ void record_error(int* status, int code) {
+  if (status) atomicCAS(status, DEV_OK, code);
+}
+
+// Strided view of a [B,H,T,d] token tensor (element strides, last stride 1).
+struct TokView {
+  const void* p;
+  int64_t sb, sh, st;
+};
+struct TokViewMut {
+  void* p;
+  int64_t sb, sh, st;
+};
+struct EtaView {
+  const float* p;
+  int64_t sb, sh, st;
+};
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// ---- mbarrier / async-proxy primitives (inline PTX) -------------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait: returns false (and records DEV_TIMEOUT) if the phase never
+// completes within kMaxPolls polls.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
+  for (uint32_t i = 0; i < kMaxPolls; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  record_error(status, DEV_TIMEOUT);
+  return false;
+}
+
+}  // namespace ttt
+
+// Host-side launchers implemented in the kernel translation units.
+namespace ttt {
+
+struct LinearArgs {
+  TokView q, k, v;
+  EtaView eta;
+  const float* W0;
+  int64_t w0_sb;   // 0 when W0 is shared over the batch
+  TokViewMut out;
+  float* W_final;  // may be null
+  int B, H, T, dk, dv, chunk, loss;
+  int* status;
+};
+
+cudaError_t launch_ttt_linear_f32(const LinearArgs& a, cudaStream_t s);
+cudaError_t launch_ttt_linear_bf16(const LinearArgs& a, cudaStream_t s, bool* supported);
+
+}  // namespace ttt

@@ -1,0 +1,146 @@
+// TTT-Linear / inner-product layer forward for fp32 tokens (CUDA cores, fp32
+// throughout).
+//
+// Computes, per (batch, head), the mini-batch GD rule of the "Test-Time
+// Training (TTT)" summary ("병렬화: Mini-batch Gradient Descent"): with t' the
+// chunk start,  y_t = q_t W_t,  W_t = W_{t'} - sum_{i=t'}^{t} eta_i k_i^T e_i,
+// e_i = k_i W_{t'} - v_i (MSE, "예시 2") or e_i = -v_i (inner product,
+// "예시 1"). It walks a chunk in blocks of 16 tokens and keeps two fp32
+// matrices in shared memory: the chunk-start weights W_{t'} and the running
+// sum dW of the chunk's updates so far, so that for a token t in the current
+// block
+//   y_t = q_t (W_{t'} - dW) - sum_{i in block, i <= t} eta_i (q_t . k_i) e_i.
+// Any chunk size works, including a shorter last chunk.
+//
+// Grid: (B*H, ceil(dv/32)); each CTA owns 32 output columns of one head. The
+// columns of W are independent in this rule, so no CTA talks to another.
+#include "common.cuh"
+
+namespace ttt {
+namespace {
+
+constexpr int kCols = 32;     // W columns per CTA
+constexpr int kTB = 16;       // tokens per block
+constexpr int kThreads = 256;
+
+template <typename T>
+__device__ __forceinline__ const T* tok_row(const TokView& v, int b, int h, int64_t t) {
+  return static_cast<const T*>(v.p) + b * v.sb + h * v.sh + t * v.st;
+}
+
+__global__ void __launch_bounds__(kThreads)
+ttt_linear_f32_kernel(LinearArgs a) {
+  extern __shared__ float smem[];
+  const int dk = a.dk, dv = a.dv;
+  const int bh = blockIdx.x;
+  const int b = bh / a.H, h = bh % a.H;
+  const int j0 = blockIdx.y * kCols;
+  const int ncol = min(kCols, dv - j0);
+  const int tid = threadIdx.x;
+
+  float* Wst = smem;                 // [dk][kCols] chunk-start weights
+  float* dW = Wst + dk * kCols;      // [dk][kCols] sum of this chunk's updates
+  float* Qs = dW + dk * kCols;       // [kTB][dk]
+  float* Ks = Qs + kTB * dk;         // [kTB][dk]
+  float* Vs = Ks + kTB * dk;         // [kTB][kCols]
+  float* Es = Vs + kTB * kCols;      // [kTB][kCols]
+  float* Ss = Es + kTB * kCols;      // [kTB][kTB]  q_t . k_i
+  float* etas = Ss + kTB * kTB;      // [kTB]
+
+  const float* W0 = a.W0 + b * a.w0_sb + (int64_t)h * dk * dv;
+  for (int x = tid; x < dk * kCols; x += kThreads) {
+    int r = x / kCols, c = x % kCols;
+    Wst[x] = (c < ncol) ? W0[(int64_t)r * dv + j0 + c] : 0.f;
+    dW[x] = 0.f;
+  }
+  __syncthreads();
+
+  const float* eta = a.eta.p + b * a.eta.sb + h * a.eta.sh;
+  for (int cs = 0; cs < a.T; cs += a.chunk) {
+    const int ce = min(cs + a.chunk, a.T);
+    for (int t0 = cs; t0 < ce; t0 += kTB) {
+      const int nt = min(kTB, ce - t0);
+      for (int x = tid; x < kTB * dk; x += kThreads) {
+        int i = x / dk, c = x % dk;
+        bool ok = i < nt;
+        Qs[x] = ok ? tok_row<float>(a.q, b, h, t0 + i)[c] : 0.f;
+        Ks[x] = ok ? tok_row<float>(a.k, b, h, t0 + i)[c] : 0.f;
+      }
+      for (int x = tid; x < kTB * kCols; x += kThreads) {
+        int i = x / kCols, c = x % kCols;
+        Vs[x] = (i < nt && c < ncol) ? tok_row<float>(a.v, b, h, t0 + i)[j0 + c] : 0.f;
+      }
+      if (tid < kTB) etas[tid] = tid < nt ? eta[(int64_t)(t0 + tid) * a.eta.st] : 0.f;
+      __syncthreads();
+
+      // e_i at the chunk-start weights; scores q_t . k_i.
+      for (int x = tid; x < kTB * kCols; x += kThreads) {
+        int i = x / kCols, c = x % kCols;
+        float acc = 0.f;
+        if (a.loss == TTT_LOSS_MSE)
+          for (int r = 0; r < dk; ++r) acc = fmaf(Ks[i * dk + r], Wst[r * kCols + c], acc);
+        Es[x] = acc - Vs[x];
+      }
+      {
+        int t = tid / kTB, i = tid % kTB;
+        float acc = 0.f;
+        if (i <= t)
+          for (int r = 0; r < dk; ++r) acc = fmaf(Qs[t * dk + r], Ks[i * dk + r], acc);
+        Ss[tid] = acc;
+      }
+      __syncthreads();
+
+      // y_t = q_t (W_{t'} - dW) - sum_{i<=t} eta_i s_ti e_i
+      for (int x = tid; x < kTB * kCols; x += kThreads) {
+        int t = x / kCols, c = x % kCols;
+        if (t < nt && c < ncol) {
+          float acc = 0.f;
+          for (int r = 0; r < dk; ++r)
+            acc = fmaf(Qs[t * dk + r], Wst[r * kCols + c] - dW[r * kCols + c], acc);
+          for (int i = 0; i <= t; ++i) acc = fmaf(-etas[i] * Ss[t * kTB + i], Es[i * kCols + c], acc);
+          float* o = static_cast<float*>(a.out.p) + b * a.out.sb + h * a.out.sh +
+                     (int64_t)(t0 + t) * a.out.st;
+          o[j0 + c] = acc;
+        }
+      }
+      __syncthreads();
+
+      // dW += sum_i eta_i k_i^T e_i
+      for (int x = tid; x < dk * kCols; x += kThreads) {
+        int r = x / kCols, c = x % kCols;
+        float acc = dW[x];
+        for (int i = 0; i < nt; ++i) acc = fmaf(etas[i] * Ks[i * dk + r], Es[i * kCols + c], acc);
+        dW[x] = acc;
+      }
+      __syncthreads();
+    }
+    for (int x = tid; x < dk * kCols; x += kThreads) {
+      Wst[x] -= dW[x];
+      dW[x] = 0.f;
+    }
+    __syncthreads();
+  }
+
+  if (a.W_final) {
+    float* Wf = a.W_final + (int64_t)bh * dk * dv;
+    for (int x = tid; x < dk * kCols; x += kThreads) {
+      int r = x / kCols, c = x % kCols;
+      if (c < ncol) Wf[(int64_t)r * dv + j0 + c] = Wst[x];
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_ttt_linear_f32(const LinearArgs& a, cudaStream_t s) {
+  const size_t smem =
+      sizeof(float) * (2 * a.dk * kCols + 2 * kTB * a.dk + 2 * kTB * kCols + kTB * kTB + kTB);
+  cudaError_t e = cudaFuncSetAttribute(ttt_linear_f32_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.B * a.H, (a.dv + kCols - 1) / kCols);
+  ttt_linear_f32_kernel<<<grid, kThreads, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace ttt

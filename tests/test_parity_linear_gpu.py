@@ -1,0 +1,89 @@
+"""GPU parity of ttt_linear_fwd (C ABI) against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import ttt_oracle as O
+from linear_attention_ttt_b200 import ops, synth
+from tests.gpu_util import check, run_linear, upload_linear, max_row_rel
+
+pytestmark = pytest.mark.gpu
+
+
+def oracle_linear(w, definition=False):
+    fn = O.ttt_linear_minibatch if definition else O.ttt_linear_dual
+    return fn(w.q, w.k, w.v, w.eta, w.W0, w.chunk, w.loss)
+
+
+def test_f32_mse_full_size_workload():
+    """TTT-Linear MSE, fp32, batch 1, 2 heads, T=256, d=64, chunk 16."""
+    w = synth.config(1)
+    y, Wf = run_linear(w)
+    yo, Wo = oracle_linear(w, definition=True)
+    check(y, yo, w.dtype, "y")
+    check(Wf, Wo, w.dtype, "W_final")
+
+
+@pytest.mark.parametrize("loss", [ops.TTT_LOSS_MSE, ops.TTT_LOSS_NEG_DOT])
+@pytest.mark.parametrize("T,chunk", [(1, 16), (37, 16), (40, 1), (33, 64), (100, 7), (64, 64)])
+def test_f32_ragged_and_degenerate_chunks(loss, T, chunk):
+    w = synth.make_ttt_linear(2, 2, T, 64, 64, chunk, synth.F32, loss, seed=T * 7 + chunk,
+                              eta_kind="softplus", eta_scale=0.05)
+    y, Wf = run_linear(w)
+    yo, Wo = oracle_linear(w, definition=True)
+    check(y, yo, w.dtype, "y")
+    check(Wf, Wo, w.dtype, "W_final")
+
+
+@pytest.mark.parametrize("dk,dv", [(16, 16), (48, 80), (128, 128), (256, 256), (256, 40)])
+def test_f32_head_sizes(dk, dv):
+    w = synth.make_ttt_linear(1, 2, 45, dk, dv, 16, synth.F32, ops.TTT_LOSS_MSE, seed=dk + dv,
+                              eta_kind="softplus", eta_scale=0.05)
+    y, Wf = run_linear(w)
+    yo, Wo = oracle_linear(w)
+    check(y, yo, w.dtype, "y")
+    check(Wf, Wo, w.dtype, "W_final")
+
+
+def test_f32_per_sequence_w0_and_strided_tokens():
+    """W0 given per (batch, head), and q/k/v/out as [B,T,H,d] storage viewed
+    as [B,H,T,d] (non-contiguous strides)."""
+    w = synth.make_ttt_linear(3, 4, 50, 64, 64, 16, synth.F32, ops.TTT_LOSS_MSE, seed=5,
+                              eta_kind="sigmoid", eta_scale=0.1, w0_batched=True)
+    t = upload_linear(w)
+    for n in ("q", "k", "v"):
+        t[n] = t[n].permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3)
+    out = torch.empty((3, 50, 4, 64), device="cuda").permute(0, 2, 1, 3)
+    ops.ttt_linear_fwd(t["q"], t["k"], t["v"], t["eta"], t["W0"], 16, ops.TTT_LOSS_MSE, out=out)
+    torch.cuda.synchronize()
+    yo, _ = oracle_linear(w)
+    check(out.cpu().numpy(), yo, w.dtype, "y")
+
+
+def test_f32_empty_sequence_copies_w0():
+    w = synth.make_ttt_linear(2, 2, 0, 64, 64, 16, synth.F32, ops.TTT_LOSS_MSE, seed=1)
+    y, Wf = run_linear(w)
+    assert y.shape == (2, 2, 0, 64)
+    assert np.array_equal(Wf, np.broadcast_to(w.W0, Wf.shape))
+
+
+def test_f32_zero_learning_rate():
+    w = synth.make_ttt_linear(1, 2, 40, 64, 64, 16, synth.F32, ops.TTT_LOSS_MSE, seed=2)
+    w.eta[:] = 0
+    y, Wf = run_linear(w)
+    assert np.array_equal(Wf, np.broadcast_to(w.W0, Wf.shape))
+    assert max_row_rel(y, np.einsum("bhta,hac->bhtc", w.q.astype(np.float64), w.W0)) < 1e-5
+
+
+def test_f32_resume_from_w_final():
+    w = synth.make_ttt_linear(2, 2, 96, 64, 64, 16, synth.F32, ops.TTT_LOSS_MSE, seed=3,
+                              eta_kind="softplus", eta_scale=0.05)
+    t = upload_linear(w)
+    y, Wf = ops.ttt_linear_fwd(t["q"], t["k"], t["v"], t["eta"], t["W0"], 16, 0)
+    ya, Wa = ops.ttt_linear_fwd(t["q"][:, :, :48], t["k"][:, :, :48], t["v"][:, :, :48],
+                                t["eta"][:, :, :48], t["W0"], 16, 0)
+    yb, Wb = ops.ttt_linear_fwd(t["q"][:, :, 48:], t["k"][:, :, 48:], t["v"][:, :, 48:],
+                                t["eta"][:, :, 48:].contiguous(), Wa, 16, 0)
+    torch.cuda.synchronize()
+    assert torch.equal(torch.cat([ya, yb], dim=2), y)
+    assert torch.equal(Wb, Wf)
