@@ -1,0 +1,434 @@
+"""Benchmark of the chunked TTT-layer forward on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 2] [--impl ours|reference]
+
+A step is one forward pass of the layer over one batch of synthetic inputs
+(seeded, shaped like the pages' workloads; see linear_attention_ttt_b200.synth).
+Default workload: the inner-product-loss layer (chunked causal linear
+attention), batch 4, 16 heads, T=4096, d=128, chunk 64, bf16 tokens, fp32
+state. Workloads 1-5 can be selected with --workload.
+
+Multi-GPU: one process per GPU (torchrun). (batch, head) pairs are
+independent, so every rank runs its own replica of the workload with no
+collective on the data path (weak scaling); timing is the max over ranks.
+
+Timing: W untimed warm-up steps, then K steps between CUDA events on the
+launching stream, bracketed by a barrier and device synchronisation. Inputs
+of the default workload (q, k, v: 201 MB) exceed the 126 MB L2, so no flush is
+needed between steps; smaller workloads flush L2 by writing a 256 MB buffer
+before every step, outside the events of the kernel timing (see "l2").
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from linear_attention_ttt_b200 import ops, synth  # noqa: E402
+
+METRIC = "TTT-layer tokens/s on 1 B200; % of bf16 tensor peak or HBM GB/s roofline"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        p["_source"] = "measured"
+        return p
+    p = dict(FALLBACK_PEAKS)
+    p["_source"] = "fallback"
+    return p
+
+
+# ---------------------------------------------------------------------------
+# Workload accounting (algorithmic bytes / flops per step)
+# ---------------------------------------------------------------------------
+
+def linear_bytes(w):
+    es = 2 if w.dtype == synth.BF16 else 4
+    per_head_token = (2 * w.dk + 2 * w.dv) * es + 4        # q, k, v in, y out, eta
+    state = w.dk * w.dv * 4 * 2                             # W0 read + W_final write
+    return w.B * w.H * (w.T * per_head_token + state)
+
+
+def linear_flops(w):
+    # qW, kW and K^T(NE) at 2 dk dv each (MSE) or qW and K^T(NV) (inner
+    # product), plus the causal half of the intra-chunk products.
+    n_w = 3 if w.loss == synth.LOSS_MSE else 2
+    intra = (w.chunk + 1) * (w.dk + w.dv)
+    return w.B * w.H * w.T * (n_w * 2 * w.dk * w.dv + intra)
+
+
+def lact_flops(w):
+    per_tok = 18 * w.dk * w.dh  # apply 6 d dh, key fwd 4 d dh, backprop 8 d dh (d = dk = dv)
+    f = w.B * w.H * w.T * per_tok
+    if w.update_rule == synth.UPDATE_MUON:
+        nchunks = (w.T + w.chunk - 1) // w.chunk
+        m, n = max(w.dh, w.dk), min(w.dh, w.dk)
+        ns = 5 * (2 * 2 * m * n * n + 2 * n ** 3)
+        f += w.B * w.H * nchunks * 3 * ns
+    return f
+
+
+def lact_bytes(w):
+    es = 2 if w.dtype == synth.BF16 else 4
+    return w.B * w.H * w.T * (4 * w.dk * es + 4)
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling during the timed region (NVML, falling back to nvidia-smi)
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append(mhz)
+                for bit, name in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                return
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# Runners
+# ---------------------------------------------------------------------------
+
+def upload(w, device):
+    def t(x, dtype):
+        a = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+        a = a.to(device)
+        return a.to(torch.bfloat16) if dtype == synth.BF16 else a
+    d = {"q": t(w.q, w.dtype), "k": t(w.k, w.dtype), "v": t(w.v, w.dtype),
+         "eta": t(w.eta, synth.F32)}
+    if w.variant == "lact":
+        d.update(W1=t(w.W1, synth.F32), W2=t(w.W2, synth.F32), W3=t(w.W3, synth.F32))
+    else:
+        d["W0"] = t(w.W0, synth.F32)
+    return d
+
+
+class Step:
+    """One forward of the layer on resident device tensors (outputs preallocated)."""
+
+    def __init__(self, w, d):
+        self.w, self.d = w, d
+        dt = d["q"].dtype
+        self.out = torch.empty((w.B, w.H, w.T, w.dv), dtype=dt, device=d["q"].device)
+        if w.variant == "lact":
+            self.launches = None
+        else:
+            self.Wf = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=d["q"].device)
+            self.launches = 1
+
+    def __call__(self):
+        w, d = self.w, self.d
+        if w.variant == "lact":
+            ops.lact_swiglu_fwd(d["q"], d["k"], d["v"], d["eta"], d["W1"], d["W2"], d["W3"],
+                                w.chunk, w.update_rule, w.causal, out=self.out)
+        else:
+            ops.ttt_linear_fwd(d["q"], d["k"], d["v"], d["eta"], d["W0"], w.chunk, w.loss,
+                               out=self.out, W_final=self.Wf)
+
+
+def source_sha(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel_key, sha):
+    """DRAM bytes per launch from a committed ncu capture, if taken on this
+    exact kernel source (profiles/traffic.json)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(kernel_key)
+    if not rec or rec.get("source_sha") != sha:
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+KERNEL_SOURCES = {
+    "ttt_linear_bf16": ["linear_attention_ttt_b200/csrc/ttt_linear_bf16.cu",
+                        "linear_attention_ttt_b200/csrc/common.cuh",
+                        "linear_attention_ttt_b200/csrc/tma.cuh"],
+    "ttt_linear_f32": ["linear_attention_ttt_b200/csrc/ttt_linear_f32.cu",
+                       "linear_attention_ttt_b200/csrc/common.cuh"],
+}
+
+
+def kernel_key(w):
+    if w.variant == "lact":
+        return "lact"
+    return "ttt_linear_bf16" if w.dtype == synth.BF16 else "ttt_linear_f32"
+
+
+def cpu_oracle_step(w, sample_heads):
+    """Runs the fp64 oracle on the first `sample_heads` (batch, head)
+    sequences of the workload (all of them for sample_heads >= B*H); returns
+    (seconds, tokens) with tokens counted in the metric's unit (batch rows x T:
+    one (batch, head) sequence is 1/H of a batch row)."""
+    from oracle import ttt_oracle as O
+    n = min(sample_heads, w.B * w.H)
+    nb, nh = (n // w.H, w.H) if n >= w.H else (1, n)
+    sl = (slice(0, nb), slice(0, nh))
+    t0 = time.perf_counter()
+    if w.variant == "lact":
+        O.lact_swiglu(w.q[sl], w.k[sl], w.v[sl], w.eta[sl], w.W1[:nh], w.W2[:nh], w.W3[:nh],
+                      w.chunk, w.update_rule, w.causal)
+    else:
+        W0 = w.W0[:nh] if w.W0.ndim == 3 else w.W0[sl]
+        O.ttt_linear_dual(w.q[sl], w.k[sl], w.v[sl], w.eta[sl], W0, w.chunk, w.loss)
+    dt = time.perf_counter() - t0
+    return dt, w.T * nb * nh / w.H
+
+
+def cpu_sample_heads(w):
+    """All sequences for TTT-Linear workloads (a few seconds of fp64 work);
+    two sequences for LaCT (each costs tens of GFLOP in fp64)."""
+    return w.B * w.H if w.variant != "lact" else 2
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", type=int, default=2)
+    ap.add_argument("--chunk", type=int, default=None)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    w = synth.config(args.workload, chunk=args.chunk)
+    tokens_per_step = w.B * w.T
+    base_cfg = {"workload": w.name, "batch": w.B, "heads": w.H, "seq_len": w.T, "dk": w.dk,
+                "dv": w.dv, "chunk": w.chunk, "variant": w.variant,
+                "loss": ("mse" if w.loss == 0 else "neg_dot") if w.variant != "lact" else "neg_dot_swiglu",
+                "parallelism": f"replicas{world}"}
+    if w.variant == "lact":
+        base_cfg.update(dh=w.dh, update_rule="muon" if w.update_rule else "gd",
+                        causal=w.causal)
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        steps = []
+        sample_heads = max(1, cpu_sample_heads(w) // 4)
+        for i in range(args.warmup + args.steps):
+            dt, toks = cpu_oracle_step(w, sample_heads)
+            if i >= args.warmup:
+                steps.append(toks / dt)
+        v = float(statistics.median(steps))
+        sample = f"fp64 numpy oracle on {sample_heads} (batch, head) sequence(s) of the workload per step"
+        line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
+                "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
+                "higher_is_better": True, "dtype": "f64", "data": "synthetic",
+                "config": base_cfg,
+                "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": blas_threads(),
+                                 "kind": "oracle", "sample": sample},
+                "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    device = torch.device("cuda", torch.cuda.current_device())
+    ops.load()
+
+    d = upload(w, device)
+    step = Step(w, d)
+    in_bytes = sum(x.numel() * x.element_size() for x in d.values())
+    l2_flush = in_bytes < 2 * L2_BYTES
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device) if l2_flush else None
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- device-resident timing (whole step == the kernel launches) ----
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(device.index if world == 1 else local)
+    with sampler:
+        t_wall = time.perf_counter()
+        for i in range(args.steps):
+            if flush is not None:
+                flush.zero_()
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        t_wall = time.perf_counter() - t_wall
+    barrier()
+    per = [a.elapsed_time(b) for a, b in ev]
+    total_ms = float(sum(per))
+    if dist is not None:
+        tt = torch.tensor([total_ms], device=device)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    ms_per_step = total_ms / args.steps
+    value = tokens_per_step * world / (ms_per_step / 1e3)
+
+    # ---- end to end through the public API with host buffers ----
+    host = {k: v.to("cpu").pin_memory() for k, v in d.items()}
+    host_out = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = host_out.numel() * host_out.element_size()
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        for k2, v2 in host.items():
+            d[k2].copy_(v2, non_blocking=True)
+        step()
+        host_out.copy_(step.out, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(e2e_steps):
+        for k2, v2 in host.items():
+            d[k2].copy_(v2, non_blocking=True)
+        step()
+        host_out.copy_(step.out, non_blocking=True)
+    b.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = a.elapsed_time(b) / e2e_steps
+    if dist is not None:
+        tt = torch.tensor([e2e_ms], device=device)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    e2e_value = tokens_per_step * world / (e2e_ms / 1e3)
+
+    pk = peaks()
+    key = kernel_key(w)
+    if w.variant == "lact":
+        flops = lact_flops(w)
+        peak = pk["bf16_tflops_sustained"] if "bf16_tflops_sustained" in pk else pk["bf16_tflops"]
+        achieved = flops / (ms_per_step / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None,
+                "peak_source": pk["_source"] + " bf16 (sustained)", "kernel": "lact step"}
+    else:
+        byts = linear_bytes(w)
+        launch_ms = ms_per_step  # one launch per step
+        achieved = byts / (launch_ms / 1e3) / 1e9
+        sha = source_sha(KERNEL_SOURCES[key])
+        roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / pk["hbm_gbs"], "traffic": recorded_traffic(key, sha),
+                "peak_source": pk["_source"] + " hbm_gbs", "kernel": key,
+                "algorithmic_bytes_per_launch": byts, "kernel_source_sha": sha}
+
+    cfg = dict(base_cfg)
+    cfg["l2"] = ("flushed (256 MB write) before every timed step" if l2_flush
+                 else f"inputs {in_bytes / 1e6:.0f} MB > L2 126 MB, no flush")
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == synth.BF16 else "f32", "data": "synthetic",
+            "config": cfg, "roofline": roof,
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d * world,
+                    "d2h_bytes_per_step": d2h * world},
+            "gpu_launches": (step.launches or 0) * args.steps,
+            "clocks": sampler.summary(), "wall_s_timed": t_wall}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n = cpu_sample_heads(w)
+        dt, toks = cpu_oracle_step(w, n)
+        line["cpu_baseline"] = {"value": toks / dt, "unit": "tokens/s", "cores": blas_threads(),
+                                "kind": "oracle",
+                                "sample": f"fp64 numpy oracle (dual form / LaCT scan) on {n} of "
+                                          f"{w.B * w.H} (batch, head) sequences, {dt:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

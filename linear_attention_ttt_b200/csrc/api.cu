@@ -67,6 +67,7 @@ ttt_status check_tokens(const ttt_tensor* t, int64_t B, int64_t H, int64_t T, in
   if (t->shape[0] != B || t->shape[1] != H || t->shape[2] != T || t->shape[3] != d)
     return TTT_ERR_SHAPE;
   if (t->dtype != dtype) return TTT_ERR_DTYPE;
+  if (B * H * T * d == 0) return TTT_OK;  // no elements: strides are irrelevant
   if (t->stride[3] != 1 && d > 1) return TTT_ERR_LAYOUT;
   const int64_t es = (int64_t)elem_size(dtype);
   for (int i = 0; i < 3; ++i) {
@@ -139,7 +140,7 @@ ttt_status ttt_linear_fwd(const ttt_tensor* q, const ttt_tensor* k, const ttt_te
   if (eta->dtype != TTT_F32) return TTT_ERR_DTYPE;
   if (!eta->data && T > 0) return TTT_ERR_NULL;
   for (int i = 0; i < 3; ++i)
-    if (eta->stride[i] < 0) return TTT_ERR_LAYOUT;
+    if (eta->stride[i] < 0 && T > 0) return TTT_ERR_LAYOUT;
   if (!aligned16(eta->data)) return TTT_ERR_LAYOUT;
   // W0 [H,dk,dv] or [B,H,dk,dv] fp32 contiguous
   if (!W0->data) return TTT_ERR_NULL;
@@ -189,7 +190,7 @@ ttt_status ttt_linear_fwd(const ttt_tensor* q, const ttt_tensor* k, const ttt_te
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   cudaError_t e;
-  if (dt == TTT_F32) {
+  if (dt == TTT_F32 || T == 0) {  // T == 0 only copies W0 to W_final
     e = ttt::launch_ttt_linear_f32(a, s);
   } else {
     bool supported = false;

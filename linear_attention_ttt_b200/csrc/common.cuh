@@ -12,9 +12,15 @@ namespace ttt {
 // Error codes a kernel can record in the device status word.
 enum : int { DEV_OK = 0, DEV_TIMEOUT = 1, DEV_BAD_ARGS = 2 };
 
-// Upper bound on polls of one barrier before a kernel gives up (far above any
-// legitimate wait: a poll is tens of ns, so this is on the order of seconds).
-constexpr uint32_t kMaxPolls = 1u << 26;
+// A wait on one barrier gives up after this many nanoseconds of %globaltimer
+// (legitimate waits in these kernels last microseconds).
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
 
 __device__ __forceinline__ void record_error(int* status, int code) {
   if (status) atomicCAS(status, DEV_OK, code);
@@ -72,11 +78,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait: returns false (and records DEV_TIMEOUT) if the phase never
-// completes within kMaxPolls polls.
+// Bounded wait: returns false (and records DEV_TIMEOUT) if the phase has not
+// completed within kWaitLimitNs.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
-  for (uint32_t i = 0; i < kMaxPolls; ++i)
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 255) == 0 && global_ns() - t0 > kWaitLimitNs) break;
+  }
   record_error(status, DEV_TIMEOUT);
   return false;
 }

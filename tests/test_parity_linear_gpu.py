@@ -87,3 +87,80 @@ def test_f32_resume_from_w_final():
     torch.cuda.synchronize()
     assert torch.equal(torch.cat([ya, yb], dim=2), y)
     assert torch.equal(Wb, Wf)
+
+
+# ---------------------------------------------------------------------------
+# bf16 tokens, fp32 state
+# ---------------------------------------------------------------------------
+
+def test_bf16_linear_attention_full_size_workload():
+    """Inner-product loss (chunked causal linear attention): batch 4, 16
+    heads, T=4096, d=128, chunk 64, bf16, W0=0, eta=0.1*sigmoid(N(0,1))."""
+    w = synth.config(2)
+    y, Wf = run_linear(w)
+    yo, Wo = oracle_linear(w)
+    check(y, yo, w.dtype, "y")
+    check(Wf, Wo, w.dtype, "W_final")
+
+
+@pytest.mark.parametrize("chunk", [16, 256])
+def test_bf16_mse_full_size_workload(chunk):
+    """TTT-Linear MSE: batch 8, 16 heads, T=8192, d=64, bf16, chunk 16/256."""
+    w = synth.config(3, chunk=chunk)
+    y, Wf = run_linear(w)
+    yo, Wo = oracle_linear(w)
+    check(y, yo, w.dtype, "y")
+    check(Wf, Wo, w.dtype, "W_final")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("loss", [ops.TTT_LOSS_MSE, ops.TTT_LOSS_NEG_DOT])
+@pytest.mark.parametrize("T,chunk", [(1, 16), (37, 16), (300, 64), (100, 5), (70, 24), (64, 256)])
+def test_bf16_ragged_and_odd_chunks(d, loss, T, chunk):
+    w = synth.make_ttt_linear(2, 3, T, d, d, chunk, synth.BF16, loss, seed=T + chunk + d,
+                              eta_kind="softplus", eta_scale=0.05)
+    y, Wf = run_linear(w)
+    yo, Wo = oracle_linear(w, definition=True)
+    check(y, yo, w.dtype, "y")
+    check(Wf, Wo, w.dtype, "W_final")
+
+
+def test_bf16_per_sequence_w0_strided_tokens_and_empty():
+    w = synth.make_ttt_linear(2, 3, 80, 64, 64, 16, synth.BF16, ops.TTT_LOSS_MSE, seed=11,
+                              eta_kind="softplus", eta_scale=0.05, w0_batched=True)
+    t = upload_linear(w)
+    for n in ("q", "k", "v"):
+        t[n] = t[n].permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3)
+    out = torch.empty((2, 80, 3, 64), device="cuda", dtype=torch.bfloat16).permute(0, 2, 1, 3)
+    _, Wf = ops.ttt_linear_fwd(t["q"], t["k"], t["v"], t["eta"], t["W0"], 16, 0, out=out)
+    torch.cuda.synchronize()
+    yo, Wo = oracle_linear(w)
+    check(out.float().cpu().numpy(), yo, w.dtype, "y")
+    check(Wf.cpu().numpy(), Wo, w.dtype, "W_final")
+    e = synth.make_ttt_linear(1, 2, 0, 128, 128, 64, synth.BF16, ops.TTT_LOSS_NEG_DOT, seed=1)
+    y, Wf = run_linear(e)
+    assert np.array_equal(Wf, np.broadcast_to(e.W0, Wf.shape))
+
+
+@pytest.mark.parametrize("loss", [ops.TTT_LOSS_MSE, ops.TTT_LOSS_NEG_DOT])
+def test_bf16_resume_from_w_final_is_bit_exact(loss):
+    w = synth.make_ttt_linear(2, 2, 256, 64, 64, 32, synth.BF16, loss, seed=4,
+                              eta_kind="softplus", eta_scale=0.05)
+    t = upload_linear(w)
+    y, Wf = ops.ttt_linear_fwd(t["q"], t["k"], t["v"], t["eta"], t["W0"], 32, loss)
+    sl = lambda x, a, b: x[:, :, a:b]
+    ya, Wa = ops.ttt_linear_fwd(sl(t["q"], 0, 96), sl(t["k"], 0, 96), sl(t["v"], 0, 96),
+                                sl(t["eta"], 0, 96), t["W0"], 32, loss)
+    yb, Wb = ops.ttt_linear_fwd(sl(t["q"], 96, 256), sl(t["k"], 96, 256), sl(t["v"], 96, 256),
+                                sl(t["eta"], 96, 256), Wa, 32, loss)
+    torch.cuda.synchronize()
+    assert torch.equal(torch.cat([ya, yb], dim=2), y)
+    assert torch.equal(Wb, Wf)
+
+
+def test_bf16_unsupported_head_size_is_rejected():
+    w = synth.make_ttt_linear(1, 1, 16, 32, 32, 16, synth.BF16, 0, seed=1)
+    t = upload_linear(w)
+    with pytest.raises(ops.TTTError) as e:
+        ops.ttt_linear_fwd(t["q"], t["k"], t["v"], t["eta"], t["W0"], 16, 0)
+    assert e.value.code == -5
