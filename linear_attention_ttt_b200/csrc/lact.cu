@@ -1,8 +1,643 @@
-// LaCT SwiGLU fast-weight layer forward (placeholder until the kernels land).
+// LaCT SwiGLU fast-weight layer forward ("Test-Time Training Done Right"
+// review, sections 3.2-3.3 and 4 / Figure 3).
+//
+// Per (batch, head) z the fast weights W1, W3 [dh][dk] and W2 [dv][dh] live
+// in fp32 master copies in scratch memory, with bf16 operand copies refreshed
+// after every update (W1 and W3 rows interleaved in blocks of 64 into W13 so
+// one 128-column tile holds matching h1/h3 columns). One chunk step, all heads
+// at once (causal order: apply with the weights before the chunk, then
+// update):
+//   L1  Gz = -eta (V W2)                     [b x dh] fp32
+//       Aq = silu(Q W1^T) * (Q W3^T)         [b x dh] bf16          (causal)
+//   L2  from H = K [W1;W3]^T:  Ak' = eta silu(H1) H3, dH3 = Gz silu(H1),
+//       dH1 = Gz H3 silu'(H1)                [b x dh] bf16
+//       Y  = Aq W2^T -> layer output         [b x dv]               (causal)
+//   L3  G1 = dH1^T K, G3 = dH3^T K           [dh x dk] fp32 (split-K, atomics)
+//       G2 = -V^T Ak'                        [dv x dh]
+//   L4  Muon: G <- NS5(G) (fp32, CUDA cores)
+//   L5  W <- W - G; each row rescaled to its initial L2 norm; bf16 copies.
+// Non-causal (update, then apply): L1 without Aq, L2 without Y, L3, L4, L5,
+// then Aq and Y with the updated weights.
+// Precision: GD uses bf16 operands with fp32 accumulation; Muon uses
+// split-bf16 operands (x = hi + lo, products hi*hi + lo*hi + hi*lo) because
+// the unit-step Muon scan amplifies per-chunk rounding across chunks.
+#include <vector>
+
+#include "gemm_tc.cuh"
 #include "lact.cuh"
 
 namespace ttt {
+namespace {
 
-ttt_status lact_forward(const LactArgs&, cudaStream_t) { return TTT_ERR_UNSUPPORTED; }
+using gemm::Operand;
+using gemm::Params;
+using gemm::Problem;
+
+constexpr int BN = 128;
+
+// ---------------------------------------------------------------------------
+// Row kernels: prepare / update / renormalise the fast weights
+// ---------------------------------------------------------------------------
+
+struct RowArgs {
+  float* Wm[3];            // masters: W1 [Z][dh][dk], W3 [Z][dh][dk], W2 [Z][dv][dh]
+  const float* Win[3];     // inputs (prep only), per-head or per-(batch, head)
+  int64_t win_sz[3];       // non-zero when the input holds one matrix per (batch, head)
+  float* rho[3];           // initial row norms [Z][rows]
+  float* G[3];             // gradients (update input; zeroed after use)
+  __nv_bfloat16 *w13_hi, *w13_lo, *w2_hi, *w2_lo;
+  int Z, H, dk, dv, dh;
+  int prep;                // 1: copy inputs and record norms; 0: W -= G then renorm
+  int split;
+};
+
+// One warp per (z, row of W1 | W3 | W2).
+__global__ void __launch_bounds__(256) lact_rows_kernel(RowArgs a) {
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  const int rows_z = 2 * a.dh + a.dv;
+  if (gw >= a.Z * rows_z) return;
+  const int z = gw / rows_z;
+  int r = gw % rows_z, m;
+  if (r < a.dh) {
+    m = 0;
+  } else if (r < 2 * a.dh) {
+    m = 1;
+    r -= a.dh;
+  } else {
+    m = 2;
+    r -= 2 * a.dh;
+  }
+  const int len = (m == 2) ? a.dh : a.dk;
+  const int nrows = (m == 2) ? a.dv : a.dh;
+  float* W = a.Wm[m] + ((int64_t)z * nrows + r) * len;
+  float* G = a.G[m] + ((int64_t)z * nrows + r) * len;
+  float v[32];
+  float ss = 0.f;
+  const int per = len / 32;  // len is a multiple of 32
+  if (a.prep) {
+    const int zin = a.win_sz[m] ? z : z % a.H;
+    const float* src = a.Win[m] + ((int64_t)zin * nrows + r) * len;
+    for (int i = 0; i < per; ++i) {
+      v[i] = src[lane + 32 * i];
+      ss += v[i] * v[i];
+    }
+  } else {
+    for (int i = 0; i < per; ++i) {
+      v[i] = W[lane + 32 * i] - G[lane + 32 * i];
+      ss += v[i] * v[i];
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float nrm = sqrtf(ss);
+  float* rho = a.rho[m] + (int64_t)z * nrows + r;
+  if (a.prep) {
+    if (lane == 0) *rho = nrm;
+  } else {
+    const float target = *rho;
+    const float s = nrm > 0.f ? target / nrm : 1.f;
+    for (int i = 0; i < per; ++i) v[i] *= s;
+  }
+  __nv_bfloat16 *hi, *lo;
+  int64_t orow;
+  if (m == 2) {
+    hi = a.w2_hi;
+    lo = a.w2_lo;
+    orow = (int64_t)z * a.dv + r;
+  } else {
+    hi = a.w13_hi;
+    lo = a.w13_lo;
+    orow = (int64_t)z * 2 * a.dh + (r / 64) * 128 + (m == 1 ? 64 : 0) + (r % 64);
+  }
+  for (int i = 0; i < per; ++i) {
+    const int c = lane + 32 * i;
+    W[c] = v[i];
+    G[c] = 0.f;
+    const __nv_bfloat16 h = __float2bfloat16_rn(v[i]);
+    hi[orow * len + c] = h;
+    if (a.split) lo[orow * len + c] = __float2bfloat16_rn(v[i] - __bfloat162float(h));
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Newton-Schulz (Muon) on the CUDA cores, fp32: one CTA per gradient matrix.
+// ---------------------------------------------------------------------------
+
+struct NsArgs {
+  float* G[3];   // in/out, [Z][rows][cols] row-major
+  int rows[3], cols[3];
+  float* scratch;  // per (z, m): gram [s*s], poly [s*s], xn [rows*cols]
+  int64_t scratch_stride;
+  float a, b, c, eps;
+  int steps;
+};
+
+constexpr int kNsThreads = 1024;
+constexpr int kTile = 32;
+
+// C[M x N] = alpha * op(A) op(B) + beta * Cin, all row-major in global memory
+// (L2-resident scratch). op(A) is A or A^T (tA), same for B. Computed by the
+// whole CTA with 32x32 shared-memory tiles.
+__device__ void cta_gemm(float* C, const float* Cin, const float* A, const float* B, int M, int N,
+                         int K, bool tA, bool tB, int lda, int ldb, float alpha, float beta) {
+  __shared__ float As[kTile][kTile + 1], Bs[kTile][kTile + 1];
+  const int tx = threadIdx.x % kTile, ty = threadIdx.x / kTile;  // 32 x 32 threads
+  for (int i0 = 0; i0 < M; i0 += kTile)
+    for (int j0 = 0; j0 < N; j0 += kTile) {
+      float acc = 0.f;
+      for (int k0 = 0; k0 < K; k0 += kTile) {
+        // A tile: rows i0+ty, cols k0+tx of op(A)
+        {
+          const int i = i0 + ty, k = k0 + tx;
+          As[ty][tx] = (i < M && k < K) ? (tA ? A[(int64_t)k * lda + i] : A[(int64_t)i * lda + k]) : 0.f;
+        }
+        {
+          const int k = k0 + ty, j = j0 + tx;
+          Bs[ty][tx] = (k < K && j < N) ? (tB ? B[(int64_t)j * ldb + k] : B[(int64_t)k * ldb + j]) : 0.f;
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int kk = 0; kk < kTile; ++kk) acc = fmaf(As[ty][kk], Bs[kk][tx], acc);
+        __syncthreads();
+      }
+      const int i = i0 + ty, j = j0 + tx;
+      if (i < M && j < N) {
+        const float prev = (beta != 0.f) ? Cin[(int64_t)i * N + j] : 0.f;
+        C[(int64_t)i * N + j] = alpha * acc + beta * prev;
+      }
+    }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kNsThreads) ns_kernel(NsArgs a) {
+  const int z = blockIdx.x / 3, m = blockIdx.x % 3;
+  const int R = a.rows[m], C = a.cols[m];
+  float* X = a.G[m] + (int64_t)z * R * C;
+  const int s = min(R, C);
+  float* gram = a.scratch + (int64_t)blockIdx.x * a.scratch_stride;
+  float* poly = gram + (int64_t)s * s;
+  float* xn = poly + (int64_t)s * s;
+  __shared__ float red[32];
+  float ss = 0.f;
+  for (int64_t i = threadIdx.x; i < (int64_t)R * C; i += blockDim.x) ss += X[i] * X[i];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float t = red[threadIdx.x];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    if (threadIdx.x == 0) red[0] = t;
+  }
+  __syncthreads();
+  const float inv = 1.f / (sqrtf(red[0]) + a.eps);
+  for (int64_t i = threadIdx.x; i < (int64_t)R * C; i += blockDim.x) X[i] *= inv;
+  __syncthreads();
+  const bool tall = R >= C;
+  for (int it = 0; it < a.steps; ++it) {
+    // gram: tall -> X^T X (C x C); wide -> X X^T (R x R)
+    if (tall)
+      cta_gemm(gram, nullptr, X, X, s, s, R, true, false, C, C, 1.f, 0.f);
+    else
+      cta_gemm(gram, nullptr, X, X, s, s, C, false, true, C, C, 1.f, 0.f);
+    // poly = c * gram @ gram + b * gram
+    cta_gemm(poly, gram, gram, gram, s, s, s, false, false, s, s, a.c, a.b);
+    // xn = X poly (tall) or poly X (wide); X = a X + xn
+    if (tall)
+      cta_gemm(xn, X, X, poly, R, C, C, false, false, C, C, 1.f, a.a);
+    else
+      cta_gemm(xn, X, poly, X, R, C, R, false, false, R, C, 1.f, a.a);
+    for (int64_t i = threadIdx.x; i < (int64_t)R * C; i += blockDim.x) X[i] = xn[i];
+    __syncthreads();
+  }
+}
+
+__global__ void copy_kernel(float* dst, const float* src, int64_t n) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x)
+    dst[i] = src[i];
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+
+bool map_tokens(CUtensorMap* m, const TokView& v, int B, int H, int T, int d, int box_inner,
+                int box_rows) {
+  TokView x = v;
+  if (B == 1) x.sb = (int64_t)H * T * d;
+  if (H == 1) x.sh = (int64_t)T * d;
+  if (T == 1) x.st = d;
+  uint64_t dims[4] = {(uint64_t)d, (uint64_t)T, (uint64_t)H, (uint64_t)B};
+  uint64_t strides[3] = {(uint64_t)x.st * 2, (uint64_t)x.sh * 2, (uint64_t)x.sb * 2};
+  uint32_t box[4] = {(uint32_t)box_inner, (uint32_t)box_rows, 1, 1};
+  return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, x.p, dims, strides, box,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// [Z][rows_alloc][cols] bf16 buffer as a 4-d map {cols, rows, Z, 1}; only the
+// first `rows` rows of each z are visible (later rows read as zeros).
+bool map_buf(CUtensorMap* m, const void* base, int Z, int rows, int rows_alloc, int cols,
+             int box_inner, int box_rows) {
+  uint64_t dims[4] = {(uint64_t)cols, (uint64_t)rows, (uint64_t)Z, 1};
+  uint64_t strides[3] = {(uint64_t)cols * 2, (uint64_t)cols * 2 * rows_alloc,
+                         (uint64_t)cols * 2 * rows_alloc * Z};
+  uint32_t box[4] = {(uint32_t)box_inner, (uint32_t)box_rows, 1, 1};
+  return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+struct Scratch {
+  float *Wm[3], *rho[3], *G[3], *gz, *ns;
+  __nv_bfloat16 *w13[2], *w2[2];          // hi, lo
+  __nv_bfloat16 *aq[2], *ak[2], *dh1[2], *dh3[2];
+  int64_t ns_stride;
+};
+
+void fill_problem_tiles(Params& P) {
+  int t = 0;
+  for (int i = 0; i < P.nprob; ++i) {
+    Problem& p = P.p[i];
+    p.mtiles = (p.M + gemm::BM - 1) / gemm::BM;
+    p.ntiles = (p.N + BN - 1) / BN;
+    p.tile_begin = t;
+    t += p.nz * p.ksplit * p.mtiles * p.ntiles;
+  }
+  P.total_tiles = t;
+}
+
+cudaError_t launch_gemm(Params& P, cudaStream_t s) {
+  fill_problem_tiles(P);
+  if (P.total_tiles == 0) return cudaSuccess;
+  const size_t smem = sizeof(gemm::Smem<BN>) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(gemm::gemm_kernel<BN>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  gemm::gemm_kernel<BN><<<P.total_tiles, gemm::kThreads, smem, s>>>(P);
+  return cudaGetLastError();
+}
+
+// Operand helpers -----------------------------------------------------------
+// K-major token operand (rows = tokens of the chunk): storage [T][d].
+bool tok_kmajor(Operand& o, const TokView& v, const LactArgs& a, int d, int row0, int box_rows) {
+  o.mn_major = 0;
+  o.row0 = row0;
+  o.zdiv = a.H;
+  return map_tokens(&o.map[0], v, a.B, a.H, a.T, d, 64, box_rows) &&
+         map_tokens(&o.map[1], v, a.B, a.H, a.T, d, 64, box_rows);
+}
+// MN-major token operand (tokens = K dimension): storage [T][d], d = M or N.
+bool tok_mnmajor(Operand& o, const TokView& v, const LactArgs& a, int d, int row0) {
+  o.mn_major = 1;
+  o.row0 = row0;
+  o.zdiv = a.H;
+  return map_tokens(&o.map[0], v, a.B, a.H, a.T, d, 64, 64) &&
+         map_tokens(&o.map[1], v, a.B, a.H, a.T, d, 64, 64);
+}
+bool buf_op(Operand& o, __nv_bfloat16* const* hl, int Z, int rows, int rows_alloc, int cols,
+            int mn_major, int box_rows, bool split) {
+  o.mn_major = mn_major;
+  o.row0 = 0;
+  o.zdiv = Z;
+  const int br = mn_major ? 64 : box_rows;
+  return map_buf(&o.map[0], hl[0], Z, rows, rows_alloc, cols, 64, br) &&
+         map_buf(&o.map[1], split ? hl[1] : hl[0], Z, rows, rows_alloc, cols, 64, br);
+}
+
+void segs(Problem& p, int n, const int (*ab)[2]) {
+  p.nseg = n;
+  for (int i = 0; i < n; ++i) {
+    p.seg_a[i] = ab[i][0];
+    p.seg_b[i] = ab[i][1];
+  }
+}
+const int kSegExact[1][2] = {{0, 0}};
+const int kSegBsplit[2][2] = {{0, 0}, {0, 1}};
+const int kSegAsplit[2][2] = {{0, 0}, {1, 0}};
+const int kSegBoth[3][2] = {{0, 0}, {1, 0}, {0, 1}};
+
+gemm::EpiArgs epi_base(const LactArgs& a, int s0, int rows_valid) {
+  gemm::EpiArgs e;
+  memset(&e, 0, sizeof(e));
+  e.eta = a.eta;
+  e.eta_t0 = s0;
+  e.H = a.H;
+  e.out = a.out;
+  e.out_bf16 = a.dtype == TTT_BF16;
+  e.rows_valid = rows_valid;
+  e.scale = 1.f;
+  return e;
+}
+
+int pick_ksplit(int kblocks, int tiles) {
+  int ks = 1;
+  while (ks < kblocks && tiles * ks < 4 * 148) ks *= 2;
+  return ks < 1 ? 1 : (ks > kblocks ? kblocks : ks);
+}
+
+}  // namespace
+
+ttt_status lact_forward(const LactArgs& a, cudaStream_t s) {
+  if (a.dtype != TTT_BF16) return TTT_ERR_UNSUPPORTED;
+  if (a.dk != a.dv || (a.dk != 64 && a.dk != 128 && a.dk != 256)) return TTT_ERR_UNSUPPORTED;
+  if (a.dh % 128 != 0 || a.dh > 1024) return TTT_ERR_UNSUPPORTED;
+  const int Z = a.B * a.H, dk = a.dk, dv = a.dv, dh = a.dh;
+  const int chunk = a.T > 0 ? (a.chunk < a.T ? a.chunk : a.T) : 1;
+  const bool split = a.update_rule == LACT_UPDATE_MUON;
+
+  // ---- scratch (stream-ordered) ----
+  const int64_t nW[3] = {(int64_t)dh * dk, (int64_t)dh * dk, (int64_t)dv * dh};
+  const int64_t nrows[3] = {dh, dh, dv};
+  const int s_max = dk < dh ? dk : dh;
+  const int64_t ns_stride = 2 * (int64_t)s_max * s_max + (int64_t)dh * dk;
+  size_t f32n = 0;
+  for (int m = 0; m < 3; ++m) f32n += (size_t)Z * (2 * nW[m] + nrows[m]);
+  f32n += (size_t)Z * chunk * dh;                     // gz
+  if (split) f32n += (size_t)Z * 3 * ns_stride;       // NS scratch
+  size_t bfn = (size_t)Z * (2 * dh * dk + dv * dh) * (split ? 2 : 1);
+  bfn += (size_t)Z * chunk * dh * 4 * (split ? 2 : 1);
+  const size_t bytes = f32n * 4 + bfn * 2 + 4096;
+  void* base = nullptr;
+  if (cudaMallocAsync(&base, bytes, s) != cudaSuccess) {
+    cudaGetLastError();
+    return TTT_ERR_ALLOC;
+  }
+  Scratch sc;
+  {
+    float* f = static_cast<float*>(base);
+    for (int m = 0; m < 3; ++m) {
+      sc.Wm[m] = f;
+      f += Z * nW[m];
+      sc.G[m] = f;
+      f += Z * nW[m];
+      sc.rho[m] = f;
+      f += Z * nrows[m];
+    }
+    sc.gz = f;
+    f += (size_t)Z * chunk * dh;
+    sc.ns = split ? f : nullptr;
+    if (split) f += (size_t)Z * 3 * ns_stride;
+    uintptr_t up = (reinterpret_cast<uintptr_t>(f) + 255) & ~uintptr_t(255);
+    __nv_bfloat16* b = reinterpret_cast<__nv_bfloat16*>(up);
+    auto take = [&](size_t n) {
+      __nv_bfloat16* r = b;
+      b += (n + 127) / 128 * 128;
+      return r;
+    };
+    for (int x = 0; x < (split ? 2 : 1); ++x) {
+      sc.w13[x] = take((size_t)Z * 2 * dh * dk);
+      sc.w2[x] = take((size_t)Z * dv * dh);
+      sc.aq[x] = take((size_t)Z * chunk * dh);
+      sc.ak[x] = take((size_t)Z * chunk * dh);
+      sc.dh1[x] = take((size_t)Z * chunk * dh);
+      sc.dh3[x] = take((size_t)Z * chunk * dh);
+    }
+    if (!split)
+      sc.w13[1] = sc.w13[0], sc.w2[1] = sc.w2[0], sc.aq[1] = sc.ak[1] = sc.dh1[1] = sc.dh3[1] = nullptr;
+  }
+  sc.ns_stride = ns_stride;
+
+  ttt_status result = TTT_OK;
+  auto check = [&](cudaError_t e) {
+    if (e != cudaSuccess && result == TTT_OK) result = TTT_ERR_CUDA;
+    return e == cudaSuccess;
+  };
+
+  RowArgs ra;
+  memset(&ra, 0, sizeof(ra));
+  for (int m = 0; m < 3; ++m) {
+    ra.Wm[m] = sc.Wm[m];
+    ra.rho[m] = sc.rho[m];
+    ra.G[m] = sc.G[m];
+  }
+  // row-kernel matrix order is (W1, W3, W2); LactArgs::w_sb is (W1, W2, W3)
+  ra.win_sz[0] = a.w_sb[0];
+  ra.win_sz[1] = a.w_sb[2];
+  ra.win_sz[2] = a.w_sb[1];
+  ra.Win[0] = a.W1;
+  ra.Win[1] = a.W3;
+  ra.Win[2] = a.W2;
+  ra.w13_hi = sc.w13[0];
+  ra.w13_lo = sc.w13[1];
+  ra.w2_hi = sc.w2[0];
+  ra.w2_lo = sc.w2[1];
+  ra.Z = Z;
+  ra.H = a.H;
+  ra.dk = dk;
+  ra.dv = dv;
+  ra.dh = dh;
+  ra.split = split;
+  const int row_warps = Z * (2 * dh + dv);
+  const int row_blocks = (row_warps * 32 + 255) / 256;
+  ra.prep = 1;
+  lact_rows_kernel<<<row_blocks, 256, 0, s>>>(ra);
+  check(cudaGetLastError());
+  ra.prep = 0;
+
+  NsArgs na;
+  memset(&na, 0, sizeof(na));
+  if (split) {
+    for (int m = 0; m < 3; ++m) na.G[m] = sc.G[m];
+    na.rows[0] = na.rows[1] = dh;
+    na.cols[0] = na.cols[1] = dk;
+    na.rows[2] = dv;
+    na.cols[2] = dh;
+    na.scratch = sc.ns;
+    na.scratch_stride = ns_stride;
+    na.a = 3.4445f;
+    na.b = -4.7750f;
+    na.c = 2.0315f;
+    na.eps = 1e-7f;
+    na.steps = 5;
+  }
+
+  const int* segW = split ? &kSegBsplit[0][0] : &kSegExact[0][0];
+  const int nsegW = split ? 2 : 1;
+
+  for (int s0 = 0; s0 < a.T && result == TTT_OK; s0 += chunk) {
+    const int bc = (a.T - s0) < chunk ? (a.T - s0) : chunk;
+    // shared operands for this chunk
+    Operand W13, W2mn, W2k, Qk, Kk, Vk, Kmn, Vmn, AQk, DH1mn, DH3mn, AKmn;
+    bool ok = true;
+    ok &= buf_op(W13, sc.w13, Z, 2 * dh, 2 * dh, dk, 0, BN, split);
+    ok &= buf_op(W2mn, sc.w2, Z, dv, dv, dh, 1, 64, split);
+    ok &= buf_op(W2k, sc.w2, Z, dv, dv, dh, 0, BN, split);
+    ok &= tok_kmajor(Qk, a.q, a, dk, s0, gemm::BM);
+    ok &= tok_kmajor(Kk, a.k, a, dk, s0, gemm::BM);
+    ok &= tok_kmajor(Vk, a.v, a, dv, s0, gemm::BM);
+    ok &= tok_mnmajor(Kmn, a.k, a, dk, s0);
+    ok &= tok_mnmajor(Vmn, a.v, a, dv, s0);
+    ok &= buf_op(AQk, sc.aq, Z, bc, chunk, dh, 0, gemm::BM, split);
+    ok &= buf_op(DH1mn, sc.dh1, Z, bc, chunk, dh, 1, 64, split);
+    ok &= buf_op(DH3mn, sc.dh3, Z, bc, chunk, dh, 1, 64, split);
+    ok &= buf_op(AKmn, sc.ak, Z, bc, chunk, dh, 1, 64, split);
+    if (!ok) {
+      result = TTT_ERR_CUDA;
+      break;
+    }
+    auto add_apply = [&](Params& P, int stage) {
+      // stage 0: Aq from Q; stage 1: Y from Aq
+      Problem& p = P.p[P.nprob++];
+      memset(&p, 0, sizeof(p));
+      p.nz = Z;
+      p.ksplit = 1;
+      if (stage == 0) {
+        p.a = Qk;
+        p.b = W13;
+        p.M = bc;
+        p.N = 2 * dh;
+        p.K = dk;
+        segs(p, nsegW, reinterpret_cast<const int(*)[2]>(segW));
+        p.epi = gemm::EPI_AQ;
+        p.e = epi_base(a, s0, bc);
+        p.e.bo[0] = sc.aq[0];
+        p.e.bo_lo[0] = split ? sc.aq[1] : nullptr;
+        p.e.b_sz = (int64_t)chunk * dh;
+        p.e.b_sr = dh;
+      } else {
+        p.a = AQk;
+        p.b = W2k;
+        p.M = bc;
+        p.N = dv;
+        p.K = dh;
+        if (split)
+          segs(p, 3, kSegBoth);
+        else
+          segs(p, 1, kSegExact);
+        p.epi = gemm::EPI_Y;
+        p.e = epi_base(a, s0, bc);
+      }
+    };
+
+    // L1: Gz (+ Aq when causal)
+    {
+      Params P;
+      memset(&P, 0, sizeof(P));
+      P.status = a.status;
+      Problem& p = P.p[P.nprob++];
+      p.a = Vk;
+      p.b = W2mn;
+      p.M = bc;
+      p.N = dh;
+      p.K = dv;
+      p.nz = Z;
+      p.ksplit = 1;
+      segs(p, nsegW, reinterpret_cast<const int(*)[2]>(segW));
+      p.epi = gemm::EPI_GZ;
+      p.e = epi_base(a, s0, bc);
+      p.e.f32 = sc.gz;
+      p.e.f32_sz = (int64_t)chunk * dh;
+      p.e.f32_sr = dh;
+      if (a.causal) add_apply(P, 0);
+      check(launch_gemm(P, s));
+    }
+    // L2: key forward + backprop epilogue (+ Y when causal)
+    {
+      Params P;
+      memset(&P, 0, sizeof(P));
+      P.status = a.status;
+      Problem& p = P.p[P.nprob++];
+      p.a = Kk;
+      p.b = W13;
+      p.M = bc;
+      p.N = 2 * dh;
+      p.K = dk;
+      p.nz = Z;
+      p.ksplit = 1;
+      segs(p, nsegW, reinterpret_cast<const int(*)[2]>(segW));
+      p.epi = gemm::EPI_HK;
+      p.e = epi_base(a, s0, bc);
+      p.e.gz = sc.gz;
+      p.e.gz_sz = (int64_t)chunk * dh;
+      p.e.gz_sr = dh;
+      p.e.bo[0] = sc.ak[0];
+      p.e.bo[1] = sc.dh1[0];
+      p.e.bo[2] = sc.dh3[0];
+      p.e.bo_lo[0] = split ? sc.ak[1] : nullptr;
+      p.e.bo_lo[1] = split ? sc.dh1[1] : nullptr;
+      p.e.bo_lo[2] = split ? sc.dh3[1] : nullptr;
+      p.e.b_sz = (int64_t)chunk * dh;
+      p.e.b_sr = dh;
+      if (a.causal) add_apply(P, 1);
+      check(launch_gemm(P, s));
+    }
+    // L3: weight gradients (token reductions, split-K with atomics)
+    {
+      Params P;
+      memset(&P, 0, sizeof(P));
+      P.status = a.status;
+      const int kblocks = (bc + gemm::BK - 1) / gemm::BK;
+      const int tiles = Z * (2 * ((dh + 127) / 128) * ((dk + BN - 1) / BN) +
+                             ((dv + 127) / 128) * ((dh + BN - 1) / BN));
+      const int ks = pick_ksplit(kblocks, tiles);
+      for (int g = 0; g < 3; ++g) {
+        Problem& p = P.p[P.nprob++];
+        memset(&p, 0, sizeof(p));
+        p.nz = Z;
+        p.ksplit = ks;
+        p.K = bc;
+        p.epi = gemm::EPI_GRAD;
+        if (g < 2) {
+          p.a = g == 0 ? DH1mn : DH3mn;
+          p.b = Kmn;
+          p.M = dh;
+          p.N = dk;
+          if (split)
+            segs(p, 2, kSegAsplit);
+          else
+            segs(p, 1, kSegExact);
+          p.e = epi_base(a, s0, dh);
+          p.e.f32 = g == 0 ? sc.G[0] : sc.G[1];
+          p.e.f32_sz = (int64_t)dh * dk;
+          p.e.f32_sr = dk;
+        } else {
+          p.a = Vmn;
+          p.b = AKmn;
+          p.M = dv;
+          p.N = dh;
+          if (split)
+            segs(p, 2, kSegBsplit);
+          else
+            segs(p, 1, kSegExact);
+          p.e = epi_base(a, s0, dv);
+          p.e.f32 = sc.G[2];
+          p.e.f32_sz = (int64_t)dv * dh;
+          p.e.f32_sr = dh;
+          p.e.scale = -1.f;
+        }
+      }
+      check(launch_gemm(P, s));
+    }
+    // L4 / L5: Muon orthogonalisation, update and row renormalisation
+    if (split) {
+      ns_kernel<<<Z * 3, kNsThreads, 0, s>>>(na);
+      check(cudaGetLastError());
+    }
+    lact_rows_kernel<<<row_blocks, 256, 0, s>>>(ra);
+    check(cudaGetLastError());
+    if (!a.causal) {
+      Params P;
+      memset(&P, 0, sizeof(P));
+      P.status = a.status;
+      add_apply(P, 0);
+      check(launch_gemm(P, s));
+      Params P2;
+      memset(&P2, 0, sizeof(P2));
+      P2.status = a.status;
+      add_apply(P2, 1);
+      check(launch_gemm(P2, s));
+    }
+  }
+
+  float* finals[3] = {a.W1_final, a.W3_final, a.W2_final};
+  for (int m = 0; m < 3 && result == TTT_OK; ++m) {
+    if (!finals[m]) continue;
+    copy_kernel<<<148, 256, 0, s>>>(finals[m], sc.Wm[m], Z * nW[m]);
+    check(cudaGetLastError());
+  }
+  if (cudaFreeAsync(base, s) != cudaSuccess && result == TTT_OK) result = TTT_ERR_CUDA;
+  return result;
+}
 
 }  // namespace ttt
