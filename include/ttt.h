@@ -80,7 +80,8 @@ typedef enum {
   TTT_ERR_CUDA = -6,        /* a CUDA runtime call failed (launch, memory) */
   TTT_ERR_TIMEOUT = -7,     /* a device-side bounded wait gave up */
   TTT_ERR_ALLOC = -8,       /* stream-ordered scratch allocation failed */
-  TTT_ERR_ARG = -9          /* scalar argument out of range (chunk, enums) */
+  TTT_ERR_ARG = -9,         /* scalar argument out of range (chunk, enums) */
+  TTT_ERR_SCRATCH = -10     /* scratch need exceeds lact_swiglu_fwd_noalloc's fixed pool */
 } ttt_status;
 
 typedef enum { TTT_F32 = 0, TTT_BF16 = 1 } ttt_dtype;
@@ -136,6 +137,37 @@ ttt_status lact_swiglu_fwd_ex(const ttt_tensor* q, const ttt_tensor* k, const tt
                               int32_t causal, const ttt_tensor* out,
                               const ttt_tensor* W1_final, const ttt_tensor* W2_final,
                               const ttt_tensor* W3_final, void* stream);
+
+/*
+ * lact_swiglu_fwd_ex without any device memory allocation. (The pages have
+ * no counterpart to this call: it exists for callers that cannot allocate.)
+ *
+ * Who needs it: callers whose device memory is reserved up front by their
+ * own allocator (a serving engine or training framework that claims nearly
+ * the whole GPU), where a stream-ordered allocation by this library would
+ * fail or fragment memory, and latency-critical code that must not contain
+ * allocation calls. Arguments, results and errors are those of
+ * lact_swiglu_fwd_ex; the caller still passes every input and output.
+ *
+ * Scratch: a fixed 32 MiB device array inside the library (each device that
+ * loads the library holds it until the process exits). A problem whose
+ * scratch need exceeds it is rejected with TTT_ERR_SCRATCH before anything
+ * is launched. The need is about, per (batch, head), 4 bytes x (3 x 2 x
+ * weight elements + chunk x dh) + 2 bytes x (weight elements + 4 x chunk x
+ * dh), doubled for the bf16 parts under Muon.
+ * The first call on a device looks up the array's device address with that
+ * device current; make that first call before any stream capture.
+ * All calls share the one array: calls whose GPU work overlaps (on
+ * different streams, or from different host threads) race on it and give
+ * wrong results; serialise them. What a previous call left in the array does
+ * not affect a call.
+ */
+ttt_status lact_swiglu_fwd_noalloc(const ttt_tensor* q, const ttt_tensor* k, const ttt_tensor* v,
+                                   const ttt_tensor* eta, const ttt_tensor* W1,
+                                   const ttt_tensor* W2, const ttt_tensor* W3, int32_t chunk,
+                                   int32_t update_rule, int32_t causal, const ttt_tensor* out,
+                                   const ttt_tensor* W1_final, const ttt_tensor* W2_final,
+                                   const ttt_tensor* W3_final, void* stream);
 
 /* Static description of a status code (never NULL). */
 const char* ttt_status_string(int32_t status);

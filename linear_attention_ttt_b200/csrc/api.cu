@@ -80,6 +80,36 @@ ttt_status check_tokens(const ttt_tensor* t, int64_t B, int64_t H, int64_t T, in
 
 ttt::TokView view(const ttt_tensor* t) { return {t->data, t->stride[0], t->stride[1], t->stride[2]}; }
 
+ttt_status lact_check_weight(const ttt_tensor* W, int64_t B, int64_t H, int64_t r,
+                                    int64_t c, int64_t* sb) {
+  if (!W->data) return TTT_ERR_NULL;
+  if (W->dtype != TTT_F32) return TTT_ERR_DTYPE;
+  if (W->ndim == 3) {
+    if (W->shape[0] != H || W->shape[1] != r || W->shape[2] != c) return TTT_ERR_SHAPE;
+    *sb = 0;
+  } else if (W->ndim == 4) {
+    if (W->shape[0] != B || W->shape[1] != H || W->shape[2] != r || W->shape[3] != c)
+      return TTT_ERR_SHAPE;
+    *sb = H * r * c;
+  } else {
+    return TTT_ERR_SHAPE;
+  }
+  if (!contiguous(W) || !aligned16(W->data)) return TTT_ERR_LAYOUT;
+  return TTT_OK;
+}
+
+ttt_status lact_check_final(const ttt_tensor* W, int64_t B, int64_t H, int64_t r,
+                                   int64_t c) {
+  if (!W) return TTT_OK;
+  if (!W->data) return TTT_ERR_NULL;
+  if (W->dtype != TTT_F32) return TTT_ERR_DTYPE;
+  if (W->ndim != 4 || W->shape[0] != B || W->shape[1] != H || W->shape[2] != r ||
+      W->shape[3] != c)
+    return TTT_ERR_SHAPE;
+  if (!contiguous(W) || !aligned16(W->data)) return TTT_ERR_LAYOUT;
+  return TTT_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -98,6 +128,7 @@ const char* ttt_status_string(int32_t s) {
     case TTT_ERR_TIMEOUT: return "a device-side bounded wait gave up";
     case TTT_ERR_ALLOC: return "stream-ordered scratch allocation failed";
     case TTT_ERR_ARG: return "scalar argument out of range";
+    case TTT_ERR_SCRATCH: return "scratch need exceeds the fixed pool of lact_swiglu_fwd_noalloc";
     default: return "unknown status";
   }
 }
@@ -200,42 +231,15 @@ ttt_status ttt_linear_fwd(const ttt_tensor* q, const ttt_tensor* k, const ttt_te
   return e == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
 }
 
-static ttt_status lact_check_weight(const ttt_tensor* W, int64_t B, int64_t H, int64_t r,
-                                    int64_t c, int64_t* sb) {
-  if (!W->data) return TTT_ERR_NULL;
-  if (W->dtype != TTT_F32) return TTT_ERR_DTYPE;
-  if (W->ndim == 3) {
-    if (W->shape[0] != H || W->shape[1] != r || W->shape[2] != c) return TTT_ERR_SHAPE;
-    *sb = 0;
-  } else if (W->ndim == 4) {
-    if (W->shape[0] != B || W->shape[1] != H || W->shape[2] != r || W->shape[3] != c)
-      return TTT_ERR_SHAPE;
-    *sb = H * r * c;
-  } else {
-    return TTT_ERR_SHAPE;
-  }
-  if (!contiguous(W) || !aligned16(W->data)) return TTT_ERR_LAYOUT;
-  return TTT_OK;
-}
+}  // extern "C"
 
-static ttt_status lact_check_final(const ttt_tensor* W, int64_t B, int64_t H, int64_t r,
-                                   int64_t c) {
-  if (!W) return TTT_OK;
-  if (!W->data) return TTT_ERR_NULL;
-  if (W->dtype != TTT_F32) return TTT_ERR_DTYPE;
-  if (W->ndim != 4 || W->shape[0] != B || W->shape[1] != H || W->shape[2] != r ||
-      W->shape[3] != c)
-    return TTT_ERR_SHAPE;
-  if (!contiguous(W) || !aligned16(W->data)) return TTT_ERR_LAYOUT;
-  return TTT_OK;
-}
+namespace ttt {
 
-ttt_status lact_swiglu_fwd_ex(const ttt_tensor* q, const ttt_tensor* k, const ttt_tensor* v,
-                              const ttt_tensor* eta, const ttt_tensor* W1, const ttt_tensor* W2,
-                              const ttt_tensor* W3, int32_t chunk, int32_t update_rule,
-                              int32_t causal, const ttt_tensor* out,
-                              const ttt_tensor* W1_final, const ttt_tensor* W2_final,
-                              const ttt_tensor* W3_final, void* stream) {
+ttt_status lact_build_args(const ttt_tensor* q, const ttt_tensor* k, const ttt_tensor* v,
+                           const ttt_tensor* eta, const ttt_tensor* W1, const ttt_tensor* W2,
+                           const ttt_tensor* W3, int32_t chunk, int32_t update_rule,
+                           int32_t causal, const ttt_tensor* out, const ttt_tensor* W1_final,
+                           const ttt_tensor* W2_final, const ttt_tensor* W3_final, LactArgs* ap) {
   if (!q || !k || !v || !eta || !W1 || !W2 || !W3 || !out) return TTT_ERR_NULL;
   if (chunk < 1) return TTT_ERR_ARG;
   if (update_rule != LACT_UPDATE_GD && update_rule != LACT_UPDATE_MUON) return TTT_ERR_ARG;
@@ -275,7 +279,7 @@ ttt_status lact_swiglu_fwd_ex(const ttt_tensor* q, const ttt_tensor* k, const tt
       if (o != o2 && overlaps(o, o2)) return TTT_ERR_ARG;
   }
 
-  ttt::LactArgs a;
+  LactArgs& a = *ap;
   a.q = view(q);
   a.k = view(k);
   a.v = view(v);
@@ -302,6 +306,23 @@ ttt_status lact_swiglu_fwd_ex(const ttt_tensor* q, const ttt_tensor* k, const tt
   a.dtype = dt;
   a.status = device_status_ptr();
   if (!a.status) return TTT_ERR_CUDA;
+  return TTT_OK;
+}
+
+}  // namespace ttt
+
+extern "C" {
+
+ttt_status lact_swiglu_fwd_ex(const ttt_tensor* q, const ttt_tensor* k, const ttt_tensor* v,
+                              const ttt_tensor* eta, const ttt_tensor* W1, const ttt_tensor* W2,
+                              const ttt_tensor* W3, int32_t chunk, int32_t update_rule,
+                              int32_t causal, const ttt_tensor* out,
+                              const ttt_tensor* W1_final, const ttt_tensor* W2_final,
+                              const ttt_tensor* W3_final, void* stream) {
+  ttt::LactArgs a;
+  ttt_status st = ttt::lact_build_args(q, k, v, eta, W1, W2, W3, chunk, update_rule, causal, out,
+                                       W1_final, W2_final, W3_final, &a);
+  if (st != TTT_OK) return st;
   return ttt::lact_forward(a, static_cast<cudaStream_t>(stream));
 }
 

@@ -338,31 +338,71 @@ int pick_ksplit(int kblocks, int tiles) {
 
 }  // namespace
 
-ttt_status lact_forward(const LactArgs& a, cudaStream_t s) {
-  if (a.dtype != TTT_BF16) return TTT_ERR_UNSUPPORTED;
-  if (a.dk != a.dv || (a.dk != 64 && a.dk != 128 && a.dk != 256)) return TTT_ERR_UNSUPPORTED;
-  if (a.dh % 128 != 0 || a.dh > 1024) return TTT_ERR_UNSUPPORTED;
-  const int Z = a.B * a.H, dk = a.dk, dv = a.dv, dh = a.dh;
-  const int chunk = a.T > 0 ? (a.chunk < a.T ? a.chunk : a.T) : 1;
-  const bool split = a.update_rule == LACT_UPDATE_MUON;
+namespace {
 
-  // ---- scratch (stream-ordered) ----
-  const int64_t nW[3] = {(int64_t)dh * dk, (int64_t)dh * dk, (int64_t)dv * dh};
-  const int64_t nrows[3] = {dh, dh, dv};
+struct Sizes {
+  bool ok;
+  int Z, chunk;
+  bool split;
+  int64_t nW[3], nrows[3], ns_stride;
+  size_t f32n, bfn, bytes;
+};
+
+Sizes lact_sizes(const LactArgs& a) {
+  Sizes z;
+  memset(&z, 0, sizeof(z));
+  z.ok = a.dtype == TTT_BF16 && a.dk == a.dv && (a.dk == 64 || a.dk == 128 || a.dk == 256) &&
+         a.dh % 128 == 0 && a.dh <= 1024;
+  if (!z.ok) return z;
+  const int dk = a.dk, dv = a.dv, dh = a.dh;
+  z.Z = a.B * a.H;
+  z.chunk = a.T > 0 ? (a.chunk < a.T ? a.chunk : a.T) : 1;
+  z.split = a.update_rule == LACT_UPDATE_MUON;
+  z.nW[0] = z.nW[1] = (int64_t)dh * dk;
+  z.nW[2] = (int64_t)dv * dh;
+  z.nrows[0] = z.nrows[1] = dh;
+  z.nrows[2] = dv;
   const int s_max = dk < dh ? dk : dh;
-  const int64_t ns_stride = 2 * (int64_t)s_max * s_max + (int64_t)dh * dk;
-  size_t f32n = 0;
-  for (int m = 0; m < 3; ++m) f32n += (size_t)Z * (2 * nW[m] + nrows[m]);
-  f32n += (size_t)Z * chunk * dh;                     // gz
-  if (split) f32n += (size_t)Z * 3 * ns_stride;       // NS scratch
-  size_t bfn = (size_t)Z * (2 * dh * dk + dv * dh) * (split ? 2 : 1);
-  bfn += (size_t)Z * chunk * dh * 4 * (split ? 2 : 1);
-  const size_t bytes = f32n * 4 + bfn * 2 + 4096;
+  z.ns_stride = 2 * (int64_t)s_max * s_max + (int64_t)dh * dk;
+  for (int m = 0; m < 3; ++m) z.f32n += (size_t)z.Z * (2 * z.nW[m] + z.nrows[m]);
+  z.f32n += (size_t)z.Z * z.chunk * dh;                  // gz
+  if (z.split) z.f32n += (size_t)z.Z * 3 * z.ns_stride;  // Newton-Schulz scratch
+  z.bfn = (size_t)z.Z * (2 * dh * dk + dv * dh) * (z.split ? 2 : 1);
+  z.bfn += (size_t)z.Z * z.chunk * dh * 4 * (z.split ? 2 : 1);
+  z.bytes = z.f32n * 4 + z.bfn * 2 + 4096;
+  return z;
+}
+
+}  // namespace
+
+size_t lact_scratch_bytes(const LactArgs& a) {
+  Sizes z = lact_sizes(a);
+  return z.ok ? z.bytes : 0;
+}
+
+ttt_status lact_forward(const LactArgs& a, cudaStream_t s) {
+  const Sizes z = lact_sizes(a);
+  if (!z.ok) return TTT_ERR_UNSUPPORTED;
   void* base = nullptr;
-  if (cudaMallocAsync(&base, bytes, s) != cudaSuccess) {
+  if (cudaMallocAsync(&base, z.bytes, s) != cudaSuccess) {
     cudaGetLastError();
     return TTT_ERR_ALLOC;
   }
+  ttt_status r = lact_run(a, s, base, z.bytes);
+  if (cudaFreeAsync(base, s) != cudaSuccess && r == TTT_OK) r = TTT_ERR_CUDA;
+  return r;
+}
+
+ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes) {
+  const Sizes zz = lact_sizes(a);
+  if (!zz.ok) return TTT_ERR_UNSUPPORTED;
+  if (!base || bytes < zz.bytes || (reinterpret_cast<uintptr_t>(base) & 255u)) return TTT_ERR_ARG;
+  const int Z = zz.Z, dk = a.dk, dv = a.dv, dh = a.dh;
+  const int chunk = zz.chunk;
+  const bool split = zz.split;
+  const int64_t* nW = zz.nW;
+  const int64_t* nrows = zz.nrows;
+  const int64_t ns_stride = zz.ns_stride;
   Scratch sc;
   {
     float* f = static_cast<float*>(base);
@@ -636,7 +676,6 @@ ttt_status lact_forward(const LactArgs& a, cudaStream_t s) {
     copy_kernel<<<148, 256, 0, s>>>(finals[m], sc.Wm[m], Z * nW[m]);
     check(cudaGetLastError());
   }
-  if (cudaFreeAsync(base, s) != cudaSuccess && result == TTT_OK) result = TTT_ERR_CUDA;
   return result;
 }
 

@@ -16,7 +16,22 @@ struct LactArgs {
   int* status;
 };
 
-// Enqueues the whole layer forward on `s`; returns a ttt_status.
+// Enqueues the whole layer forward on `s`, taking its scratch from the
+// device's default stream-ordered memory pool; returns a ttt_status.
 ttt_status lact_forward(const LactArgs& a, cudaStream_t s);
+
+// Bytes of device scratch lact_run needs for `a` (0 if `a` is unsupported).
+size_t lact_scratch_bytes(const LactArgs& a);
+
+// Same computation on caller-provided scratch of `bytes` >= lact_scratch_bytes(a),
+// 256-byte aligned. Allocates nothing.
+ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* scratch, size_t bytes);
+
+// Validates the C-ABI arguments of lact_swiglu_fwd_ex and fills `a`.
+ttt_status lact_build_args(const ttt_tensor* q, const ttt_tensor* k, const ttt_tensor* v,
+                           const ttt_tensor* eta, const ttt_tensor* W1, const ttt_tensor* W2,
+                           const ttt_tensor* W3, int32_t chunk, int32_t update_rule,
+                           int32_t causal, const ttt_tensor* out, const ttt_tensor* W1_final,
+                           const ttt_tensor* W2_final, const ttt_tensor* W3_final, LactArgs* a);
 
 }  // namespace ttt

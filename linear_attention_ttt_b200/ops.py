@@ -22,7 +22,7 @@ LACT_UPDATE_GD, LACT_UPDATE_MUON = 0, 1
 STATUS = {
     0: "TTT_OK", -1: "TTT_ERR_NULL", -2: "TTT_ERR_SHAPE", -3: "TTT_ERR_DTYPE",
     -4: "TTT_ERR_LAYOUT", -5: "TTT_ERR_UNSUPPORTED", -6: "TTT_ERR_CUDA",
-    -7: "TTT_ERR_TIMEOUT", -8: "TTT_ERR_ALLOC", -9: "TTT_ERR_ARG",
+    -7: "TTT_ERR_TIMEOUT", -8: "TTT_ERR_ALLOC", -9: "TTT_ERR_ARG", -10: "TTT_ERR_SCRATCH",
 }
 
 
@@ -54,6 +54,8 @@ SIGNATURES = {
                          ctypes.c_void_p], ctypes.c_int32),
     "lact_swiglu_fwd_ex": ([P, P, P, P, P, P, P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                             P, P, P, P, ctypes.c_void_p], ctypes.c_int32),
+    "lact_swiglu_fwd_noalloc": ([P, P, P, P, P, P, P, ctypes.c_int32, ctypes.c_int32,
+                                 ctypes.c_int32, P, P, P, P, ctypes.c_void_p], ctypes.c_int32),
     "ttt_status_string": ([ctypes.c_int32], ctypes.c_char_p),
     "ttt_get_device_status": ([ctypes.c_void_p], ctypes.c_int32),
     "ttt_version": ([], ctypes.c_int32),
@@ -148,6 +150,32 @@ def lact_swiglu_fwd(q, k, v, eta, W1, W2, W3, chunk: int, update_rule: int = LAC
     code = load().lact_swiglu_fwd_ex(*r[:7], int(chunk), int(update_rule), int(causal), r[7],
                                      r[8], r[9], r[10], _stream(stream))
     _check(code, "lact_swiglu_fwd")
+    return (out, *F) if finals else out
+
+
+def lact_swiglu_fwd_noalloc(q, k, v, eta, W1, W2, W3, chunk: int,
+                            update_rule: int = LACT_UPDATE_GD, causal: int = 1, out=None,
+                            finals=False, stream=None):
+    """lact_swiglu_fwd on the library's fixed device scratch pool: the C call
+    allocates no device memory (for callers that cannot allocate; see
+    include/ttt.h). Output tensors passed in are written in place; tensors
+    created here (when `out` or the finals are omitted) are the caller's
+    convenience, made before the call."""
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    dh = W1.shape[-2]
+    if out is None:
+        out = torch.empty((B, H, T, dv), dtype=q.dtype, device=q.device)
+    F = [None, None, None]
+    if finals:
+        F = [torch.empty((B, H, dh, dk), dtype=torch.float32, device=q.device),
+             torch.empty((B, H, dv, dh), dtype=torch.float32, device=q.device),
+             torch.empty((B, H, dh, dk), dtype=torch.float32, device=q.device)]
+    ds = [describe(x) for x in (q, k, v, eta, W1, W2, W3, out, *F)]
+    r = [_ref(d) for d in ds]
+    code = load().lact_swiglu_fwd_noalloc(*r[:7], int(chunk), int(update_rule), int(causal), r[7],
+                                          r[8], r[9], r[10], _stream(stream))
+    _check(code, "lact_swiglu_fwd_noalloc")
     return (out, *F) if finals else out
 
 
