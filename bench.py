@@ -222,6 +222,27 @@ def kernel_key(w):
     return "ttt_linear_bf16" if w.dtype == synth.BF16 else "ttt_linear_f32"
 
 
+def rank_workload(index, rank, chunk=None):
+    """Each rank runs its own replica: the same workload shape with an
+    independent draw of the inputs (weak scaling, no data-path collective)."""
+    return synth.config(index, chunk=chunk, replica=rank)
+
+
+def max_over_ranks(value, dist=None, device=None):
+    """Max of a per-rank scalar over all ranks (a float on every rank)."""
+    if dist is None:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_step, world, ms_per_step):
+    """Whole-job tokens/s: every rank processed tokens_per_step per step and
+    the job's step time is the slowest rank's."""
+    return tokens_per_step * world / (ms_per_step / 1e3)
+
+
 def cpu_oracle_step(w, sample_heads):
     """Runs the fp64 oracle on the first `sample_heads` (batch, head)
     sequences of the workload (all of them for sample_heads >= B*H); returns
@@ -271,7 +292,7 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
 
-    w = synth.config(args.workload, chunk=args.chunk)
+    w = rank_workload(args.workload, rank, chunk=args.chunk)
     tokens_per_step = w.B * w.T
     base_cfg = {"workload": w.name, "batch": w.B, "heads": w.H, "seq_len": w.T, "dk": w.dk,
                 "dv": w.dv, "chunk": w.chunk, "variant": w.variant,
@@ -347,13 +368,9 @@ def main():
         t_wall = time.perf_counter() - t_wall
     barrier()
     per = [a.elapsed_time(b) for a, b in ev]
-    total_ms = float(sum(per))
-    if dist is not None:
-        tt = torch.tensor([total_ms], device=device)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(sum(per), dist, device)
     ms_per_step = total_ms / args.steps
-    value = tokens_per_step * world / (ms_per_step / 1e3)
+    value = job_throughput(tokens_per_step, world, ms_per_step)
 
     # ---- end to end through the public API with host buffers ----
     host = {k: v.to("cpu").pin_memory() for k, v in d.items()}
@@ -377,12 +394,8 @@ def main():
         host_out.copy_(step.out, non_blocking=True)
     b.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = a.elapsed_time(b) / e2e_steps
-    if dist is not None:
-        tt = torch.tensor([e2e_ms], device=device)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
-    e2e_value = tokens_per_step * world / (e2e_ms / 1e3)
+    e2e_ms = max_over_ranks(a.elapsed_time(b) / e2e_steps, dist, device)
+    e2e_value = job_throughput(tokens_per_step, world, e2e_ms)
 
     pk = peaks()
     key = kernel_key(w)

@@ -158,10 +158,12 @@ CONFIG_NAMES = {
 
 
 def config(index: int, chunk: Optional[int] = None, T: Optional[int] = None,
-           B: Optional[int] = None, H: Optional[int] = None) -> Workload:
+           B: Optional[int] = None, H: Optional[int] = None, replica: int = 0) -> Workload:
     """Named workload ``index`` (1..5); T/B/H overrides give smaller cases with
-    the same distributions (used for parity runs the oracle finishes quickly)."""
-    seed = 1000 + index
+    the same distributions (used for parity runs the oracle finishes quickly).
+    ``replica`` > 0 draws an independent batch of the same workload (one per
+    rank of a multi-GPU run)."""
+    seed = 1000 + index + 100 * replica
     if index == 1:
         w = make_ttt_linear(B or 1, H or 2, T or 256, 64, 64, chunk or 16, F32, LOSS_MSE,
                             seed, qk_norm=True, eta_kind="const", eta_scale=0.1, w0_std=0.02)
