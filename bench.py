@@ -208,6 +208,10 @@ def recorded_traffic(kernel_key, sha):
 
 
 KERNEL_SOURCES = {
+    "la_tc": ["linear_attention_ttt_b200/csrc/la_tc.cu",
+              "linear_attention_ttt_b200/csrc/common.cuh",
+              "linear_attention_ttt_b200/csrc/tma.cuh",
+              "linear_attention_ttt_b200/csrc/umma.cuh"],
     "ttt_linear_bf16": ["linear_attention_ttt_b200/csrc/ttt_linear_bf16.cu",
                         "linear_attention_ttt_b200/csrc/common.cuh",
                         "linear_attention_ttt_b200/csrc/tma.cuh"],
@@ -219,7 +223,11 @@ KERNEL_SOURCES = {
 def kernel_key(w):
     if w.variant == "lact":
         return "lact"
-    return "ttt_linear_bf16" if w.dtype == synth.BF16 else "ttt_linear_f32"
+    if w.dtype != synth.BF16:
+        return "ttt_linear_f32"
+    if w.loss == synth.LOSS_NEG_DOT and w.dk == 128 and w.dv == 128:
+        return "la_tc"
+    return "ttt_linear_bf16"
 
 
 def rank_workload(index, rank, chunk=None):

@@ -109,5 +109,7 @@ struct LinearArgs {
 
 cudaError_t launch_ttt_linear_f32(const LinearArgs& a, cudaStream_t s);
 cudaError_t launch_ttt_linear_bf16(const LinearArgs& a, cudaStream_t s, bool* supported);
+bool la_tc_supported(const LinearArgs& a);
+cudaError_t launch_la_tc(const LinearArgs& a, cudaStream_t s);
 
 }  // namespace ttt

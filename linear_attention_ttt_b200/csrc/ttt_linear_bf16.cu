@@ -367,6 +367,7 @@ cudaError_t launch(const LinearArgs& a, cudaStream_t s) {
 cudaError_t launch_ttt_linear_bf16(const LinearArgs& a, cudaStream_t s, bool* supported) {
   *supported = (a.dk == a.dv) && (a.dk == 64 || a.dk == 128);
   if (!*supported) return cudaSuccess;
+  if (la_tc_supported(a)) return launch_la_tc(a, s);
   return a.dk == 64 ? launch<64>(a, s) : launch<128>(a, s);
 }
 
