@@ -3,8 +3,8 @@
 //
 // Per (batch, head) z the fast weights W1, W3 [dh][dk] and W2 [dv][dh] live
 // in fp32 master copies in scratch memory, with bf16 operand copies refreshed
-// after every update (W1 and W3 rows interleaved in blocks of 64 into W13 so
-// one 128-column tile holds matching h1/h3 columns). One chunk step, all heads
+// after every update (W1 and W3 rows interleaved in blocks of 128 into W13 so
+// one 256-column tile holds matching h1/h3 columns). One chunk step, all heads
 // at once (causal order: apply with the weights before the chunk, then
 // update):
 //   L1  Gz = -eta (V W2)                     [b x dh] fp32
@@ -33,7 +33,7 @@ using gemm::Operand;
 using gemm::Params;
 using gemm::Problem;
 
-constexpr int BN = 128;
+constexpr int BN = 256;     // GEMM tile width (W13 interleave block = BN / 2)
 
 // ---------------------------------------------------------------------------
 // Row kernels: prepare / update / renormalise the fast weights
@@ -107,7 +107,7 @@ __global__ void __launch_bounds__(256) lact_rows_kernel(RowArgs a) {
   } else {
     hi = a.w13_hi;
     lo = a.w13_lo;
-    orow = (int64_t)z * 2 * a.dh + (r / 64) * 128 + (m == 1 ? 64 : 0) + (r % 64);
+    orow = (int64_t)z * 2 * a.dh + (r / (BN / 2)) * BN + (m == 1 ? BN / 2 : 0) + (r % (BN / 2));
   }
   for (int i = 0; i < per; ++i) {
     const int c = lane + 32 * i;
@@ -248,6 +248,29 @@ bool map_buf(CUtensorMap* m, const void* base, int Z, int rows, int rows_alloc, 
                    CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+// Output maps for the TMA-store epilogue: boxes of {16 columns, 32 rows}.
+bool out_map_buf(CUtensorMap* m, const void* base, bool bf16, int Z, int rows, int cols) {
+  const uint64_t es = bf16 ? 2 : 4;
+  uint64_t dims[4] = {(uint64_t)cols, (uint64_t)rows, (uint64_t)Z, 1};
+  uint64_t strides[3] = {(uint64_t)cols * es, (uint64_t)cols * es * rows,
+                         (uint64_t)cols * es * rows * Z};
+  uint32_t box[4] = {16, 32, 1, 1};
+  return make_tmap(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4,
+                   base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+bool out_map_tokens(CUtensorMap* m, const TokViewMut& v, const LactArgs& a, int d) {
+  TokViewMut x = v;
+  const uint64_t es = a.dtype == TTT_BF16 ? 2 : 4;
+  if (a.B == 1) x.sb = (int64_t)a.H * a.T * d;
+  if (a.H == 1) x.sh = (int64_t)a.T * d;
+  if (a.T == 1) x.st = d;
+  uint64_t dims[4] = {(uint64_t)d, (uint64_t)a.T, (uint64_t)a.H, (uint64_t)a.B};
+  uint64_t strides[3] = {(uint64_t)x.st * es, (uint64_t)x.sh * es, (uint64_t)x.sb * es};
+  uint32_t box[4] = {16, 32, 1, 1};
+  return make_tmap(m, es == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                   4, x.p, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
 struct Scratch {
   float *Wm[3], *rho[3], *G[3], *gz, *ns;
   __nv_bfloat16 *w13[2], *w2[2];          // hi, lo
@@ -267,6 +290,18 @@ void fill_problem_tiles(Params& P) {
   P.total_tiles = t;
 }
 
+int num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+      n = 148;
+  }
+  return n;
+}
+
+// Persistent launch: one CTA per SM (or fewer if there are fewer tiles).
 cudaError_t launch_gemm(Params& P, cudaStream_t s) {
   fill_problem_tiles(P);
   if (P.total_tiles == 0) return cudaSuccess;
@@ -274,7 +309,8 @@ cudaError_t launch_gemm(Params& P, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(gemm::gemm_kernel<BN>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  gemm::gemm_kernel<BN><<<P.total_tiles, gemm::kThreads, smem, s>>>(P);
+  const int grid = P.total_tiles < num_sms() ? P.total_tiles : num_sms();
+  gemm::gemm_kernel<BN><<<grid, gemm::kThreads, smem, s>>>(P);
   return cudaGetLastError();
 }
 
@@ -327,13 +363,17 @@ gemm::EpiArgs epi_base(const LactArgs& a, int s0, int rows_valid) {
   e.out_bf16 = a.dtype == TTT_BF16;
   e.rows_valid = rows_valid;
   e.scale = 1.f;
+  e.nsplit = 1;
+  e.ozdiv = 1;
   return e;
 }
 
+// Split the token reduction so that the gradient GEMMs give about two tiles
+// per SM, but keep at least 4 K blocks per split.
 int pick_ksplit(int kblocks, int tiles) {
   int ks = 1;
-  while (ks < kblocks && tiles * ks < 4 * 148) ks *= 2;
-  return ks < 1 ? 1 : (ks > kblocks ? kblocks : ks);
+  while (ks * 2 <= kblocks / 4 && tiles * ks < 2 * num_sms()) ks *= 2;
+  return ks;
 }
 
 }  // namespace
@@ -516,6 +556,7 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
       result = TTT_ERR_CUDA;
       break;
     }
+    bool okm = true;  // output maps built
     auto add_apply = [&](Params& P, int stage) {
       // stage 0: Aq from Q; stage 1: Y from Aq
       Problem& p = P.p[P.nprob++];
@@ -531,10 +572,10 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
         segs(p, nsegW, reinterpret_cast<const int(*)[2]>(segW));
         p.epi = gemm::EPI_AQ;
         p.e = epi_base(a, s0, bc);
-        p.e.bo[0] = sc.aq[0];
-        p.e.bo_lo[0] = split ? sc.aq[1] : nullptr;
-        p.e.b_sz = (int64_t)chunk * dh;
-        p.e.b_sr = dh;
+        p.e.nsplit = split ? 2 : 1;
+        p.e.ozdiv = Z;
+        okm &= out_map_buf(&p.e.omap[0], sc.aq[0], true, Z, chunk, dh);
+        if (split) okm &= out_map_buf(&p.e.omap[3], sc.aq[1], true, Z, chunk, dh);
       } else {
         p.a = AQk;
         p.b = W2k;
@@ -547,6 +588,9 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
           segs(p, 1, kSegExact);
         p.epi = gemm::EPI_Y;
         p.e = epi_base(a, s0, bc);
+        p.e.ozdiv = a.H;
+        p.e.orow0 = s0;
+        okm &= out_map_tokens(&p.e.omap[0], a.out, a, dv);
       }
     };
 
@@ -566,10 +610,11 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
       segs(p, nsegW, reinterpret_cast<const int(*)[2]>(segW));
       p.epi = gemm::EPI_GZ;
       p.e = epi_base(a, s0, bc);
-      p.e.f32 = sc.gz;
-      p.e.f32_sz = (int64_t)chunk * dh;
-      p.e.f32_sr = dh;
+      p.e.gz = sc.gz;
+      p.e.gz_rows = chunk;
+      p.e.gz_cols = dh;
       if (a.causal) add_apply(P, 0);
+      if (!okm) result = TTT_ERR_CUDA;
       check(launch_gemm(P, s));
     }
     // L2: key forward + backprop epilogue (+ Y when causal)
@@ -589,17 +634,17 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
       p.epi = gemm::EPI_HK;
       p.e = epi_base(a, s0, bc);
       p.e.gz = sc.gz;
-      p.e.gz_sz = (int64_t)chunk * dh;
-      p.e.gz_sr = dh;
-      p.e.bo[0] = sc.ak[0];
-      p.e.bo[1] = sc.dh1[0];
-      p.e.bo[2] = sc.dh3[0];
-      p.e.bo_lo[0] = split ? sc.ak[1] : nullptr;
-      p.e.bo_lo[1] = split ? sc.dh1[1] : nullptr;
-      p.e.bo_lo[2] = split ? sc.dh3[1] : nullptr;
-      p.e.b_sz = (int64_t)chunk * dh;
-      p.e.b_sr = dh;
+      p.e.gz_rows = chunk;
+      p.e.gz_cols = dh;
+      p.e.nsplit = split ? 2 : 1;
+      p.e.ozdiv = Z;
+      for (int x = 0; x < (split ? 2 : 1); ++x) {
+        okm &= out_map_buf(&p.e.omap[3 * x + 0], sc.ak[x], true, Z, chunk, dh);
+        okm &= out_map_buf(&p.e.omap[3 * x + 1], sc.dh1[x], true, Z, chunk, dh);
+        okm &= out_map_buf(&p.e.omap[3 * x + 2], sc.dh3[x], true, Z, chunk, dh);
+      }
       if (a.causal) add_apply(P, 1);
+      if (!okm) result = TTT_ERR_CUDA;
       check(launch_gemm(P, s));
     }
     // L3: weight gradients (token reductions, split-K with atomics)
@@ -608,8 +653,8 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
       memset(&P, 0, sizeof(P));
       P.status = a.status;
       const int kblocks = (bc + gemm::BK - 1) / gemm::BK;
-      const int tiles = Z * (2 * ((dh + 127) / 128) * ((dk + BN - 1) / BN) +
-                             ((dv + 127) / 128) * ((dh + BN - 1) / BN));
+      const int tiles = Z * (2 * ((dh + gemm::BM - 1) / gemm::BM) * ((dk + BN - 1) / BN) +
+                             ((dv + gemm::BM - 1) / gemm::BM) * ((dh + BN - 1) / BN));
       const int ks = pick_ksplit(kblocks, tiles);
       for (int g = 0; g < 3; ++g) {
         Problem& p = P.p[P.nprob++];
@@ -628,9 +673,8 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
           else
             segs(p, 1, kSegExact);
           p.e = epi_base(a, s0, dh);
-          p.e.f32 = g == 0 ? sc.G[0] : sc.G[1];
-          p.e.f32_sz = (int64_t)dh * dk;
-          p.e.f32_sr = dk;
+          p.e.ozdiv = Z;
+          okm &= out_map_buf(&p.e.omap[0], g == 0 ? sc.G[0] : sc.G[1], false, Z, dh, dk);
         } else {
           p.a = Vmn;
           p.b = AKmn;
@@ -641,12 +685,12 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
           else
             segs(p, 1, kSegExact);
           p.e = epi_base(a, s0, dv);
-          p.e.f32 = sc.G[2];
-          p.e.f32_sz = (int64_t)dv * dh;
-          p.e.f32_sr = dh;
+          p.e.ozdiv = Z;
           p.e.scale = -1.f;
+          okm &= out_map_buf(&p.e.omap[0], sc.G[2], false, Z, dv, dh);
         }
       }
+      if (!okm) result = TTT_ERR_CUDA;
       check(launch_gemm(P, s));
     }
     // L4 / L5: Muon orthogonalisation, update and row renormalisation
