@@ -14,7 +14,7 @@
 //       Y  = Aq W2^T -> layer output         [b x dv]               (causal)
 //   L3  G1 = dH1^T K, G3 = dH3^T K           [dh x dk] fp32 (split-K, atomics)
 //       G2 = -V^T Ak'                        [dv x dh]
-//   L4  Muon: G <- NS5(G) (fp32, CUDA cores)
+//   L4  Muon: G <- NS5(G) (split-bf16 tensor-core MMAs, fp32 accumulation)
 //   L5  W <- W - G; each row rescaled to its initial L2 norm; bf16 copies.
 // Non-causal (update, then apply): L1 without Aq, L2 without Y, L3, L4, L5,
 // then Aq and Y with the updated weights.
@@ -120,7 +120,8 @@ __global__ void __launch_bounds__(256) lact_rows_kernel(RowArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// Newton-Schulz (Muon) on the CUDA cores, fp32: one CTA per gradient matrix.
+// Newton-Schulz (Muon) on the tensor cores in split-bf16 precision: one CTA
+// per gradient matrix.
 // ---------------------------------------------------------------------------
 
 struct NsArgs {
@@ -133,40 +134,112 @@ struct NsArgs {
 };
 
 constexpr int kNsThreads = 1024;
-constexpr int kTile = 32;
 
-// C[M x N] = alpha * op(A) op(B) + beta * Cin, all row-major in global memory
-// (L2-resident scratch). op(A) is A or A^T (tA), same for B. Computed by the
-// whole CTA with 32x32 shared-memory tiles.
+// C[M x N] = alpha * op(A) op(B) + beta * Cin, all row-major fp32 in global
+// memory (L2-resident scratch); op(A) is A or A^T (tA), same for B. Computed
+// by the whole CTA (32 warps) on the tensor cores with m16n8k16 MMAs in
+// split-bf16 precision: each fp32 operand x is held as hi = bf16(x) and
+// lo = bf16(x - hi), and the product accumulates hi*hi + lo*hi + hi*lo in fp32
+// (relative error about 2^-16 per product, near fp32). Output tiles are
+// 128 x 128; warp (wm, wn) of a 4 x 8 grid owns rows 32*wm.., columns 16*wn...
+constexpr int kNsTM = 128, kNsTN = 128, kNsTK = 32;
+constexpr int kNsLdA = kNsTK + 8;   // padded row length (bf16) of the A tiles
+constexpr int kNsLdB = kNsTN + 8;   // padded row length (bf16) of the B tiles
+
+__device__ __forceinline__ void ns_mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                       uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7},"
+      " {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void ns_ldsm_x4(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"((uint32_t)__cvta_generic_to_shared(p)));
+}
+__device__ __forceinline__ void ns_ldsm_x4_t(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"((uint32_t)__cvta_generic_to_shared(p)));
+}
+
 __device__ void cta_gemm(float* C, const float* Cin, const float* A, const float* B, int M, int N,
                          int K, bool tA, bool tB, int lda, int ldb, float alpha, float beta) {
-  __shared__ float As[kTile][kTile + 1], Bs[kTile][kTile + 1];
-  const int tx = threadIdx.x % kTile, ty = threadIdx.x / kTile;  // 32 x 32 threads
-  for (int i0 = 0; i0 < M; i0 += kTile)
-    for (int j0 = 0; j0 < N; j0 += kTile) {
-      float acc = 0.f;
-      for (int k0 = 0; k0 < K; k0 += kTile) {
-        // A tile: rows i0+ty, cols k0+tx of op(A)
-        {
-          const int i = i0 + ty, k = k0 + tx;
-          As[ty][tx] = (i < M && k < K) ? (tA ? A[(int64_t)k * lda + i] : A[(int64_t)i * lda + k]) : 0.f;
+  __shared__ __align__(16) __nv_bfloat16 sa[2][kNsTM * kNsLdA];  // [hi|lo][m][k]
+  __shared__ __align__(16) __nv_bfloat16 sb[2][kNsTK * kNsLdB];  // [hi|lo][k][n]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int wm = warp >> 3, wn = warp & 7;
+  const int mi = lane >> 3, rr = lane & 7, g = lane >> 2, c4 = lane & 3;
+  for (int i0 = 0; i0 < M; i0 += kNsTM)
+    for (int j0 = 0; j0 < N; j0 += kNsTN) {
+      float acc[2][2][4] = {};
+      for (int k0 = 0; k0 < K; k0 += kNsTK) {
+        // A tile [128 x 32] and B tile [32 x 128]: fp32 -> bf16 hi / lo
+        for (int e = tid; e < kNsTM * kNsTK; e += kNsThreads) {
+          int m, k;
+          if (tA) { m = e % kNsTM; k = e / kNsTM; } else { m = e / kNsTK; k = e % kNsTK; }
+          const int gi = i0 + m, gk = k0 + k;
+          float x = 0.f;
+          if (gi < M && gk < K) x = tA ? A[(int64_t)gk * lda + gi] : A[(int64_t)gi * lda + gk];
+          const __nv_bfloat16 h = __float2bfloat16_rn(x);
+          sa[0][m * kNsLdA + k] = h;
+          sa[1][m * kNsLdA + k] = __float2bfloat16_rn(x - __bfloat162float(h));
         }
-        {
-          const int k = k0 + ty, j = j0 + tx;
-          Bs[ty][tx] = (k < K && j < N) ? (tB ? B[(int64_t)j * ldb + k] : B[(int64_t)k * ldb + j]) : 0.f;
+        for (int e = tid; e < kNsTK * kNsTN; e += kNsThreads) {
+          int k, n;
+          if (tB) { k = e % kNsTK; n = e / kNsTK; } else { k = e / kNsTN; n = e % kNsTN; }
+          const int gk = k0 + k, gj = j0 + n;
+          float x = 0.f;
+          if (gk < K && gj < N) x = tB ? B[(int64_t)gj * ldb + gk] : B[(int64_t)gk * ldb + gj];
+          const __nv_bfloat16 h = __float2bfloat16_rn(x);
+          sb[0][k * kNsLdB + n] = h;
+          sb[1][k * kNsLdB + n] = __float2bfloat16_rn(x - __bfloat162float(h));
         }
         __syncthreads();
-#pragma unroll 8
-        for (int kk = 0; kk < kTile; ++kk) acc = fmaf(As[ty][kk], Bs[kk][tx], acc);
+#pragma unroll
+        for (int kk = 0; kk < kNsTK; kk += 16) {
+          uint32_t af[2][2][4], bf[2][2][2];  // [hi|lo][m or n tile]
+#pragma unroll
+          for (int x = 0; x < 2; ++x) {
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+              ns_ldsm_x4(af[x][mt], &sa[x][(32 * wm + 16 * mt + rr + 8 * (mi & 1)) * kNsLdA + kk +
+                                           8 * (mi >> 1)]);
+            uint32_t r[4];
+            ns_ldsm_x4_t(r, &sb[x][(kk + rr + 8 * (mi & 1)) * kNsLdB + 16 * wn + 8 * (mi >> 1)]);
+            bf[x][0][0] = r[0];
+            bf[x][0][1] = r[1];
+            bf[x][1][0] = r[2];
+            bf[x][1][1] = r[3];
+          }
+#pragma unroll
+          for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+              ns_mma(acc[mt][nt], af[0][mt], bf[0][nt][0], bf[0][nt][1]);  // hi * hi
+              ns_mma(acc[mt][nt], af[1][mt], bf[0][nt][0], bf[0][nt][1]);  // lo * hi
+              ns_mma(acc[mt][nt], af[0][mt], bf[1][nt][0], bf[1][nt][1]);  // hi * lo
+            }
+        }
         __syncthreads();
       }
-      const int i = i0 + ty, j = j0 + tx;
-      if (i < M && j < N) {
-        const float prev = (beta != 0.f) ? Cin[(int64_t)i * N + j] : 0.f;
-        C[(int64_t)i * N + j] = alpha * acc + beta * prev;
-      }
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int i = i0 + 32 * wm + 16 * mt + g + 8 * (q >> 1);
+            const int j = j0 + 16 * wn + 8 * nt + 2 * c4 + (q & 1);
+            if (i < M && j < N) {
+              const float prev = (beta != 0.f) ? Cin[(int64_t)i * N + j] : 0.f;
+              C[(int64_t)i * N + j] = alpha * acc[mt][nt][q] + beta * prev;
+            }
+          }
+      __syncthreads();
     }
-  __syncthreads();
 }
 
 __global__ void __launch_bounds__(kNsThreads) ns_kernel(NsArgs a) {
