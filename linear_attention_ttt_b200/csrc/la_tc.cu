@@ -10,21 +10,25 @@
 // requested chunk, with (Q, K, V one tile, Vt = diag(eta) V, P = tril(Q K^T)):
 //   Y^T = S^T Q^T + Vt^T P^T          (output tile, transposed)
 //   S^T = S^T + Vt^T K                (state after the tile)
-// S^T is a 128 x 128 fp32 accumulator in tensor memory for the whole sequence:
-// the ΔS MMA accumulates into it, and the output MMA reads it directly as its
-// A operand (kind::tf32, A from TMEM), so the state never leaves tensor memory
-// and the sequential dependence stays inside the in-order MMA pipe.
+// Tensor memory (512 columns) holds, for the whole sequence:
+//   S^T   fp32, 128 lanes x 128 columns: the exact state, accumulated by MMA;
+//   S^T   bf16 copy (2 per column), the A operand of S^T Q^T, refreshed from
+//         the fp32 state after each tile;
+//   Vt^T  bf16 (2 per column), written per tile by the threads that scale V
+//         by eta, the A operand of Vt^T P^T and of the state update;
+//   the score tile Q K^T (2 buffers) and the output tile Y^T (2 buffers).
+// The A operands come from tensor memory, so the only shared-memory operands
+// are Q, K (from TMA) and P (written by the score warps).
 //
 // One CTA per (batch, head), 16 warps:
-//   warp 0      TMA producer: Q tiles into a 2-slot ring (released once the
-//               score MMA and the fp32 conversion have read them), K and V
-//               tiles into a 3-stage ring (released when the tile's MMAs are
-//               done), L2 prefetch further ahead; eta to smem
+//   warp 0      TMA producer: Q, K, V tiles into a 4-stage ring (plus L2
+//               prefetch further ahead); eta to smem
 //   warp 1      TMEM owner; one thread issues all tcgen05.mma
-//   warps 2-7   converters: fp32 copy of Q (the tf32 B operand)
-//   warps 8-11  score epilogue: P = tril(scores) -> bf16 smem, Vt = eta * V in place
-//   warps 12-15 output epilogue: S^T init from W0, Y tiles (staged in smem, then
-//               stored as 16-byte row pieces), W_final
+//   warps 4-7   Vt^T into tensor memory (eta * V, transposed by lane = dv)
+//   warps 8-11  score epilogue: P = tril(scores) -> bf16 smem
+//   warps 12-15 state/output warps: S^T init from W0, the bf16 refresh of S^T
+//               after each tile, Y tiles (staged in smem, stored as 16-byte
+//               row pieces), W_final
 // Every barrier wait is bounded (%globaltimer); a timeout is recorded in the
 // device status word and the kernel returns.
 #include "common.cuh"
@@ -36,27 +40,29 @@ namespace {
 
 constexpr int D = 128;         // dk = dv
 constexpr int TT = 64;         // tokens per tile
-constexpr int kStages = 3;     // Q/K/V ring
+constexpr int kStages = 4;     // Q/K/V ring
 constexpr int kThreads = 512;
-constexpr int kConvWarps = 6;
-constexpr int kEpiWarp0 = 8;    // score epilogue warps 8-11
-constexpr int kOutWarp0 = 12;   // output epilogue warps 12-15
+constexpr int kVtWarp0 = 4, kScWarp0 = 8, kOutWarp0 = 12;
 constexpr int kL2Ahead = 4;    // tiles prefetched into L2 ahead of the smem ring
 constexpr uint32_t kTileBytes = TT * D * 2;   // one bf16 [64 x 128] tile, 16 KB
 
-// TMEM columns: S^T [0,128), scores [128,256) (2 x 64), Y^T [256,384) (2 x 64)
-constexpr uint32_t kColS = 0, kColSc = 128, kColY = 256, kTmemCols = 512;
+// TMEM columns
+constexpr uint32_t kColS = 0;      // S^T fp32            [0, 128)
+constexpr uint32_t kColSb = 128;   // S^T bf16 pairs       [128, 192)
+constexpr uint32_t kColSc = 192;   // scores, 2 x 64       [192, 320)
+constexpr uint32_t kColY = 320;    // Y^T, 2 x 64          [320, 448)
+constexpr uint32_t kColVt = 448;   // Vt^T bf16 pairs 2x32 [448, 512)
+constexpr uint32_t kTmemCols = 512;
 
 struct Smem {
-  alignas(1024) uint8_t q[2][kTileBytes];          // Q ring, 2 boxes [64 t][64 d], 128B swizzle
-  alignas(1024) uint8_t k[kStages][kTileBytes];    // K/V ring
-  alignas(1024) uint8_t v[kStages][kTileBytes];    // becomes eta * V in place
-  alignas(1024) uint8_t q32[2][TT * D * 4];        // 4 boxes [64 t][32 d] fp32
+  alignas(1024) uint8_t q[kStages][kTileBytes];    // 2 boxes [64 t][64 d], 128B swizzle
+  alignas(1024) uint8_t k[kStages][kTileBytes];
+  alignas(1024) uint8_t v[kStages][kTileBytes];
   alignas(1024) uint8_t p[2][TT * TT * 2];         // [64 t][64 i] bf16, 128B swizzle
   alignas(1024) __nv_bfloat16 ystage[TT * D];      // output tile [t][dv]
   float eta[kStages][TT];
-  uint64_t full_q[2], q_free[2], full[kStages], conv[kStages], stage_free[kStages];
-  uint64_t sc_full[2], p_ready[2], y_full[2], y_free[2], done;
+  uint64_t full[kStages], stage_free[kStages];
+  uint64_t sc_full[2], p_ready[2], vt_ready[2], y_full[2], y_free[2], s_ready, done;
   uint32_t tmem_base;
 };
 
@@ -76,6 +82,40 @@ __device__ __forceinline__ uint32_t swz(int r, int c16) {
   return r * 128 + ((c16 ^ (r & 7)) << 4);
 }
 
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// 32 lanes x 32 consecutive 32-bit TMEM columns from 32 registers.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+      "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+      "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+      "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// bf16 copy of the fp32 state row held by this lane (128 columns -> 64 pairs).
+__device__ __forceinline__ void refresh_state_copy(uint32_t tmem_lane) {
+  for (int half = 0; half < 2; ++half) {
+    uint32_t pk[32];
+#pragma unroll
+    for (int c = 0; c < 64; c += 16) {
+      float v[16];
+      umma::tmem_ld16(tmem_lane + kColS + 64 * half + c, v);
+#pragma unroll
+      for (int u = 0; u < 16; u += 2) pk[(c + u) / 2] = pack2(v[u], v[u + 1]);
+    }
+    tmem_st32(tmem_lane + kColSb + 32 * half, pk);
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1) la_tc_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -87,19 +127,16 @@ __global__ void __launch_bounds__(kThreads, 1) la_tc_kernel(const __grid_constan
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.conv[s], kConvWarps);
       mbar_init(&sm.stage_free[s], 1);
-    }
-    for (int x = 0; x < 2; ++x) {
-      mbar_init(&sm.full_q[x], 1);
-      mbar_init(&sm.q_free[x], 1 + kConvWarps);  // score MMAs done + every converter warp
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(&sm.sc_full[x], 1);
       mbar_init(&sm.p_ready[x], 4);
+      mbar_init(&sm.vt_ready[x], 4);
       mbar_init(&sm.y_full[x], 1);
       mbar_init(&sm.y_free[x], 4);
     }
+    mbar_init(&sm.s_ready, 4);
     mbar_init(&sm.done, 1);
     fence_mbar_init();
   }
@@ -109,20 +146,22 @@ __global__ void __launch_bounds__(kThreads, 1) la_tc_kernel(const __grid_constan
   umma::fence_after();
   const uint32_t tmem = sm.tmem_base;
 
-  // S^T <- W0^T (output warps; lane = dv row r, columns = dk)
+  // S^T <- W0^T in fp32 and its bf16 copy (state warps; lane = dv row r)
   if (warp >= kOutWarp0) {
     const int q4 = warp & 3, r = q4 * 32 + lane;
+    const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
     const float* W0 = p.W0 + b * p.w0_sb + (int64_t)h * D * D;
     for (int c = 0; c < D; c += 16) {
       float v[16];
 #pragma unroll
       for (int u = 0; u < 16; ++u) v[u] = W0[(int64_t)(c + u) * D + r];
-      umma::tmem_st16(tmem + ((uint32_t)(q4 * 32) << 16) + kColS + c, v);
+      umma::tmem_st16(tl + kColS + c, v);
     }
+    refresh_state_copy(tl);
+    umma::fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.s_ready);  // phase 0: S_0
   }
-  umma::fence_before();
-  __syncthreads();
-  umma::fence_after();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -130,15 +169,26 @@ __global__ void __launch_bounds__(kThreads, 1) la_tc_kernel(const __grid_constan
       prefetch_tmap(&p.tq);
       prefetch_tmap(&p.tk);
       prefetch_tmap(&p.tv);
-    }
-    const float* eta = p.eta.p + b * p.eta.sb + h * p.eta.sh;
-    if (lane == 0)
       for (int j = 0; j < kL2Ahead && j < ntiles; ++j)
         for (int x = 0; x < 2; ++x) {
           tma_prefetch_l2_4d(&p.tq, 64 * x, j * TT, h, b);
           tma_prefetch_l2_4d(&p.tk, 64 * x, j * TT, h, b);
           tma_prefetch_l2_4d(&p.tv, 64 * x, j * TT, h, b);
         }
+    }
+    // eta of the next 4 tiles stays in flight in registers (2 values per lane
+    // per tile), so no tile waits for a global load of its learning rates.
+    const float* eta = p.eta.p + b * p.eta.sb + h * p.eta.sh;
+    auto load_eta = [&](int j, float& e0, float& e1) {
+      const int t = j * TT + lane;
+      e0 = (j < ntiles && t < p.T) ? eta[(int64_t)t * p.eta.st] : 0.f;
+      e1 = (j < ntiles && t + 32 < p.T) ? eta[(int64_t)(t + 32) * p.eta.st] : 0.f;
+    };
+    float r0a, r0b, r1a, r1b, r2a, r2b, r3a, r3b;
+    load_eta(0, r0a, r0b);
+    load_eta(1, r1a, r1b);
+    load_eta(2, r2a, r2b);
+    load_eta(3, r3a, r3b);
     for (int j = 0; j < ntiles; ++j) {
       const int s = j % kStages;
       if (lane == 0 && j + kL2Ahead < ntiles)
@@ -147,22 +197,18 @@ __global__ void __launch_bounds__(kThreads, 1) la_tc_kernel(const __grid_constan
           tma_prefetch_l2_4d(&p.tk, 64 * x, (j + kL2Ahead) * TT, h, b);
           tma_prefetch_l2_4d(&p.tv, 64 * x, (j + kL2Ahead) * TT, h, b);
         }
-      const int t0 = j * TT;
-      const int xq = j & 1;
-      if (j >= 2 && !mbar_wait(&sm.q_free[xq], ((j >> 1) - 1) & 1, p.status)) return;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&sm.full_q[xq], kTileBytes);
-        for (int x = 0; x < 2; ++x)
-          tma_load_4d(sm.q[xq] + x * 8192, &p.tq, &sm.full_q[xq], 64 * x, t0, h, b);
-      }
       if (j >= kStages && !mbar_wait(&sm.stage_free[s], ((j / kStages) - 1) & 1, p.status))
         return;
-      for (int i = lane; i < TT; i += 32)
-        sm.eta[s][i] = (t0 + i < p.T) ? eta[(int64_t)(t0 + i) * p.eta.st] : 0.f;
+      const int t0 = j * TT;
+      sm.eta[s][lane] = r0a;
+      sm.eta[s][lane + 32] = r0b;
+      r0a = r1a, r0b = r1b, r1a = r2a, r1b = r2b, r2a = r3a, r2b = r3b;
+      load_eta(j + 4, r3a, r3b);
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive_expect_tx(&sm.full[s], 2 * kTileBytes);
+        mbar_arrive_expect_tx(&sm.full[s], 3 * kTileBytes);
         for (int x = 0; x < 2; ++x) {
+          tma_load_4d(sm.q[s] + x * 8192, &p.tq, &sm.full[s], 64 * x, t0, h, b);
           tma_load_4d(sm.k[s] + x * 8192, &p.tk, &sm.full[s], 64 * x, t0, h, b);
           tma_load_4d(sm.v[s] + x * 8192, &p.tv, &sm.full[s], 64 * x, t0, h, b);
         }
@@ -171,22 +217,18 @@ __global__ void __launch_bounds__(kThreads, 1) la_tc_kernel(const __grid_constan
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t id_sc = umma::instr_desc(1, TT, TT, 0, 0);    // Q K^T
-      const uint32_t id_yq = umma::instr_desc(2, D, TT, 0, 0);     // S^T Q^T (tf32, A in TMEM)
-      const uint32_t id_yp = umma::instr_desc(1, D, TT, 1, 0);     // Vt^T P^T
-      const uint32_t id_ds = umma::instr_desc(1, D, D, 1, 1);      // Vt^T K
+      const uint32_t id_sc = umma::instr_desc(1, TT, TT, 0, 0);   // Q K^T            (M=64)
+      const uint32_t id_y = umma::instr_desc(1, D, TT, 0, 0);     // S^T Q^T, Vt^T P^T (A in TMEM)
+      const uint32_t id_ds = umma::instr_desc(1, D, D, 0, 1);     // Vt^T K           (A in TMEM)
       auto issue_scores = [&](int j, bool block) -> int {  // 1 issued, 0 not ready, -1 timeout
         const int s = j % kStages;
         if (block) {
-          if (!mbar_wait(&sm.full[s], (j / kStages) & 1, p.status) ||
-              !mbar_wait(&sm.full_q[j & 1], (j >> 1) & 1, p.status))
-            return -1;
-        } else if (!mbar_try_wait(&sm.full[s], (j / kStages) & 1) ||
-                   !mbar_try_wait(&sm.full_q[j & 1], (j >> 1) & 1)) {
+          if (!mbar_wait(&sm.full[s], (j / kStages) & 1, p.status)) return -1;
+        } else if (!mbar_try_wait(&sm.full[s], (j / kStages) & 1)) {
           return 0;
         }
         umma::fence_after();
-        const uint32_t qa = smem_u32(sm.q[j & 1]), ka = smem_u32(sm.k[s]);
+        const uint32_t qa = smem_u32(sm.q[s]), ka = smem_u32(sm.k[s]);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 8192 + (kk & 3) * 32;
@@ -194,43 +236,42 @@ __global__ void __launch_bounds__(kThreads, 1) la_tc_kernel(const __grid_constan
                          umma::smem_desc(ka + off, 16, 1024), id_sc, kk > 0);
         }
         umma::commit(&sm.sc_full[j & 1]);
-        umma::commit(&sm.q_free[j & 1]);
         return 1;
       };
       bool ok = true;
       int issued = 0;  // score tiles issued so far
       for (int j = 0; j < ntiles && ok; ++j) {
         const int s = j % kStages, x = j & 1;
-        // the epilogue needs scores of tiles j and j+1 in flight
+        // the score epilogue needs the scores of tiles j and j+1 in flight
         while (ok && issued < j + 2 && issued < ntiles) {
           ok = issue_scores(issued, true) > 0;
           ++issued;
         }
         if (!ok) break;
         ok = mbar_wait(&sm.p_ready[x], (j >> 1) & 1, p.status) &&
-             mbar_wait(&sm.conv[s], (j / kStages) & 1, p.status) &&
+             mbar_wait(&sm.vt_ready[x], (j >> 1) & 1, p.status) &&
+             mbar_wait(&sm.s_ready, j & 1, p.status) &&
              (j < 2 || mbar_wait(&sm.y_free[x], ((j - 2) >> 1) & 1, p.status));
         if (!ok) break;
         umma::fence_after();
         const uint32_t dY = tmem + kColY + x * TT;
-        const uint32_t q32 = smem_u32(sm.q32[x]), va = smem_u32(sm.v[s]),
-                       pa = smem_u32(sm.p[x]), ka = smem_u32(sm.k[s]);
-        // Y^T = S^T Q^T   (tf32, K = 128 in steps of 8; Q32 boxes of 32 columns)
+        const uint32_t vt = tmem + kColVt + x * 32;
+        const uint32_t qa = smem_u32(sm.q[s]), pa = smem_u32(sm.p[x]), ka = smem_u32(sm.k[s]);
+        // Y^T = S^T Q^T   (A = bf16 state copy in TMEM, K = 128 in steps of 16)
 #pragma unroll
-        for (int kk = 0; kk < D / 8; ++kk)
-          umma::mma_tf32_tmem_a(dY, tmem + kColS + 8 * kk,
-                                umma::smem_desc(q32 + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
-                                id_yq, kk > 0);
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma::mma_bf16_tmem_a(dY, tmem + kColSb + 8 * kk,
+                                umma::smem_desc(qa + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
+                                id_y, kk > 0);
         // Y^T += Vt^T P^T   (K = 64 tokens i)
 #pragma unroll
         for (int kk = 0; kk < TT / 16; ++kk)
-          umma::mma_bf16(dY, umma::smem_desc(va + kk * 2048, 8192, 1024),
-                         umma::smem_desc(pa + kk * 32, 16, 1024), id_yp, 1);
-        // S^T += Vt^T K   (K = 64 tokens)
+          umma::mma_bf16_tmem_a(dY, vt + 8 * kk, umma::smem_desc(pa + kk * 32, 16, 1024), id_y, 1);
+        // S^T += Vt^T K   (K = 64 tokens; K tile read MN-major)
 #pragma unroll
         for (int kk = 0; kk < TT / 16; ++kk)
-          umma::mma_bf16(tmem + kColS, umma::smem_desc(va + kk * 2048, 8192, 1024),
-                         umma::smem_desc(ka + kk * 2048, 8192, 1024), id_ds, 1);
+          umma::mma_bf16_tmem_a(tmem + kColS, vt + 8 * kk,
+                                umma::smem_desc(ka + kk * 2048, 8192, 1024), id_ds, 1);
         umma::commit(&sm.y_full[x]);
         umma::commit(&sm.stage_free[s]);
         if (issued == j + 2 && issued < ntiles) {
@@ -241,44 +282,33 @@ __global__ void __launch_bounds__(kThreads, 1) la_tc_kernel(const __grid_constan
       }
       umma::commit(&sm.done);
     }
-  } else if (warp < kEpiWarp0) {
-    // ------------------------------------------------------------ converters
-    const int ct = threadIdx.x - 64;  // 0 .. 32*kConvWarps-1
-    constexpr int NC = 32 * kConvWarps;
+  } else if (warp >= kVtWarp0 && warp < kScWarp0) {
+    // ------------------------------------------------------------ Vt^T -> TMEM
+    const int q4 = warp & 3, r = q4 * 32 + lane;   // dv row
+    const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
+    // column r of the V tile: box r / 64, 16-byte chunk (r % 64) / 8, byte 2 * (r % 8)
+    const uint32_t box = (uint32_t)(r >> 6) * 8192, chunk = (r & 63) >> 3, byte = (r & 7) * 2;
     for (int j = 0; j < ntiles; ++j) {
       const int s = j % kStages, x = j & 1;
-      if (!mbar_wait(&sm.full_q[x], (j >> 1) & 1, p.status)) return;
-      // the fp32-Q buffer of tile j-2 is free once that tile's MMAs are done
+      if (!mbar_wait(&sm.full[s], (j / kStages) & 1, p.status)) return;
+      // the Vt^T buffer of tile j-2 is free once that tile's MMAs are done
       if (j >= 2 && !mbar_wait(&sm.y_full[x], ((j - 2) >> 1) & 1, p.status)) return;
-      // Q (bf16, 2 boxes of 64 cols) -> Q32 (fp32, 4 boxes of 32 cols): 8 columns per item
-      for (int it = ct; it < TT * 16; it += NC) {
-        const int r = it >> 4, g = it & 15;   // row, group of 8 columns
-        const int col = g * 8;
-        const uint4 a = *reinterpret_cast<const uint4*>(sm.q[x] + (col >> 6) * 8192 +
-                                                        swz(r, (col & 63) >> 3));
-        const uint32_t w[4] = {a.x, a.y, a.z, a.w};
-        float4 lo, hi;
-        lo.x = __uint_as_float(w[0] << 16);
-        lo.y = __uint_as_float(w[0] & 0xffff0000u);
-        lo.z = __uint_as_float(w[1] << 16);
-        lo.w = __uint_as_float(w[1] & 0xffff0000u);
-        hi.x = __uint_as_float(w[2] << 16);
-        hi.y = __uint_as_float(w[2] & 0xffff0000u);
-        hi.z = __uint_as_float(w[3] << 16);
-        hi.w = __uint_as_float(w[3] & 0xffff0000u);
-        uint8_t* dst = sm.q32[x] + (col >> 5) * 8192;
-        const int d16 = (col & 31) >> 2;
-        *reinterpret_cast<float4*>(dst + swz(r, d16)) = lo;
-        *reinterpret_cast<float4*>(dst + swz(r, d16 + 1)) = hi;
+      const uint8_t* vb = sm.v[s] + box + byte;
+      const float* et = sm.eta[s];
+      uint32_t pk[32];
+#pragma unroll 8
+      for (int i = 0; i < TT; i += 2) {
+        const float v0 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(vb + swz(i, chunk)));
+        const float v1 =
+            __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(vb + swz(i + 1, chunk)));
+        pk[i >> 1] = pack2(et[i] * v0, et[i + 1] * v1);
       }
-      umma::fence_proxy_async_smem();
+      tmem_st32(tl + kColVt + x * 32, pk);
+      umma::fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&sm.conv[s]);
-        mbar_arrive(&sm.q_free[x]);
-      }
+      if (lane == 0) mbar_arrive(&sm.vt_ready[x]);
     }
-  } else if (warp < kOutWarp0) {
+  } else if (warp >= kScWarp0 && warp < kOutWarp0) {
     // ------------------------------------------------------------ score epilogue
     const int q4 = warp & 3;
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
@@ -293,30 +323,13 @@ __global__ void __launch_bounds__(kThreads, 1) la_tc_kernel(const __grid_constan
         float v[16];
         umma::tmem_ld16(tmem + lane_base + kColSc + x * TT + c, v);
         if (lane < 16) {
-          __align__(16) __nv_bfloat16 o[16];
+          uint4 o[2];
+          uint32_t* ow = reinterpret_cast<uint32_t*>(o);
 #pragma unroll
-          for (int u = 0; u < 16; ++u) o[u] = __float2bfloat16_rn((c + u <= t) ? v[u] : 0.f);
-          *reinterpret_cast<uint4*>(prow + swz(t, c >> 3)) = reinterpret_cast<uint4*>(o)[0];
-          *reinterpret_cast<uint4*>(prow + swz(t, (c >> 3) + 1)) = reinterpret_cast<uint4*>(o)[1];
-        }
-      }
-      // Vt = eta * V in place (stage j % kStages; its data landed before the scores)
-      {
-        const int s = j % kStages;
-        const int ti = threadIdx.x - 32 * kEpiWarp0;  // 0..127
-        for (int it = ti; it < TT * 16; it += 128) {
-          const int r = it >> 4, c = it & 15;  // row, 16-byte chunk
-          uint8_t* ptr = sm.v[s] + (c >> 3) * 8192 + swz(r, c & 7);
-          uint4 a = *reinterpret_cast<uint4*>(ptr);
-          const float er = sm.eta[s][r];
-          uint32_t* w = reinterpret_cast<uint32_t*>(&a);
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            __nv_bfloat162 v2 = __floats2bfloat162_rn(er * __uint_as_float(w[u] << 16),
-                                                      er * __uint_as_float(w[u] & 0xffff0000u));
-            w[u] = *reinterpret_cast<uint32_t*>(&v2);
-          }
-          *reinterpret_cast<uint4*>(ptr) = a;
+          for (int u = 0; u < 16; u += 2)
+            ow[u / 2] = pack2((c + u <= t) ? v[u] : 0.f, (c + u + 1 <= t) ? v[u + 1] : 0.f);
+          *reinterpret_cast<uint4*>(prow + swz(t, c >> 3)) = o[0];
+          *reinterpret_cast<uint4*>(prow + swz(t, (c >> 3) + 1)) = o[1];
         }
       }
       umma::fence_before();
@@ -324,49 +337,54 @@ __global__ void __launch_bounds__(kThreads, 1) la_tc_kernel(const __grid_constan
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.p_ready[x]);
     }
-  } else {
-    // ------------------------------------------------------------ output epilogue
+  } else if (warp >= kOutWarp0) {
+    // ------------------------------------------------------------ state / output
     const int q4 = warp & 3;
-    const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
-    auto do_y = [&](int j) -> bool {
+    const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
+    const int r = q4 * 32 + lane;  // dv row
+    for (int j = 0; j < ntiles; ++j) {
       const int x = j & 1;
+      // On a timeout the warp still takes part in both named barriers below.
       const bool ok = mbar_wait(&sm.y_full[x], (j >> 1) & 1, p.status);
       umma::fence_after();
-      const int r = q4 * 32 + lane;  // dv row
+      // 1) bf16 copy of the updated state for the next tile's S^T Q^T
+      if (ok && j + 1 < ntiles) {
+        refresh_state_copy(tl);
+        umma::fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.s_ready);
+      }
+      // 2) Y^T tile -> [t][dv] bf16 staging -> 16-byte row pieces
       const int t0 = j * TT;
       __nv_bfloat16* st = sm.ystage;
       for (int c = 0; c < TT && ok; c += 16) {
         float v[16];
-        umma::tmem_ld16(tmem + lane_base + kColY + x * TT + c, v);
+        umma::tmem_ld16(tl + kColY + x * TT + c, v);
 #pragma unroll
         for (int u = 0; u < 16; ++u) st[(c + u) * D + r] = __float2bfloat16_rn(v[u]);
       }
       umma::fence_before();
-      asm volatile("bar.sync 1, 128;" ::: "memory");  // the 4 output warps
+      asm volatile("bar.sync 1, 128;" ::: "memory");  // the 4 state/output warps
       if (lane == 0) mbar_arrive(&sm.y_free[x]);       // TMEM tile read
-      // 64 rows x 256 bytes: each thread stores 16-byte pieces of whole rows
-      const int ti = threadIdx.x - 32 * kOutWarp0;  // 0..127
+      const int ti = threadIdx.x - 32 * kOutWarp0;     // 0..127
       __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out.p) + b * p.out.sb + h * p.out.sh;
       for (int it = ti; it < TT * 16 && ok; it += 128) {
-        const int t = it >> 4, c = it & 15;
-        if (t0 + t < p.T)
-          *reinterpret_cast<uint4*>(o + (int64_t)(t0 + t) * p.out.st + c * 8) =
-              *reinterpret_cast<const uint4*>(st + t * D + c * 8);
+        const int tt = it >> 4, c = it & 15;
+        if (t0 + tt < p.T)
+          *reinterpret_cast<uint4*>(o + (int64_t)(t0 + tt) * p.out.st + c * 8) =
+              *reinterpret_cast<const uint4*>(st + tt * D + c * 8);
       }
       asm volatile("bar.sync 1, 128;" ::: "memory");  // staging buffer free again
-      return ok;
-    };
-    for (int j = 0; j < ntiles; ++j)
-      if (!do_y(j)) return;
+      if (!ok) return;
+    }
     // final state
     if (p.W_final) {
       if (!mbar_wait(&sm.done, 0, p.status)) return;
       umma::fence_after();
-      const int r = q4 * 32 + lane;
       float* Wf = p.W_final + (int64_t)bh * D * D;
       for (int c = 0; c < D; c += 16) {
         float v[16];
-        umma::tmem_ld16(tmem + lane_base + kColS + c, v);
+        umma::tmem_ld16(tl + kColS + c, v);
 #pragma unroll
         for (int u = 0; u < 16; ++u) Wf[(int64_t)(c + u) * D + r] = v[u];
       }

@@ -129,15 +129,35 @@ ttt_linear_bf16_kernel(const __grid_constant__ Params p) {
       prefetch_tmap(&p.tk);
       prefetch_tmap(&p.tv);
     }
+    // The next 4 blocks' starts and learning rates stay in flight in
+    // registers (lane l < 16 holds eta of the block's token l), so no block
+    // waits for a global load of its learning rates.
     const float* eta = p.eta.p + b * p.eta.sb + h * p.eta.sh;
-    int it = 0;
-    for (int s = 0; s < p.T; ++it) {
-      int nb;
+    int sr[4], nr[4];
+    float er[4];
+    int s_next = 0;  // start of the next block to enter the ring
+    auto fill = [&](int k) {
+      int nb = 0;
       bool ce;
-      next_block(p, s, nb, ce);
+      if (s_next < p.T) next_block(p, s_next, nb, ce);
+      sr[k] = s_next;
+      nr[k] = nb;
+      er[k] = (lane < nb) ? eta[(int64_t)(s_next + lane) * p.eta.st] : 0.f;
+      s_next += nb;
+    };
+#pragma unroll
+    for (int k = 0; k < 4; ++k) fill(k);
+    int it = 0;
+    while (nr[0] > 0) {
+      const int s = sr[0];
+      const float e = er[0];
       const int st = it % kStages;
       if (it >= kStages && !mbar_wait(&sm.empty[st], ((it / kStages) - 1) & 1, p.status)) return;
-      if (lane < kTB) sm.eta[st][lane] = lane < nb ? eta[(int64_t)(s + lane) * p.eta.st] : 0.f;
+      if (lane < kTB) sm.eta[st][lane] = e;
+      // rotate the ring and request the block after the last one in it
+#pragma unroll
+      for (int k = 0; k < 3; ++k) sr[k] = sr[k + 1], nr[k] = nr[k + 1], er[k] = er[k + 1];
+      fill(3);
       __syncwarp();
       if (lane == 0) {
         mbar_arrive_expect_tx(&sm.full[st], 3 * Smem<D>::kTile);
@@ -147,7 +167,7 @@ ttt_linear_bf16_kernel(const __grid_constant__ Params p) {
           tma_load_4d(sm.v[st] + x * 2048, &p.tv, &sm.full[st], x * 64, s, h, b);
         }
       }
-      s += nb;
+      ++it;
     }
     return;
   }
