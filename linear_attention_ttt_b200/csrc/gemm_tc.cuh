@@ -5,6 +5,9 @@
 //     D_z[M x N] = sum_seg A_seg,z[M x K] * B_seg,z[N x K]^T
 // over 1-3 "segments" (operand pairs accumulated into the same TMEM
 // accumulator; used for split-precision products hi*hi + lo*hi + hi*lo).
+// A problem may carry a second product (operands a2, b2) whose tn/2 columns
+// land beside the first product's tn columns in the same accumulator tile;
+// the fused key-side LaCT epilogue uses it for V W2 next to K [W1; W3]^T.
 // Operands are bf16 tensors read by TMA with the 128-byte swizzle, either
 // K-major (storage [rows=M|N][K]) or MN-major (storage [rows=K][M|N]).
 // Tiles are 128 x BN with a 64-wide K step. The kernel is persistent: each CTA
@@ -13,10 +16,12 @@
 // stages; warp 1 owns two TMEM accumulators and one elected thread issues
 // tcgen05.mma into them alternately; warps 2-9 run the epilogue of one
 // accumulator (two warps per 32-lane quarter of TMEM, each taking half of the
-// tile's columns) while the MMAs of the next tile fill the other. The epilogue
-// writes through TMA: each warp stages 32 rows x 16 columns in shared memory
-// and issues a tensor store (or an fp32 add-reduction for split-K gradients),
-// so global writes are full row segments. All barrier waits are bounded.
+// tile's columns) while the MMAs of the next tile fill the other. Each
+// epilogue warp stages 32 rows x 128 bytes (64 bf16 or 32 fp32 columns) in its
+// 128-byte-swizzled shared-memory buffer (conflict-free in both directions)
+// and then writes it as full 128-byte row segments, four rows per store
+// instruction; split-K gradients leave the same buffer as fp32 TMA
+// add-reductions. All barrier waits are bounded.
 #pragma once
 
 #include "common.cuh"
@@ -33,14 +38,18 @@ constexpr int kThreads = 320;   // 2 + 8 warps
 constexpr int kEpiWarps = 8;
 constexpr int kMaxProblems = 4;
 
+// W1 and W3 rows are interleaved in blocks of kHid (W13 rows: W1 0..63,
+// W3 0..63, W1 64..127, ...), so a 2*kHid-wide column range of K W13^T holds
+// h1 and h3 of the same kHid hidden units.
+constexpr int kHid = 64;
+
 enum Epi : int {
-  EPI_GZ = 0,     // gz = -eta_i * D  (fp32, lane-interleaved layout, see gz_off)
   EPI_AQ = 1,     // aq = silu(h1) * h3                  (bf16 hi [+lo])
-  EPI_HK = 2,     // ak = eta*silu(h1)*h3, dh3 = gz*silu(h1), dh1 = gz*h3*silu'(h1)
-                  // (for both, a BN-wide tile holds BN/2 h1 columns, then the
-                  //  BN/2 matching h3 columns)
+  EPI_HKG = 2,    // tile [h1 | h3 | u] for kHid hidden units, u = (V W2) columns,
+                  // gz = -eta_i u:  ak = eta*silu(h1)*h3, dh3 = gz*silu(h1),
+                  // dh1 = gz*h3*silu'(h1)                 (bf16 hi [+lo])
   EPI_Y = 3,      // out tokens = D                      (bf16 or fp32, strided)
-  EPI_GRAD = 4,   // g[z][m][n] += scale * D             (fp32 atomics, split-K)
+  EPI_GRAD = 4,   // g[z][m][n] += scale * D             (fp32 TMA add, split-K)
 };
 
 struct Operand {
@@ -51,16 +60,16 @@ struct Operand {
 };
 
 struct EpiArgs {
-  // TMA maps of the outputs, boxes of {16 columns, 32 rows, 1, 1}:
-  //  EPI_AQ: omap[0] aq hi, [3] aq lo; EPI_HK: omap[0..2] ak, dh1, dh3 hi, [3..5] lo;
-  //  EPI_Y: omap[0] output tokens {dv, T, H, B}; EPI_GRAD: omap[0] g {N, M, Z, 1}.
-  CUtensorMap omap[6];
+  // EPI_GRAD: TMA map of g {N, M, Z, 1} fp32, box {32, 32, 1, 1}, 128-byte swizzle.
+  CUtensorMap gmap;
+  // bf16 activation outputs [Z][orows][ocols] (row-major):
+  //  EPI_AQ: optr[0] aq hi, [3] aq lo; EPI_HKG: optr[0..2] ak, dh1, dh3 hi, [3..5] lo.
+  void* optr[6];
+  int64_t orows;
+  int ocols;
   int nsplit;              // 1 or 2 (bf16 outputs with residuals)
-  int ozdiv;               // z -> (z % ozdiv, z / ozdiv) for output coords 2, 3
+  int ozdiv;               // EPI_GRAD: z -> (z % ozdiv, z / ozdiv) for map coords 2, 3
   int orow0;               // output row offset (chunk start for EPI_Y)
-  float* gz;               // EPI_GZ destination / EPI_HK source
-  int64_t gz_rows;         // rows per z of the gz layout (allocated chunk length)
-  int gz_cols;             // hidden units
   EtaView eta;             // per-token learning rates
   int eta_t0;              // chunk start (token index of row 0)
   int H;                   // heads (z = b * H + h)
@@ -72,9 +81,11 @@ struct EpiArgs {
 
 struct Problem {
   Operand a, b;
-  int M, N, K;      // K per segment
-  int nseg;
-  int seg_a[3], seg_b[3];
+  Operand a2, b2;   // second product (nseg2 > 0): tn/2 columns at accumulator column tn
+  int M, N, K;      // K per segment (both products)
+  int tn;           // tile width in columns of the first product (<= BN)
+  int nseg, nseg2;
+  int seg_a[3], seg_b[3], seg2_a[3], seg2_b[3];
   int nz, ksplit, mtiles, ntiles, tile_begin;
   int epi;
   EpiArgs e;
@@ -91,65 +102,123 @@ template <int BN>
 struct Smem {
   alignas(1024) uint8_t a[kStages][BM * BK * 2];
   alignas(1024) uint8_t b[kStages][BN * BK * 2];
-  alignas(128) float ostage[kEpiWarps][2][32 * 16];  // per-warp TMA store staging (x2)
+  alignas(1024) uint8_t ostage[kEpiWarps][32 * 128];  // per-warp staging, swizzled
   uint64_t full[kStages], empty[kStages], acc_full[2], acc_empty[2];
   uint32_t tmem_base;
 };
 
-// Offset of gz element (z, row, col) in the lane-interleaved layout
-// [z][col/16][row][16]: 32 consecutive rows x 16 columns are 2 KB contiguous,
-// so a warp (one row per lane) reads or writes them fully coalesced.
-__device__ __forceinline__ int64_t gz_off(const EpiArgs& e, int z, int row, int col) {
-  return ((((int64_t)z * (e.gz_cols / 16) + col / 16) * e.gz_rows + row) << 4) + (col & 15);
+// Per-warp staging buffers of 32 rows x 128 bytes with the 128-byte swizzle:
+// 16-byte chunk j of row r sits at r * 128 + ((j ^ (r & 7)) << 4), so a lane
+// writing its own row and eight lanes reading one row both hit 32 distinct
+// banks per 128 bytes.
+__device__ __forceinline__ uint32_t sw128(int r, int j) {
+  return (uint32_t)(r * 128 + ((j ^ (r & 7)) << 4));
 }
 
-// Per-warp TMA output staging: lane = tile row, 16 columns per store.
-struct Stager {
-  float* buf[2];
-  int lane, next;
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
 
-  __device__ __forceinline__ void* slot() {
-    // the slot about to be rewritten was used two stores ago
-    if (lane == 0) bulk_wait_read<1>();
-    __syncwarp();
-    return buf[next];
+// Row `lane` of the buffer, columns [16p, 16p + 16) as bf16 (chunks 2p, 2p+1):
+// bf16(v), or the residual v - bf16(v) when lo.
+__device__ __forceinline__ void put_bf16(uint8_t* s, int lane, int p, const float (&v)[16],
+                                         bool lo) {
+  uint32_t w[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    float a = v[2 * u], b = v[2 * u + 1];
+    if (lo) {
+      a -= __bfloat162float(__float2bfloat16_rn(a));
+      b -= __bfloat162float(__float2bfloat16_rn(b));
+    }
+    w[u] = pack_bf16x2(a, b);
   }
-  __device__ __forceinline__ void issue(const CUtensorMap* m, void* src, int c0, int c1, int c2,
-                                        int c3, bool reduce) {
+  *reinterpret_cast<uint4*>(s + sw128(lane, 2 * p)) = make_uint4(w[0], w[1], w[2], w[3]);
+  *reinterpret_cast<uint4*>(s + sw128(lane, 2 * p + 1)) = make_uint4(w[4], w[5], w[6], w[7]);
+}
+// Row `lane`, fp32 columns [16p, 16p + 16) (chunks 4p .. 4p+3).
+__device__ __forceinline__ void put_f32(uint8_t* s, int lane, int p, const float (&v)[16]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    *reinterpret_cast<float4*>(s + sw128(lane, 4 * p + q)) =
+        make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+}
+__device__ __forceinline__ void get_f32(const uint8_t* s, int lane, int p, float* v) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float4 t = *reinterpret_cast<const float4*>(s + sw128(lane, 4 * p + q));
+    v[4 * q] = t.x, v[4 * q + 1] = t.y, v[4 * q + 2] = t.z, v[4 * q + 3] = t.w;
+  }
+}
+// Staged rows r < nrows -> dst + r * ld (bytes): each store instruction
+// writes four complete 128-byte rows.
+__device__ __forceinline__ void flush_rows(const uint8_t* s, int lane, uint8_t* dst, int64_t ld,
+                                           int nrows) {
+  __syncwarp();
+  uint4 x[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) x[i] = *reinterpret_cast<const uint4*>(s + sw128(4 * i + (lane >> 3), lane & 7));
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int r = 4 * i + (lane >> 3);
+    if (r < nrows) *reinterpret_cast<uint4*>(dst + r * ld + (lane & 7) * 16) = x[i];
+  }
+  __syncwarp();
+}
+// Rows r < nrows of src + r * ld (128 bytes each) -> staging (zeros beyond).
+__device__ __forceinline__ void fill_rows(uint8_t* s, int lane, const uint8_t* src, int64_t ld,
+                                          int nrows) {
+  __syncwarp();
+  uint4 x[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int r = 4 * i + (lane >> 3);
+    x[i] = r < nrows ? *reinterpret_cast<const uint4*>(src + r * ld + (lane & 7) * 16)
+                     : make_uint4(0, 0, 0, 0);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) *reinterpret_cast<uint4*>(s + sw128(4 * i + (lane >> 3), lane & 7)) = x[i];
+  __syncwarp();
+}
+
+// The staging buffer of one epilogue warp. Synchronous use (stage, then
+// flush_rows) needs no bookkeeping; a TMA add-reduction reads the buffer
+// asynchronously, so the buffer is rewritten only after that read is done.
+struct Stage {
+  uint8_t* buf;
+  int lane;
+  bool pending;  // a TMA read may still be in flight (warp-uniform)
+
+  __device__ __forceinline__ void drain() {
+    if (pending) {
+      if (lane == 0) bulk_wait_read<0>();
+      __syncwarp();
+      pending = false;
+    }
+  }
+  __device__ __forceinline__ void reduce(const CUtensorMap* m, int c0, int c1, int c2, int c3) {
     umma::fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-      if (reduce)
-        tma_reduce_add_4d(m, src, c0, c1, c2, c3);
-      else
-        tma_store_4d(m, src, c0, c1, c2, c3);
+      tma_reduce_add_4d(m, buf, c0, c1, c2, c3);
       bulk_commit();
     }
-    next ^= 1;
-  }
-  __device__ __forceinline__ void f32(const CUtensorMap* m, const float (&v)[16], int c0, int c1,
-                                      int c2, int c3, bool reduce) {
-    float* d = static_cast<float*>(slot()) + lane * 16;
-#pragma unroll
-    for (int u = 0; u < 16; u += 4)
-      *reinterpret_cast<float4*>(d + u) = make_float4(v[u], v[u + 1], v[u + 2], v[u + 3]);
-    issue(m, d - lane * 16, c0, c1, c2, c3, reduce);
-  }
-  // bf16 of v (lo = false) or of the residual v - bf16(v) (lo = true)
-  __device__ __forceinline__ void bf16(const CUtensorMap* m, const float (&v)[16], bool lo, int c0,
-                                       int c1, int c2, int c3) {
-    __nv_bfloat16* d = static_cast<__nv_bfloat16*>(slot()) + lane * 16;
-    __align__(16) __nv_bfloat16 o[16];
-#pragma unroll
-    for (int u = 0; u < 16; ++u) {
-      const __nv_bfloat16 h = __float2bfloat16_rn(v[u]);
-      o[u] = lo ? __float2bfloat16_rn(v[u] - __bfloat162float(h)) : h;
-    }
-    reinterpret_cast<uint4*>(d)[0] = reinterpret_cast<const uint4*>(o)[0];
-    reinterpret_cast<uint4*>(d)[1] = reinterpret_cast<const uint4*>(o)[1];
-    issue(m, d - lane * 16, c0, c1, c2, c3, false);
+    pending = true;
   }
 };
+
+// Two 16-column TMEM loads in flight, then one wait.
+__device__ __forceinline__ void tmem_ld2x16(uint32_t ta, uint32_t tb, float (&a)[16],
+                                            float (&b)[16]) {
+  uint32_t ra[16], rb[16];
+  umma::tmem_ld16_async(ta, ra);
+  umma::tmem_ld16_async(tb, rb);
+  umma::tmem_wait_ld(ra);
+  umma::tmem_wait_ld(rb);
+#pragma unroll
+  for (int u = 0; u < 16; ++u) a[u] = __uint_as_float(ra[u]), b[u] = __uint_as_float(rb[u]);
+}
 
 
 struct TileCoord {
@@ -170,11 +239,14 @@ __device__ __forceinline__ TileCoord decode_tile(const Params& P, int t) {
   c.ks = local % pr.ksplit;
   c.z = local / pr.ksplit;
   c.m0 = mt * BM;
-  c.n0 = nt;  // n-tile index; the kernel scales it by BN
+  c.n0 = nt;  // n-tile index; the kernel scales it by the problem's tile width
   return c;
 }
 
-__device__ __forceinline__ float sigmoidf_(float x) { return __frcp_rn(1.f + __expf(-x)); }
+// Logistic function from the fast exponential and the approximate division
+// (relative error ~1e-7; 1 / inf = 0 for very negative x). A correctly rounded
+// reciprocal costs about ten times as much and dominated the epilogues.
+__device__ __forceinline__ float sigmoidf_(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
 
 // Epilogue for 16 consecutive accumulator columns [c0, c0+16) of row `row` of
 // tile (m0, n0). For EPI_AQ / EPI_HK the tile's 128 columns hold 64 columns of
@@ -196,93 +268,155 @@ __device__ __forceinline__ void k_range(const Problem& pr, int ks, int& kb0, int
 
 // Epilogue of one accumulator tile, run by one warp: its 32 TMEM lanes (tile
 // rows quarter*32 ...) and the columns of half `ch` (0 or 1) of the tile.
-// Rows and columns outside an output tensor are clipped by TMA; rows between
-// the chunk end and the tensor end may receive values that the caller's later
-// work overwrites or never reads.
+// Rows at or beyond min(M, rows_valid) are not written.
 template <int BN>
 __device__ __forceinline__ void epilogue_tile(const Problem& pr, const TileCoord& tc, int quarter,
-                                              uint32_t tbase, bool live_tile, int ch, Stager& sg) {
+                                              uint32_t tbase, bool live_tile, int ch, Stage& sg) {
   const EpiArgs& e = pr.e;
-  const int z = tc.z, n0 = tc.n0 * BN;
+  const int z = tc.z, n0 = tc.n0 * pr.tn;
   const int row0 = tc.m0 + quarter * 32;  // first tile row of this warp
   const int lim = min(pr.M, e.rows_valid);
-  const bool live = live_tile && row0 < lim;    // warp-uniform
-  const int grow = row0 + sg.lane;
-  const bool lane_ok = grow < lim;              // this lane's row exists
-  const int oz2 = z % e.ozdiv, oz3 = z / e.ozdiv;
-  if (pr.epi == EPI_AQ || pr.epi == EPI_HK) {
-    constexpr int HALF = BN / 2;
-    const int hid0 = n0 / 2;  // first hidden unit of this tile
-    float eta_i = 0.f;
-    if (live && pr.epi == EPI_HK && lane_ok) eta_i = eta_of(e, z, grow);
-    for (int c = ch * (HALF / 2); c < (ch + 1) * (HALF / 2); c += 16) {
-      float h1[16], h3[16];
-      umma::tmem_ld16(tbase + c, h1);
-      umma::tmem_ld16(tbase + HALF + c, h3);
-      if (!live) continue;
-      const int col = hid0 + c;
-      float sgm[16], s1[16];
+  if (!live_tile || row0 >= lim) return;   // warp-uniform
+  const int nrows = min(32, lim - row0);
+  const int lane = sg.lane;
+  const bool lane_ok = lane < nrows;       // this lane's row exists
+  uint8_t* const buf = sg.buf;
+  sg.drain();
+  // 64 bf16 columns of this warp's rows: values of columns [16p, 16p + 16)
+  // from val(p, v), staged as bf16 (or residuals when lo), then written.
+  auto emit = [&](uint8_t* d, int64_t ld, bool lo, auto&& val) {
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      float v[16];
+      val(p, v);
+      put_bf16(buf, lane, p, v, lo);
+    }
+    flush_rows(buf, lane, d, ld, nrows);
+  };
+
+  if (pr.epi == EPI_AQ || pr.epi == EPI_HKG) {
+    const int64_t ld = (int64_t)e.ocols * 2;
+    const bool split = e.nsplit > 1;
+    if (pr.epi == EPI_AQ) {
+      // tile columns [128ch, 128ch + 64) h1, [128ch + 64, 128ch + 128) h3
+      const int c0 = ch * 2 * kHid;
+      const int hid = n0 / 2 + ch * kHid;
+      auto aq = [&](int p, float (&a)[16]) {
+        float h1[16], h3[16];
+        tmem_ld2x16(tbase + c0 + 16 * p, tbase + c0 + kHid + 16 * p, h1, h3);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) a[u] = h1[u] * sigmoidf_(h1[u]) * h3[u];
+      };
+      const int64_t off = (((int64_t)z * e.orows + row0) * e.ocols + hid) * 2;
+      emit(static_cast<uint8_t*>(e.optr[0]) + off, ld, false, aq);
+      if (split) emit(static_cast<uint8_t*>(e.optr[3]) + off, ld, true, aq);
+      return;
+    }
+    // EPI_HKG: columns [0, 64) h1, [64, 128) h3, [128, 192) u of hidden units
+    // hid .. hid + 63. Warp half 0 writes ak and dh3, half 1 writes dh1.
+    const int hid = tc.n0 * kHid;
+    const float eta_i = lane_ok ? eta_of(e, z, row0 + lane) : 0.f;
+    auto dst = [&](int o) {
+      return static_cast<uint8_t*>(e.optr[o]) + (((int64_t)z * e.orows + row0) * e.ocols + hid) * 2;
+    };
+    auto load3 = [&](int p, float (&h1)[16], float (&h3)[16], float (&gz)[16]) {
+      uint32_t r1[16], r3[16], rg[16];
+      umma::tmem_ld16_async(tbase + 16 * p, r1);
+      umma::tmem_ld16_async(tbase + kHid + 16 * p, r3);
+      umma::tmem_ld16_async(tbase + 2 * kHid + 16 * p, rg);
+      umma::tmem_wait_ld(r1);
+      umma::tmem_wait_ld(r3);
+      umma::tmem_wait_ld(rg);
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
-        sgm[u] = sigmoidf_(h1[u]);
-        s1[u] = h1[u] * sgm[u];
+        h1[u] = __uint_as_float(r1[u]);
+        h3[u] = __uint_as_float(r3[u]);
+        gz[u] = -eta_i * __uint_as_float(rg[u]);
       }
-      if (pr.epi == EPI_AQ) {
-        float a[16];
+    };
+    if (ch == 0) {
+      auto ak = [&](int p, float (&v)[16]) {  // eta * silu(h1) * h3
+        float h1[16], h3[16];
+        tmem_ld2x16(tbase + 16 * p, tbase + kHid + 16 * p, h1, h3);
 #pragma unroll
-        for (int u = 0; u < 16; ++u) a[u] = s1[u] * h3[u];
-        for (int x = 0; x < e.nsplit; ++x) sg.bf16(&e.omap[3 * x], a, x, col, row0, oz2, oz3);
-      } else {
-        float g[16] = {};
-        if (lane_ok) {
-          const float* gp = e.gz + gz_off(e, z, grow, col);
+        for (int u = 0; u < 16; ++u) v[u] = eta_i * h1[u] * sigmoidf_(h1[u]) * h3[u];
+      };
+      auto dh3 = [&](int p, float (&v)[16]) {  // gz * silu(h1)
+        float h1[16], h3[16], gz[16];
+        load3(p, h1, h3, gz);
 #pragma unroll
-          for (int u = 0; u < 16; u += 4) {
-            const float4 t = *reinterpret_cast<const float4*>(gp + u);
-            g[u] = t.x, g[u + 1] = t.y, g[u + 2] = t.z, g[u + 3] = t.w;
-          }
-        }
-        float ak[16], d3[16], d1[16];
+        for (int u = 0; u < 16; ++u) v[u] = gz[u] * h1[u] * sigmoidf_(h1[u]);
+      };
+      emit(dst(0), ld, false, ak);
+      if (split) emit(dst(3), ld, true, ak);
+      emit(dst(2), ld, false, dh3);
+      if (split) emit(dst(5), ld, true, dh3);
+    } else {
+      // dh1 = gz * h3 * silu'(h1),  silu'(x) = sigmoid(x) (1 + x (1 - sigmoid(x)))
+      auto dh1 = [&](int p, float (&v)[16]) {
+        float h1[16], h3[16], gz[16];
+        load3(p, h1, h3, gz);
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
-          ak[u] = eta_i * s1[u] * h3[u];
-          d3[u] = g[u] * s1[u];
-          d1[u] = g[u] * h3[u] * sgm[u] * (1.f + h1[u] * (1.f - sgm[u]));
+          const float sg1 = sigmoidf_(h1[u]);
+          v[u] = gz[u] * h3[u] * sg1 * (1.f + h1[u] * (1.f - sg1));
         }
-        for (int x = 0; x < e.nsplit; ++x) {
-          sg.bf16(&e.omap[3 * x + 0], ak, x, col, row0, oz2, oz3);
-          sg.bf16(&e.omap[3 * x + 1], d1, x, col, row0, oz2, oz3);
-          sg.bf16(&e.omap[3 * x + 2], d3, x, col, row0, oz2, oz3);
-        }
-      }
+      };
+      emit(dst(1), ld, false, dh1);
+      if (split) emit(dst(4), ld, true, dh1);
     }
     return;
   }
-  float eta_i = 0.f;
-  if (live && pr.epi == EPI_GZ && lane_ok) eta_i = eta_of(e, z, grow);
-  for (int c = ch * (BN / 2); c < (ch + 1) * (BN / 2); c += 16) {
-    float v[16];
-    umma::tmem_ld16(tbase + c, v);
-    const int gc = n0 + c;
-    if (!live || gc >= pr.N) continue;
-    if (pr.epi == EPI_GZ) {
-      if (!lane_ok) continue;
-      float* gp = e.gz + gz_off(e, z, grow, gc);
-#pragma unroll
-      for (int u = 0; u < 16; u += 4)
-        *reinterpret_cast<float4*>(gp + u) =
-            make_float4(-eta_i * v[u], -eta_i * v[u + 1], -eta_i * v[u + 2], -eta_i * v[u + 3]);
-    } else if (pr.epi == EPI_GRAD) {
+
+  if (pr.epi == EPI_GRAD) {
+    const int oz2 = z % e.ozdiv, oz3 = z / e.ozdiv;
+    for (int gi = 0; gi < pr.tn / 64; ++gi) {   // 32 fp32 columns per group
+      const int gc = n0 + ch * (pr.tn / 2) + 32 * gi;
+      if (gc >= pr.N) break;
+      float v[16], w[16];
+      tmem_ld2x16(tbase + gc - n0, tbase + gc - n0 + 16, v, w);
       if (e.scale != 1.f)
 #pragma unroll
-        for (int u = 0; u < 16; ++u) v[u] *= e.scale;
-      sg.f32(&e.omap[0], v, gc, row0, oz2, oz3, true);
-    } else {  // EPI_Y
-      if (e.out_bf16)
-        sg.bf16(&e.omap[0], v, false, gc, e.orow0 + row0, oz2, oz3);
-      else
-        sg.f32(&e.omap[0], v, gc, e.orow0 + row0, oz2, oz3, false);
+        for (int u = 0; u < 16; ++u) v[u] *= e.scale, w[u] *= e.scale;
+      sg.drain();  // the previous reduction has read the buffer
+      put_f32(buf, lane, 0, v);
+      put_f32(buf, lane, 1, w);
+      sg.reduce(&e.gmap, gc, row0, oz2, oz3);
     }
+    return;
+  }
+
+  const int b = z / e.H, h = z % e.H;
+  const int64_t es = e.out_bf16 ? 2 : 4;
+  uint8_t* base = static_cast<uint8_t*>(e.out.p) +
+                  ((int64_t)b * e.out.sb + (int64_t)h * e.out.sh +
+                   (int64_t)(e.orow0 + row0) * e.out.st) * es;
+  const int64_t ld = e.out.st * es;
+  if (!e.out_bf16) {
+    // EPI_Y, fp32 output tokens: 32 columns per group
+    for (int gi = 0; gi < pr.tn / 64; ++gi) {
+      const int gc = n0 + ch * (pr.tn / 2) + 32 * gi;
+      if (gc >= pr.N) break;
+      float v[16], w[16];
+      tmem_ld2x16(tbase + gc - n0, tbase + gc - n0 + 16, v, w);
+      put_f32(buf, lane, 0, v);
+      put_f32(buf, lane, 1, w);
+      flush_rows(buf, lane, base + (int64_t)gc * 4, ld, nrows);
+    }
+    return;
+  }
+  // EPI_Y, bf16 output tokens: 64 columns per group
+  for (int gi = 0; gi < pr.tn / 128; ++gi) {
+    const int gc = n0 + ch * (pr.tn / 2) + 64 * gi;
+    if (gc >= pr.N) break;
+    auto y = [&](int p, float (&v)[16]) {
+      uint32_t r[16];
+      umma::tmem_ld16_async(tbase + gc - n0 + 16 * p, r);
+      umma::tmem_wait_ld(r);
+#pragma unroll
+      for (int u = 0; u < 16; ++u) v[u] = __uint_as_float(r[u]);
+    };
+    emit(base + (int64_t)gc * 2, ld, false, y);
   }
 }
 
@@ -320,14 +454,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         const Problem& pr = P.p[tc.pi];
         int kb0, nk;
         k_range(pr, tc.ks, kb0, nk);
-        const Operand& A = pr.a;
-        const Operand& B = pr.b;
-        const int az2 = tc.z % A.zdiv, az3 = tc.z / A.zdiv, bz2 = tc.z % B.zdiv,
-                  bz3 = tc.z / B.zdiv;
-        const int m0 = tc.m0, n0 = tc.n0 * BN;
-        for (int seg = 0; seg < pr.nseg && ok; ++seg) {
-          const CUtensorMap* am = &A.map[pr.seg_a[seg]];
-          const CUtensorMap* bm = &B.map[pr.seg_b[seg]];
+        const int tn = pr.tn, n0 = tc.n0 * tn, m0 = tc.m0;
+        for (int seg = 0; seg < pr.nseg + pr.nseg2 && ok; ++seg) {
+          const bool second = seg >= pr.nseg;
+          const Operand& A = second ? pr.a2 : pr.a;
+          const Operand& B = second ? pr.b2 : pr.b;
+          const CUtensorMap* am = &A.map[second ? pr.seg2_a[seg - pr.nseg] : pr.seg_a[seg]];
+          const CUtensorMap* bm = &B.map[second ? pr.seg2_b[seg - pr.nseg] : pr.seg_b[seg]];
+          const int bn = second ? tn / 2 : tn;   // B rows (columns of this product)
+          const int bn0 = second ? n0 / 2 : n0;
+          const int az2 = tc.z % A.zdiv, az3 = tc.z / A.zdiv, bz2 = tc.z % B.zdiv,
+                    bz3 = tc.z / B.zdiv;
           for (int kb = kb0; kb < kb0 + nk; ++kb, ++it) {
             const int st = it % kStages;
             if (it >= kStages && !mbar_wait(&sm.empty[st], ((it / kStages) - 1) & 1, P.status)) {
@@ -335,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
               break;
             }
             const int k = kb * BK;
-            mbar_arrive_expect_tx(&sm.full[st], (BM + BN) * BK * 2);
+            mbar_arrive_expect_tx(&sm.full[st], (BM + bn) * BK * 2);
             if (!A.mn_major) {
               tma_load_4d(sm.a[st], am, &sm.full[st], k, A.row0 + m0, az2, az3);
             } else {
@@ -343,11 +480,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
               tma_load_4d(sm.a[st] + 8192, am, &sm.full[st], m0 + 64, A.row0 + k, az2, az3);
             }
             if (!B.mn_major) {
-              tma_load_4d(sm.b[st], bm, &sm.full[st], k, B.row0 + n0, bz2, bz3);
+              tma_load_4d(sm.b[st], bm, &sm.full[st], k, B.row0 + bn0, bz2, bz3);
             } else {
-#pragma unroll
-              for (int x = 0; x < BN / 64; ++x)
-                tma_load_4d(sm.b[st] + x * 8192, bm, &sm.full[st], n0 + 64 * x, B.row0 + k, bz2,
+              for (int x = 0; x < bn / 64; ++x)
+                tma_load_4d(sm.b[st] + x * 8192, bm, &sm.full[st], bn0 + 64 * x, B.row0 + k, bz2,
                             bz3);
             }
           }
@@ -364,30 +500,38 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         const Problem& pr = P.p[tc.pi];
         int kb0, nk;
         k_range(pr, tc.ks, kb0, nk);
-        const int niter = nk * pr.nseg;
         const int ab = lt & 1;
         if (lt >= 2 && !mbar_wait(&sm.acc_empty[ab], ((lt >> 1) - 1) & 1, P.status)) break;
         umma::fence_after();
         const uint32_t dacc = tmem + ab * BN;
-        const uint32_t idesc = umma::instr_desc(1, BM, BN, pr.a.mn_major, pr.b.mn_major);
-        for (int i = 0; i < niter; ++i, ++it) {
-          const int st = it % kStages;
-          if (!mbar_wait(&sm.full[st], (it / kStages) & 1, P.status)) {
-            ok = false;
-            break;
-          }
-          umma::fence_after();
-          const uint32_t sa = smem_u32(sm.a[st]), sb = smem_u32(sm.b[st]);
+        for (int seg = 0; seg < pr.nseg + pr.nseg2 && ok; ++seg) {
+          const bool second = seg >= pr.nseg;
+          const Operand& A = second ? pr.a2 : pr.a;
+          const Operand& B = second ? pr.b2 : pr.b;
+          const uint32_t d = dacc + (second ? pr.tn : 0);
+          const uint32_t idesc =
+              umma::instr_desc(1, BM, second ? pr.tn / 2 : pr.tn, A.mn_major, B.mn_major);
+          const bool first_seg = seg == 0 || seg == pr.nseg;  // accumulator starts at zero
+          for (int i = 0; i < nk; ++i, ++it) {
+            const int st = it % kStages;
+            if (!mbar_wait(&sm.full[st], (it / kStages) & 1, P.status)) {
+              ok = false;
+              break;
+            }
+            umma::fence_after();
+            const uint32_t sa = smem_u32(sm.a[st]), sb = smem_u32(sm.b[st]);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = pr.a.mn_major ? umma::smem_desc(sa + kk * 2048, 8192, 1024)
-                                              : umma::smem_desc(sa + kk * 32, 16, 1024);
-            const uint64_t bd = pr.b.mn_major ? umma::smem_desc(sb + kk * 2048, 8192, 1024)
-                                              : umma::smem_desc(sb + kk * 32, 16, 1024);
-            umma::mma_bf16(dacc, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              const uint64_t ad = A.mn_major ? umma::smem_desc(sa + kk * 2048, 8192, 1024)
+                                             : umma::smem_desc(sa + kk * 32, 16, 1024);
+              const uint64_t bd = B.mn_major ? umma::smem_desc(sb + kk * 2048, 8192, 1024)
+                                             : umma::smem_desc(sb + kk * 32, 16, 1024);
+              umma::mma_bf16(d, ad, bd, idesc, (!first_seg || i > 0 || kk > 0) ? 1u : 0u);
+            }
+            umma::commit(&sm.empty[st]);
           }
-          umma::commit(&sm.empty[st]);
         }
+        if (!ok) break;
         umma::commit(&sm.acc_full[ab]);
       }
     }
@@ -395,7 +539,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     // ---------------- epilogue: warps 2..9 ----------------
     const int quarter = warp & 3;
     const int ch = (warp - 2) >> 2;       // column half
-    Stager sgr{{sm.ostage[warp - 2][0], sm.ostage[warp - 2][1]}, lane, 0};
+    Stage sgr{sm.ostage[warp - 2], lane, false};
     int lt = 0;
     for (int t = blockIdx.x; t < P.total_tiles; t += gridDim.x, ++lt) {
       const TileCoord tc = decode_tile(P, t);

@@ -176,8 +176,9 @@ __global__ void __launch_bounds__(kThreads, 1) la_tc_kernel(const __grid_constan
           tma_prefetch_l2_4d(&p.tv, 64 * x, j * TT, h, b);
         }
     }
-    // eta of the next 4 tiles stays in flight in registers (2 values per lane
-    // per tile), so no tile waits for a global load of its learning rates.
+    // Learning rates are loaded four tiles ahead into four register slots (2
+    // values per lane per tile); the loop is unrolled by four so every slot
+    // keeps a fixed register and is read only when its tile is issued.
     const float* eta = p.eta.p + b * p.eta.sb + h * p.eta.sh;
     auto load_eta = [&](int j, float& e0, float& e1) {
       const int t = j * TT + lane;
@@ -189,7 +190,9 @@ __global__ void __launch_bounds__(kThreads, 1) la_tc_kernel(const __grid_constan
     load_eta(1, r1a, r1b);
     load_eta(2, r2a, r2b);
     load_eta(3, r3a, r3b);
-    for (int j = 0; j < ntiles; ++j) {
+    int j = 0;
+    auto issue = [&](float& ea, float& eb) -> bool {
+      if (j >= ntiles) return false;
       const int s = j % kStages;
       if (lane == 0 && j + kL2Ahead < ntiles)
         for (int x = 0; x < 2; ++x) {
@@ -198,12 +201,10 @@ __global__ void __launch_bounds__(kThreads, 1) la_tc_kernel(const __grid_constan
           tma_prefetch_l2_4d(&p.tv, 64 * x, (j + kL2Ahead) * TT, h, b);
         }
       if (j >= kStages && !mbar_wait(&sm.stage_free[s], ((j / kStages) - 1) & 1, p.status))
-        return;
+        return false;
       const int t0 = j * TT;
-      sm.eta[s][lane] = r0a;
-      sm.eta[s][lane + 32] = r0b;
-      r0a = r1a, r0b = r1b, r1a = r2a, r1b = r2b, r2a = r3a, r2b = r3b;
-      load_eta(j + 4, r3a, r3b);
+      sm.eta[s][lane] = ea;
+      sm.eta[s][lane + 32] = eb;
       __syncwarp();
       if (lane == 0) {
         mbar_arrive_expect_tx(&sm.full[s], 3 * kTileBytes);
@@ -213,6 +214,11 @@ __global__ void __launch_bounds__(kThreads, 1) la_tc_kernel(const __grid_constan
           tma_load_4d(sm.v[s] + x * 8192, &p.tv, &sm.full[s], 64 * x, t0, h, b);
         }
       }
+      load_eta(j + 4, ea, eb);
+      ++j;
+      return true;
+    };
+    while (issue(r0a, r0b) && issue(r1a, r1b) && issue(r2a, r2b) && issue(r3a, r3b)) {
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer

@@ -3,21 +3,22 @@
 //
 // Per (batch, head) z the fast weights W1, W3 [dh][dk] and W2 [dv][dh] live
 // in fp32 master copies in scratch memory, with bf16 operand copies refreshed
-// after every update (W1 and W3 rows interleaved in blocks of 128 into W13 so
-// one 256-column tile holds matching h1/h3 columns). One chunk step, all heads
-// at once (causal order: apply with the weights before the chunk, then
-// update):
-//   L1  Gz = -eta (V W2)                     [b x dh] fp32
-//       Aq = silu(Q W1^T) * (Q W3^T)         [b x dh] bf16          (causal)
-//   L2  from H = K [W1;W3]^T:  Ak' = eta silu(H1) H3, dH3 = Gz silu(H1),
-//       dH1 = Gz H3 silu'(H1)                [b x dh] bf16
-//       Y  = Aq W2^T -> layer output         [b x dv]               (causal)
-//   L3  G1 = dH1^T K, G3 = dH3^T K           [dh x dk] fp32 (split-K, atomics)
+// after every update (W1 and W3 rows interleaved in blocks of 64 into W13 so
+// that 128 consecutive W13 rows give matching h1/h3 columns). One chunk step,
+// all heads at once (causal order: apply with the weights before the chunk,
+// then update):
+//   L1  Aq = silu(Q W1^T) * (Q W3^T)         [b x dh] bf16          (causal)
+//       per 128 tokens x 64 hidden units, one accumulator tile holds
+//       H1 | H3 = K [W1;W3]^T and U = V W2 for those units; with Gz = -eta U:
+//       Ak' = eta silu(H1) H3, dH3 = Gz silu(H1), dH1 = Gz H3 silu'(H1)
+//                                            [b x dh] bf16 (Gz never leaves TMEM)
+//   L2  Y  = Aq W2^T -> layer output         [b x dv]               (causal)
+//       G1 = dH1^T K, G3 = dH3^T K           [dh x dk] fp32 (split-K, TMA add)
 //       G2 = -V^T Ak'                        [dv x dh]
-//   L4  Muon: G <- NS5(G) (split-bf16 tensor-core MMAs, fp32 accumulation)
-//   L5  W <- W - G; each row rescaled to its initial L2 norm; bf16 copies.
-// Non-causal (update, then apply): L1 without Aq, L2 without Y, L3, L4, L5,
-// then Aq and Y with the updated weights.
+//   L3  Muon: G <- NS5(G) (split-bf16 tensor-core MMAs, fp32 accumulation)
+//   L4  W <- W - G; each row rescaled to its initial L2 norm; bf16 copies.
+// Non-causal (update, then apply): L1 without Aq, L2 without Y, L3, L4, then
+// Aq and Y with the updated weights.
 // Precision: GD uses bf16 operands with fp32 accumulation; Muon uses
 // split-bf16 operands (x = hi + lo, products hi*hi + lo*hi + hi*lo) because
 // the unit-step Muon scan amplifies per-chunk rounding across chunks.
@@ -107,7 +108,8 @@ __global__ void __launch_bounds__(256) lact_rows_kernel(RowArgs a) {
   } else {
     hi = a.w13_hi;
     lo = a.w13_lo;
-    orow = (int64_t)z * 2 * a.dh + (r / (BN / 2)) * BN + (m == 1 ? BN / 2 : 0) + (r % (BN / 2));
+    orow = (int64_t)z * 2 * a.dh + (r / gemm::kHid) * 2 * gemm::kHid + (m == 1 ? gemm::kHid : 0) +
+           (r % gemm::kHid);
   }
   for (int i = 0; i < per; ++i) {
     const int c = lane + 32 * i;
@@ -120,14 +122,21 @@ __global__ void __launch_bounds__(256) lact_rows_kernel(RowArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// Newton-Schulz (Muon) on the tensor cores in split-bf16 precision: one CTA
-// per gradient matrix.
+// Newton-Schulz (Muon) on the tensor cores in split-bf16 precision: a cluster
+// of kNsCluster CTAs per gradient matrix, each owning one slab of the long
+// side. Gram partials meet in L2-resident scratch between cluster barriers;
+// every CTA then forms the (small) polynomial itself and updates its slab.
 // ---------------------------------------------------------------------------
+
+constexpr int kNsCluster = 4;
 
 struct NsArgs {
   float* G[3];   // in/out, [Z][rows][cols] row-major
   int rows[3], cols[3];
-  float* scratch;  // per (z, m): gram [s*s], poly [s*s], xn [rows*cols]
+  // per (z, m), s = min(rows, cols), L = max(rows, cols) / kNsCluster:
+  // Gram partials [2][kNsCluster][s*s], then per CTA gram [s*s], poly [s*s],
+  // xn [L*s], then kNsCluster partial squared norms
+  float* scratch;
   int64_t scratch_stride;
   float a, b, c, eps;
   int steps;
@@ -136,7 +145,8 @@ struct NsArgs {
 constexpr int kNsThreads = 1024;
 
 // C[M x N] = alpha * op(A) op(B) + beta * Cin, all row-major fp32 in global
-// memory (L2-resident scratch); op(A) is A or A^T (tA), same for B. Computed
+// memory (L2-resident scratch; row strides lda, ldb, ldc and ldcin); op(A) is
+// A or A^T (tA), same for B. Computed
 // by the whole CTA (32 warps) on the tensor cores with m16n8k16 MMAs in
 // split-bf16 precision: each fp32 operand x is held as hi = bf16(x) and
 // lo = bf16(x - hi), and the product accumulates hi*hi + lo*hi + hi*lo in fp32
@@ -166,7 +176,8 @@ __device__ __forceinline__ void ns_ldsm_x4_t(uint32_t (&r)[4], const void* p) {
 }
 
 __device__ void cta_gemm(float* C, const float* Cin, const float* A, const float* B, int M, int N,
-                         int K, bool tA, bool tB, int lda, int ldb, float alpha, float beta) {
+                         int K, bool tA, bool tB, int lda, int ldb, int ldc, int ldcin,
+                         float alpha, float beta) {
   __shared__ __align__(16) __nv_bfloat16 sa[2][kNsTM * kNsLdA];  // [hi|lo][m][k]
   __shared__ __align__(16) __nv_bfloat16 sb[2][kNsTK * kNsLdB];  // [hi|lo][k][n]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -234,54 +245,91 @@ __device__ void cta_gemm(float* C, const float* Cin, const float* A, const float
             const int i = i0 + 32 * wm + 16 * mt + g + 8 * (q >> 1);
             const int j = j0 + 16 * wn + 8 * nt + 2 * c4 + (q & 1);
             if (i < M && j < N) {
-              const float prev = (beta != 0.f) ? Cin[(int64_t)i * N + j] : 0.f;
-              C[(int64_t)i * N + j] = alpha * acc[mt][nt][q] + beta * prev;
+              const float prev = (beta != 0.f) ? Cin[(int64_t)i * ldcin + j] : 0.f;
+              C[(int64_t)i * ldc + j] = alpha * acc[mt][nt][q] + beta * prev;
             }
           }
       __syncthreads();
     }
 }
 
-__global__ void __launch_bounds__(kNsThreads) ns_kernel(NsArgs a) {
-  const int z = blockIdx.x / 3, m = blockIdx.x % 3;
+__device__ __forceinline__ void cluster_sync_all() {
+  __threadfence();
+  asm volatile(
+      "barrier.cluster.arrive.release.aligned;\n\t"
+      "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ float block_sum(float v) {
+  __shared__ float red[32];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float t = 0.f;
+  for (int i = 0; i < (int)(blockDim.x >> 5); ++i) t += red[i];
+  return t;
+}
+
+// X <- NS5(X / (||X||_F + eps)). Tall X (rows >= cols): X <- a X + X (b A + c A^2)
+// with A = X^T X; wide X: X <- a X + (b A + c A^2) X with A = X X^T. CTA c of
+// the cluster owns rows (tall) or columns (wide) [c L, c L + L) of X.
+__global__ void __cluster_dims__(kNsCluster, 1, 1) __launch_bounds__(kNsThreads)
+    ns_kernel(NsArgs a) {
+  const int mat = blockIdx.x / kNsCluster, c = blockIdx.x % kNsCluster;
+  const int z = mat / 3, m = mat % 3;
   const int R = a.rows[m], C = a.cols[m];
   float* X = a.G[m] + (int64_t)z * R * C;
-  const int s = min(R, C);
-  float* gram = a.scratch + (int64_t)blockIdx.x * a.scratch_stride;
+  const bool tall = R >= C;
+  const int s = tall ? C : R;
+  const int L = (tall ? R : C) / kNsCluster;
+  float* Xc = tall ? X + (int64_t)c * L * C : X + (int64_t)c * L;  // row stride C
+  float* base = a.scratch + (int64_t)mat * a.scratch_stride;
+  float* parts = base;
+  float* gram = parts + 2 * kNsCluster * s * s + (int64_t)c * (2 * s * s + L * s);
   float* poly = gram + (int64_t)s * s;
   float* xn = poly + (int64_t)s * s;
-  __shared__ float red[32];
+  float* nrm = base + 2 * kNsCluster * s * s + (int64_t)kNsCluster * (2 * s * s + L * s);
+  const int sr = tall ? L : s, sc = tall ? s : L;  // slab rows x columns (row stride C)
+  const int tid = threadIdx.x;
+
   float ss = 0.f;
-  for (int64_t i = threadIdx.x; i < (int64_t)R * C; i += blockDim.x) ss += X[i] * X[i];
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    float t = red[threadIdx.x];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-    if (threadIdx.x == 0) red[0] = t;
+  for (int e = tid; e < sr * sc; e += kNsThreads) {
+    const float x = Xc[(int64_t)(e / sc) * C + e % sc];
+    ss += x * x;
   }
+  ss = block_sum(ss);
+  if (tid == 0) nrm[c] = ss;
+  cluster_sync_all();
+  float tot = 0.f;
+  for (int i = 0; i < kNsCluster; ++i) tot += __ldcg(nrm + i);  // other CTAs' writes: bypass L1
+  const float inv = 1.f / (sqrtf(tot) + a.eps);
+  for (int e = tid; e < sr * sc; e += kNsThreads) Xc[(int64_t)(e / sc) * C + e % sc] *= inv;
   __syncthreads();
-  const float inv = 1.f / (sqrtf(red[0]) + a.eps);
-  for (int64_t i = threadIdx.x; i < (int64_t)R * C; i += blockDim.x) X[i] *= inv;
-  __syncthreads();
-  const bool tall = R >= C;
   for (int it = 0; it < a.steps; ++it) {
-    // gram: tall -> X^T X (C x C); wide -> X X^T (R x R)
+    float* part = parts + ((int64_t)(it & 1) * kNsCluster + c) * s * s;
     if (tall)
-      cta_gemm(gram, nullptr, X, X, s, s, R, true, false, C, C, 1.f, 0.f);
+      cta_gemm(part, nullptr, Xc, Xc, s, s, L, true, false, C, C, s, s, 1.f, 0.f);
     else
-      cta_gemm(gram, nullptr, X, X, s, s, C, false, true, C, C, 1.f, 0.f);
-    // poly = c * gram @ gram + b * gram
-    cta_gemm(poly, gram, gram, gram, s, s, s, false, false, s, s, a.c, a.b);
-    // xn = X poly (tall) or poly X (wide); X = a X + xn
+      cta_gemm(part, nullptr, Xc, Xc, s, s, L, false, true, C, C, s, s, 1.f, 0.f);
+    cluster_sync_all();
+    const float* pb = parts + (int64_t)(it & 1) * kNsCluster * s * s;
+    for (int e = tid; e < s * s; e += kNsThreads) {
+      float g = 0.f;
+      for (int i = 0; i < kNsCluster; ++i) g += __ldcg(pb + (int64_t)i * s * s + e);
+      gram[e] = g;
+    }
+    __syncthreads();
+    // poly = c gram^2 + b gram
+    cta_gemm(poly, gram, gram, gram, s, s, s, false, false, s, s, s, s, a.c, a.b);
+    // xn = slab poly (tall) or poly slab (wide), plus a * slab
     if (tall)
-      cta_gemm(xn, X, X, poly, R, C, C, false, false, C, C, 1.f, a.a);
+      cta_gemm(xn, Xc, Xc, poly, L, s, s, false, false, C, s, s, C, 1.f, a.a);
     else
-      cta_gemm(xn, X, poly, X, R, C, R, false, false, R, C, 1.f, a.a);
-    for (int64_t i = threadIdx.x; i < (int64_t)R * C; i += blockDim.x) X[i] = xn[i];
+      cta_gemm(xn, Xc, poly, Xc, s, L, s, false, false, s, C, L, C, 1.f, a.a);
+    for (int e = tid; e < sr * sc; e += kNsThreads)
+      Xc[(int64_t)(e / sc) * C + e % sc] = xn[e];
     __syncthreads();
   }
 }
@@ -321,31 +369,20 @@ bool map_buf(CUtensorMap* m, const void* base, int Z, int rows, int rows_alloc, 
                    CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-// Output maps for the TMA-store epilogue: boxes of {16 columns, 32 rows}.
-bool out_map_buf(CUtensorMap* m, const void* base, bool bf16, int Z, int rows, int cols) {
-  const uint64_t es = bf16 ? 2 : 4;
+// fp32 gradient [Z][rows][cols] as a TMA add-reduction target: box of
+// {32 columns, 32 rows} (128-byte rows) with the 128-byte swizzle of the
+// epilogue's staging buffers.
+bool grad_map(CUtensorMap* m, const float* base, int Z, int rows, int cols) {
   uint64_t dims[4] = {(uint64_t)cols, (uint64_t)rows, (uint64_t)Z, 1};
-  uint64_t strides[3] = {(uint64_t)cols * es, (uint64_t)cols * es * rows,
-                         (uint64_t)cols * es * rows * Z};
-  uint32_t box[4] = {16, 32, 1, 1};
-  return make_tmap(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4,
-                   base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
-}
-bool out_map_tokens(CUtensorMap* m, const TokViewMut& v, const LactArgs& a, int d) {
-  TokViewMut x = v;
-  const uint64_t es = a.dtype == TTT_BF16 ? 2 : 4;
-  if (a.B == 1) x.sb = (int64_t)a.H * a.T * d;
-  if (a.H == 1) x.sh = (int64_t)a.T * d;
-  if (a.T == 1) x.st = d;
-  uint64_t dims[4] = {(uint64_t)d, (uint64_t)a.T, (uint64_t)a.H, (uint64_t)a.B};
-  uint64_t strides[3] = {(uint64_t)x.st * es, (uint64_t)x.sh * es, (uint64_t)x.sb * es};
-  uint32_t box[4] = {16, 32, 1, 1};
-  return make_tmap(m, es == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
-                   4, x.p, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+  uint64_t strides[3] = {(uint64_t)cols * 4, (uint64_t)cols * 4 * rows,
+                         (uint64_t)cols * 4 * rows * Z};
+  uint32_t box[4] = {32, 32, 1, 1};
+  return make_tmap(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, dims, strides, box,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 struct Scratch {
-  float *Wm[3], *rho[3], *G[3], *gz, *ns;
+  float *Wm[3], *rho[3], *G[3], *ns;
   __nv_bfloat16 *w13[2], *w2[2];          // hi, lo
   __nv_bfloat16 *aq[2], *ak[2], *dh1[2], *dh3[2];
   int64_t ns_stride;
@@ -356,7 +393,7 @@ void fill_problem_tiles(Params& P) {
   for (int i = 0; i < P.nprob; ++i) {
     Problem& p = P.p[i];
     p.mtiles = (p.M + gemm::BM - 1) / gemm::BM;
-    p.ntiles = (p.N + BN - 1) / BN;
+    p.ntiles = (p.N + p.tn - 1) / p.tn;
     p.tile_begin = t;
     t += p.nz * p.ksplit * p.mtiles * p.ntiles;
   }
@@ -476,9 +513,9 @@ Sizes lact_sizes(const LactArgs& a) {
   z.nrows[0] = z.nrows[1] = dh;
   z.nrows[2] = dv;
   const int s_max = dk < dh ? dk : dh;
-  z.ns_stride = 2 * (int64_t)s_max * s_max + (int64_t)dh * dk;
+  z.ns_stride = 2 * kNsCluster * (int64_t)s_max * s_max +
+                kNsCluster * 2 * (int64_t)s_max * s_max + (int64_t)dh * dk + 64;
   for (int m = 0; m < 3; ++m) z.f32n += (size_t)z.Z * (2 * z.nW[m] + z.nrows[m]);
-  z.f32n += (size_t)z.Z * z.chunk * dh;                  // gz
   if (z.split) z.f32n += (size_t)z.Z * 3 * z.ns_stride;  // Newton-Schulz scratch
   z.bfn = (size_t)z.Z * (2 * dh * dk + dv * dh) * (z.split ? 2 : 1);
   z.bfn += (size_t)z.Z * z.chunk * dh * 4 * (z.split ? 2 : 1);
@@ -527,8 +564,6 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
       sc.rho[m] = f;
       f += Z * nrows[m];
     }
-    sc.gz = f;
-    f += (size_t)Z * chunk * dh;
     sc.ns = split ? f : nullptr;
     if (split) f += (size_t)Z * 3 * ns_stride;
     uintptr_t up = (reinterpret_cast<uintptr_t>(f) + 255) & ~uintptr_t(255);
@@ -611,9 +646,10 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
   for (int s0 = 0; s0 < a.T && result == TTT_OK; s0 += chunk) {
     const int bc = (a.T - s0) < chunk ? (a.T - s0) : chunk;
     // shared operands for this chunk
-    Operand W13, W2mn, W2k, Qk, Kk, Vk, Kmn, Vmn, AQk, DH1mn, DH3mn, AKmn;
+    Operand W13, W13h, W2mn, W2k, Qk, Kk, Vk, Kmn, Vmn, AQk, DH1mn, DH3mn, AKmn;
     bool ok = true;
     ok &= buf_op(W13, sc.w13, Z, 2 * dh, 2 * dh, dk, 0, BN, split);
+    ok &= buf_op(W13h, sc.w13, Z, 2 * dh, 2 * dh, dk, 0, 2 * gemm::kHid, split);
     ok &= buf_op(W2mn, sc.w2, Z, dv, dv, dh, 1, 64, split);
     ok &= buf_op(W2k, sc.w2, Z, dv, dv, dh, 0, BN, split);
     ok &= tok_kmajor(Qk, a.q, a, dk, s0, gemm::BM);
@@ -630,109 +666,79 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
       break;
     }
     bool okm = true;  // output maps built
-    auto add_apply = [&](Params& P, int stage) {
-      // stage 0: Aq from Q; stage 1: Y from Aq
+    auto new_problem = [&](Params& P) -> Problem& {
       Problem& p = P.p[P.nprob++];
       memset(&p, 0, sizeof(p));
       p.nz = Z;
       p.ksplit = 1;
-      if (stage == 0) {
-        p.a = Qk;
-        p.b = W13;
-        p.M = bc;
-        p.N = 2 * dh;
-        p.K = dk;
-        segs(p, nsegW, reinterpret_cast<const int(*)[2]>(segW));
-        p.epi = gemm::EPI_AQ;
-        p.e = epi_base(a, s0, bc);
-        p.e.nsplit = split ? 2 : 1;
-        p.e.ozdiv = Z;
-        okm &= out_map_buf(&p.e.omap[0], sc.aq[0], true, Z, chunk, dh);
-        if (split) okm &= out_map_buf(&p.e.omap[3], sc.aq[1], true, Z, chunk, dh);
-      } else {
-        p.a = AQk;
-        p.b = W2k;
-        p.M = bc;
-        p.N = dv;
-        p.K = dh;
-        if (split)
-          segs(p, 3, kSegBoth);
-        else
-          segs(p, 1, kSegExact);
-        p.epi = gemm::EPI_Y;
-        p.e = epi_base(a, s0, bc);
-        p.e.ozdiv = a.H;
-        p.e.orow0 = s0;
-        okm &= out_map_tokens(&p.e.omap[0], a.out, a, dv);
-      }
+      p.tn = BN;
+      return p;
     };
-
-    // L1: Gz (+ Aq when causal)
-    {
-      Params P;
-      memset(&P, 0, sizeof(P));
-      P.status = a.status;
-      Problem& p = P.p[P.nprob++];
-      p.a = Vk;
-      p.b = W2mn;
-      p.M = bc;
-      p.N = dh;
-      p.K = dv;
-      p.nz = Z;
-      p.ksplit = 1;
-      segs(p, nsegW, reinterpret_cast<const int(*)[2]>(segW));
-      p.epi = gemm::EPI_GZ;
-      p.e = epi_base(a, s0, bc);
-      p.e.gz = sc.gz;
-      p.e.gz_rows = chunk;
-      p.e.gz_cols = dh;
-      if (a.causal) add_apply(P, 0);
-      if (!okm) result = TTT_ERR_CUDA;
-      check(launch_gemm(P, s));
-    }
-    // L2: key forward + backprop epilogue (+ Y when causal)
-    {
-      Params P;
-      memset(&P, 0, sizeof(P));
-      P.status = a.status;
-      Problem& p = P.p[P.nprob++];
-      p.a = Kk;
+    auto add_aq = [&](Params& P) {  // Aq = silu(Q W1^T) * (Q W3^T)
+      Problem& p = new_problem(P);
+      p.a = Qk;
       p.b = W13;
       p.M = bc;
       p.N = 2 * dh;
       p.K = dk;
-      p.nz = Z;
-      p.ksplit = 1;
       segs(p, nsegW, reinterpret_cast<const int(*)[2]>(segW));
-      p.epi = gemm::EPI_HK;
+      p.epi = gemm::EPI_AQ;
       p.e = epi_base(a, s0, bc);
-      p.e.gz = sc.gz;
-      p.e.gz_rows = chunk;
-      p.e.gz_cols = dh;
       p.e.nsplit = split ? 2 : 1;
-      p.e.ozdiv = Z;
-      for (int x = 0; x < (split ? 2 : 1); ++x) {
-        okm &= out_map_buf(&p.e.omap[3 * x + 0], sc.ak[x], true, Z, chunk, dh);
-        okm &= out_map_buf(&p.e.omap[3 * x + 1], sc.dh1[x], true, Z, chunk, dh);
-        okm &= out_map_buf(&p.e.omap[3 * x + 2], sc.dh3[x], true, Z, chunk, dh);
+      p.e.optr[0] = sc.aq[0];
+      p.e.optr[3] = sc.aq[1];
+      p.e.orows = chunk;
+      p.e.ocols = dh;
+    };
+    auto add_y = [&](Params& P) {  // Y = Aq W2^T -> output tokens
+      Problem& p = new_problem(P);
+      p.a = AQk;
+      p.b = W2k;
+      p.M = bc;
+      p.N = dv;
+      p.K = dh;
+      if (split)
+        segs(p, 3, kSegBoth);
+      else
+        segs(p, 1, kSegExact);
+      p.epi = gemm::EPI_Y;
+      p.e = epi_base(a, s0, bc);
+      p.e.orow0 = s0;
+    };
+    auto add_key = [&](Params& P) {  // [H1 | H3 | V W2] tiles -> Ak', dH1, dH3
+      Problem& p = new_problem(P);
+      p.a = Kk;
+      p.b = W13h;
+      p.a2 = Vk;
+      p.b2 = W2mn;
+      p.M = bc;
+      p.N = 2 * dh;
+      p.K = dk;  // = dv
+      p.tn = 2 * gemm::kHid;
+      segs(p, nsegW, reinterpret_cast<const int(*)[2]>(segW));
+      p.nseg2 = nsegW;
+      for (int i = 0; i < nsegW; ++i) {
+        p.seg2_a[i] = segW[2 * i];
+        p.seg2_b[i] = segW[2 * i + 1];
       }
-      if (a.causal) add_apply(P, 1);
-      if (!okm) result = TTT_ERR_CUDA;
-      check(launch_gemm(P, s));
-    }
-    // L3: weight gradients (token reductions, split-K with atomics)
-    {
-      Params P;
-      memset(&P, 0, sizeof(P));
-      P.status = a.status;
+      p.epi = gemm::EPI_HKG;
+      p.e = epi_base(a, s0, bc);
+      p.e.nsplit = split ? 2 : 1;
+      for (int x = 0; x < (split ? 2 : 1); ++x) {
+        p.e.optr[3 * x + 0] = sc.ak[x];
+        p.e.optr[3 * x + 1] = sc.dh1[x];
+        p.e.optr[3 * x + 2] = sc.dh3[x];
+      }
+      p.e.orows = chunk;
+      p.e.ocols = dh;
+    };
+    auto add_grads = [&](Params& P) {  // weight gradients (token reductions, split-K)
       const int kblocks = (bc + gemm::BK - 1) / gemm::BK;
       const int tiles = Z * (2 * ((dh + gemm::BM - 1) / gemm::BM) * ((dk + BN - 1) / BN) +
                              ((dv + gemm::BM - 1) / gemm::BM) * ((dh + BN - 1) / BN));
       const int ks = pick_ksplit(kblocks, tiles);
       for (int g = 0; g < 3; ++g) {
-        Problem& p = P.p[P.nprob++];
-        memset(&p, 0, sizeof(p));
-        p.nz = Z;
+        Problem& p = new_problem(P);
         p.ksplit = ks;
         p.K = bc;
         p.epi = gemm::EPI_GRAD;
@@ -747,7 +753,7 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
             segs(p, 1, kSegExact);
           p.e = epi_base(a, s0, dh);
           p.e.ozdiv = Z;
-          okm &= out_map_buf(&p.e.omap[0], g == 0 ? sc.G[0] : sc.G[1], false, Z, dh, dk);
+          okm &= grad_map(&p.e.gmap, g == 0 ? sc.G[0] : sc.G[1], Z, dh, dk);
         } else {
           p.a = Vmn;
           p.b = AKmn;
@@ -760,15 +766,35 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
           p.e = epi_base(a, s0, dv);
           p.e.ozdiv = Z;
           p.e.scale = -1.f;
-          okm &= out_map_buf(&p.e.omap[0], sc.G[2], false, Z, dv, dh);
+          okm &= grad_map(&p.e.gmap, sc.G[2], Z, dv, dh);
         }
       }
+    };
+    auto run = [&](Params& P) {
       if (!okm) result = TTT_ERR_CUDA;
       check(launch_gemm(P, s));
+    };
+    // L1: Aq (causal) and the fused key-side tiles
+    {
+      Params P;
+      memset(&P, 0, sizeof(P));
+      P.status = a.status;
+      if (a.causal) add_aq(P);
+      add_key(P);
+      run(P);
     }
-    // L4 / L5: Muon orthogonalisation, update and row renormalisation
+    // L2: Y (causal) and the weight gradients
+    {
+      Params P;
+      memset(&P, 0, sizeof(P));
+      P.status = a.status;
+      if (a.causal) add_y(P);
+      add_grads(P);
+      run(P);
+    }
+    // L3 / L4: Muon orthogonalisation, update and row renormalisation
     if (split) {
-      ns_kernel<<<Z * 3, kNsThreads, 0, s>>>(na);
+      ns_kernel<<<Z * 3 * kNsCluster, kNsThreads, 0, s>>>(na);
       check(cudaGetLastError());
     }
     lact_rows_kernel<<<row_blocks, 256, 0, s>>>(ra);
@@ -777,13 +803,13 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
       Params P;
       memset(&P, 0, sizeof(P));
       P.status = a.status;
-      add_apply(P, 0);
-      check(launch_gemm(P, s));
+      add_aq(P);
+      run(P);
       Params P2;
       memset(&P2, 0, sizeof(P2));
       P2.status = a.status;
-      add_apply(P2, 1);
-      check(launch_gemm(P2, s));
+      add_y(P2);
+      run(P2);
     }
   }
 

@@ -101,7 +101,7 @@ __device__ __forceinline__ void next_block(const Params& p, int s, int& nb, bool
   }
 }
 
-template <int D>
+template <int D, int LOSS>
 __global__ void __launch_bounds__((D / 16 + 1) * 32, 1)
 ttt_linear_bf16_kernel(const __grid_constant__ Params p) {
   constexpr int NW = D / 16;   // consumer warps
@@ -129,45 +129,50 @@ ttt_linear_bf16_kernel(const __grid_constant__ Params p) {
       prefetch_tmap(&p.tk);
       prefetch_tmap(&p.tv);
     }
-    // The next 4 blocks' starts and learning rates stay in flight in
-    // registers (lane l < 16 holds eta of the block's token l), so no block
-    // waits for a global load of its learning rates.
+    // Learning rates are loaded four blocks ahead into a ring of four register
+    // slots (lane l < 16 holds eta of the block's token l). The loop is
+    // unrolled by four so every slot keeps a fixed register: a slot is only
+    // read when its block is issued, four iterations after its load.
     const float* eta = p.eta.p + b * p.eta.sb + h * p.eta.sh;
-    int sr[4], nr[4];
-    float er[4];
     int s_next = 0;  // start of the next block to enter the ring
-    auto fill = [&](int k) {
+    auto fill = [&](int& sr, int& nr, float& er) {
       int nb = 0;
       bool ce;
       if (s_next < p.T) next_block(p, s_next, nb, ce);
-      sr[k] = s_next;
-      nr[k] = nb;
-      er[k] = (lane < nb) ? eta[(int64_t)(s_next + lane) * p.eta.st] : 0.f;
+      sr = s_next;
+      nr = nb;
+      er = (lane < nb) ? eta[(int64_t)(s_next + lane) * p.eta.st] : 0.f;
       s_next += nb;
     };
-#pragma unroll
-    for (int k = 0; k < 4; ++k) fill(k);
+    int sr0, sr1, sr2, sr3, nr0, nr1, nr2, nr3;
+    float er0, er1, er2, er3;
+    fill(sr0, nr0, er0);
+    fill(sr1, nr1, er1);
+    fill(sr2, nr2, er2);
+    fill(sr3, nr3, er3);
     int it = 0;
-    while (nr[0] > 0) {
-      const int s = sr[0];
-      const float e = er[0];
+    // issue one block from a slot, then refill the slot four blocks ahead
+    auto issue = [&](int& sr, int& nr, float& er) -> bool {
+      if (nr == 0) return false;
       const int st = it % kStages;
-      if (it >= kStages && !mbar_wait(&sm.empty[st], ((it / kStages) - 1) & 1, p.status)) return;
-      if (lane < kTB) sm.eta[st][lane] = e;
-      // rotate the ring and request the block after the last one in it
-#pragma unroll
-      for (int k = 0; k < 3; ++k) sr[k] = sr[k + 1], nr[k] = nr[k + 1], er[k] = er[k + 1];
-      fill(3);
+      if (it >= kStages && !mbar_wait(&sm.empty[st], ((it / kStages) - 1) & 1, p.status))
+        return false;
+      if (lane < kTB) sm.eta[st][lane] = er;
       __syncwarp();
       if (lane == 0) {
         mbar_arrive_expect_tx(&sm.full[st], 3 * Smem<D>::kTile);
         for (int x = 0; x < D / 64; ++x) {
-          tma_load_4d(sm.q[st] + x * 2048, &p.tq, &sm.full[st], x * 64, s, h, b);
-          tma_load_4d(sm.k[st] + x * 2048, &p.tk, &sm.full[st], x * 64, s, h, b);
-          tma_load_4d(sm.v[st] + x * 2048, &p.tv, &sm.full[st], x * 64, s, h, b);
+          tma_load_4d(sm.q[st] + x * 2048, &p.tq, &sm.full[st], x * 64, sr, h, b);
+          tma_load_4d(sm.k[st] + x * 2048, &p.tk, &sm.full[st], x * 64, sr, h, b);
+          tma_load_4d(sm.v[st] + x * 2048, &p.tv, &sm.full[st], x * 64, sr, h, b);
         }
       }
       ++it;
+      fill(sr, nr, er);
+      return true;
+    };
+    while (issue(sr0, nr0, er0) && issue(sr1, nr1, er1) && issue(sr2, nr2, er2) &&
+           issue(sr3, nr3, er3)) {
     }
     return;
   }
@@ -187,18 +192,26 @@ ttt_linear_bf16_kernel(const __grid_constant__ Params p) {
     Wc[j][2] = W0[(int64_t)c * D + r0 + g + 8];
     Wc[j][3] = W0[(int64_t)(c + 1) * D + r0 + g + 8];
   }
-  // W_{t'}^T as bf16 A fragments per k-block.
-  uint32_t Ws[KB][4];
-  auto refresh_start = [&]() {
+  // Wy: W_cur^T as bf16 A fragments per k-block (operand of W_cur^T Q^T),
+  // packed once after every block. Ws: the chunk-start copy W_{t'}^T (MSE).
+  uint32_t Wy[KB][4], Ws[KB][4];
+  auto pack_cur = [&]() {
 #pragma unroll
     for (int kb = 0; kb < KB; ++kb) {
-      Ws[kb][0] = pack_bf16(Wc[2 * kb][0], Wc[2 * kb][1]);
-      Ws[kb][1] = pack_bf16(Wc[2 * kb][2], Wc[2 * kb][3]);
-      Ws[kb][2] = pack_bf16(Wc[2 * kb + 1][0], Wc[2 * kb + 1][1]);
-      Ws[kb][3] = pack_bf16(Wc[2 * kb + 1][2], Wc[2 * kb + 1][3]);
+      Wy[kb][0] = pack_bf16(Wc[2 * kb][0], Wc[2 * kb][1]);
+      Wy[kb][1] = pack_bf16(Wc[2 * kb][2], Wc[2 * kb][3]);
+      Wy[kb][2] = pack_bf16(Wc[2 * kb + 1][0], Wc[2 * kb + 1][1]);
+      Wy[kb][3] = pack_bf16(Wc[2 * kb + 1][2], Wc[2 * kb + 1][3]);
     }
   };
-  if (p.loss == TTT_LOSS_MSE) refresh_start();
+  auto start_chunk = [&]() {
+#pragma unroll
+    for (int kb = 0; kb < KB; ++kb)
+#pragma unroll
+      for (int u = 0; u < 4; ++u) Ws[kb][u] = Wy[kb][u];
+  };
+  pack_cur();
+  if constexpr (LOSS == TTT_LOSS_MSE) start_chunk();
 
   const int mi = lane >> 3, rr = lane & 7;
   int it = 0;
@@ -212,19 +225,6 @@ ttt_linear_bf16_kernel(const __grid_constant__ Params p) {
     const uint8_t* vb = sm.v[st];
     const float* et = sm.eta[st];
 
-    // K as B operand (k = dk, n = token): Bk[kb][nt][2]
-    uint32_t Bk[KB][2][2];
-#pragma unroll
-    for (int kb = 0; kb < KB; ++kb) {
-      uint32_t r[4];
-      ldsm_x4(r, ka + sw_off(8 * (mi >> 1) + rr, 16 * kb + 8 * (mi & 1)));
-      Bk[kb][0][0] = r[0];
-      Bk[kb][0][1] = r[1];
-      Bk[kb][1][0] = r[2];
-      Bk[kb][1][1] = r[3];
-    }
-
-    // E^T = W_{t'}^T K^T - V^T  (rows dv r0+{g,g+8}, cols token 8nt+2c4+{0,1})
     float E[2][4];
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
@@ -237,71 +237,75 @@ ttt_linear_bf16_kernel(const __grid_constant__ Params p) {
       E[nt][2] = -vv(t, r0 + g + 8);
       E[nt][3] = -vv(t + 1, r0 + g + 8);
     }
-    if (p.loss == TTT_LOSS_MSE) {
+    const int i0 = 2 * c4;
+    const float n0 = -et[i0], n1 = -et[i0 + 1], n8 = -et[i0 + 8], n9 = -et[i0 + 9];
+
+    // Three independent products, each split over even / odd k-blocks so that
+    // no accumulator chain is longer than KB / 2:
+    //   E^T = W_{t'}^T K^T - V^T,  S = Q K^T,  Y^T = W_cur^T Q^T.
+    // K and Q enter as B operands (k = dk, n = token), Q also as A (rows token).
+    float E2[2][4] = {}, S[2][4] = {}, S2[2][4] = {}, Y[2][4] = {}, Y2[2][4] = {};
 #pragma unroll
-      for (int kb = 0; kb < KB; ++kb) {
-        mma16816(E[0], Ws[kb], Bk[kb][0][0], Bk[kb][0][1]);
-        mma16816(E[1], Ws[kb], Bk[kb][1][0], Bk[kb][1][1]);
+    for (int kb = 0; kb < KB; kb += 2) {
+      uint32_t Bk[2][4], Bq[2][4], Aq[2][4];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        ldsm_x4(Bk[u], ka + sw_off(8 * (mi >> 1) + rr, 16 * (kb + u) + 8 * (mi & 1)));
+        ldsm_x4(Aq[u], qa + sw_off(rr + 8 * (mi & 1), 16 * (kb + u) + 8 * (mi >> 1)));
+        ldsm_x4(Bq[u], qa + sw_off(8 * (mi >> 1) + rr, 16 * (kb + u) + 8 * (mi & 1)));
+      }
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        if constexpr (LOSS == TTT_LOSS_MSE) {
+          mma16816(E[nt], Ws[kb], Bk[0][2 * nt], Bk[0][2 * nt + 1]);
+          mma16816(E2[nt], Ws[kb + 1], Bk[1][2 * nt], Bk[1][2 * nt + 1]);
+        }
+        mma16816(S[nt], Aq[0], Bk[0][2 * nt], Bk[0][2 * nt + 1]);
+        mma16816(S2[nt], Aq[1], Bk[1][2 * nt], Bk[1][2 * nt + 1]);
+        mma16816(Y[nt], Wy[kb], Bq[0][2 * nt], Bq[0][2 * nt + 1]);
+        mma16816(Y2[nt], Wy[kb + 1], Bq[1][2 * nt], Bq[1][2 * nt + 1]);
       }
     }
-
-    // Scores S = Q K^T (rows t, cols i), then P = -eta_i S for i <= t.
-    float S[2][4] = {};
+    // K^T fragments for the update (issued while the products run)
+    uint32_t Kt[NT / 2][4];
 #pragma unroll
-    for (int kb = 0; kb < KB; ++kb) {
-      uint32_t a[4];
-      ldsm_x4(a, qa + sw_off(rr + 8 * (mi & 1), 16 * kb + 8 * (mi >> 1)));
-      mma16816(S[0], a, Bk[kb][0][0], Bk[kb][0][1]);
-      mma16816(S[1], a, Bk[kb][1][0], Bk[kb][1][1]);
-    }
-    uint32_t Pb[2][2];  // B fragments of P^T for Y n-tile (t) 0 and 1
+    for (int j = 0; j < NT; j += 2) ldsm_x4_t(Kt[j / 2], ka + sw_off(rr + 8 * (mi & 1), 8 * (j + (mi >> 1))));
+
+    // P = -eta_i S[t][i] for i <= t, as B fragments of P^T (n-tile = t).
+    uint32_t Pb[2][2];
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
-      const int i0 = 8 * nt + 2 * c4;
-      const float e0 = -et[i0], e1 = -et[i0 + 1];
+      const int ii = 8 * nt + 2 * c4;
+      const float e0 = nt ? n8 : n0, e1 = nt ? n9 : n1;
       const int t0 = g, t1 = g + 8;
-      float p00 = (i0 <= t0) ? e0 * S[nt][0] : 0.f;
-      float p01 = (i0 + 1 <= t0) ? e1 * S[nt][1] : 0.f;
-      float p10 = (i0 <= t1) ? e0 * S[nt][2] : 0.f;
-      float p11 = (i0 + 1 <= t1) ? e1 * S[nt][3] : 0.f;
-      Pb[0][nt] = pack_bf16(p00, p01);
-      Pb[1][nt] = pack_bf16(p10, p11);
+      const float s0 = S[nt][0] + S2[nt][0], s1 = S[nt][1] + S2[nt][1];
+      const float s2 = S[nt][2] + S2[nt][2], s3 = S[nt][3] + S2[nt][3];
+      Pb[0][nt] = pack_bf16((ii <= t0) ? e0 * s0 : 0.f, (ii + 1 <= t0) ? e1 * s1 : 0.f);
+      Pb[1][nt] = pack_bf16((ii <= t1) ? e0 * s2 : 0.f, (ii + 1 <= t1) ? e1 * s3 : 0.f);
     }
-
-    // Y^T = W_cur^T Q^T + E^T P^T
-    float Y[2][4] = {};
 #pragma unroll
-    for (int kb = 0; kb < KB; ++kb) {
-      uint32_t a[4] = {pack_bf16(Wc[2 * kb][0], Wc[2 * kb][1]),
-                       pack_bf16(Wc[2 * kb][2], Wc[2 * kb][3]),
-                       pack_bf16(Wc[2 * kb + 1][0], Wc[2 * kb + 1][1]),
-                       pack_bf16(Wc[2 * kb + 1][2], Wc[2 * kb + 1][3])};
-      uint32_t r[4];
-      ldsm_x4(r, qa + sw_off(8 * (mi >> 1) + rr, 16 * kb + 8 * (mi & 1)));
-      mma16816(Y[0], a, r[0], r[1]);
-      mma16816(Y[1], a, r[2], r[3]);
-    }
-    {
-      uint32_t ea[4] = {pack_bf16(E[0][0], E[0][1]), pack_bf16(E[0][2], E[0][3]),
-                        pack_bf16(E[1][0], E[1][1]), pack_bf16(E[1][2], E[1][3])};
-      mma16816(Y[0], ea, Pb[0][0], Pb[0][1]);
-      mma16816(Y[1], ea, Pb[1][0], Pb[1][1]);
-    }
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int u = 0; u < 4; ++u) E[nt][u] += E2[nt][u];
 
-    // W_cur^T += (-E^T N) K
+    // W_cur^T += (-E^T N) K   (8 independent MMAs)
     {
-      const int i0 = 2 * c4;
-      uint32_t ea[4] = {pack_bf16(-et[i0] * E[0][0], -et[i0 + 1] * E[0][1]),
-                        pack_bf16(-et[i0] * E[0][2], -et[i0 + 1] * E[0][3]),
-                        pack_bf16(-et[i0 + 8] * E[1][0], -et[i0 + 9] * E[1][1]),
-                        pack_bf16(-et[i0 + 8] * E[1][2], -et[i0 + 9] * E[1][3])};
+      const uint32_t ea[4] = {pack_bf16(n0 * E[0][0], n1 * E[0][1]),
+                              pack_bf16(n0 * E[0][2], n1 * E[0][3]),
+                              pack_bf16(n8 * E[1][0], n9 * E[1][1]),
+                              pack_bf16(n8 * E[1][2], n9 * E[1][3])};
 #pragma unroll
       for (int j = 0; j < NT; j += 2) {
-        uint32_t r[4];
-        ldsm_x4_t(r, ka + sw_off(rr + 8 * (mi & 1), 8 * (j + (mi >> 1))));
-        mma16816(Wc[j], ea, r[0], r[1]);
-        mma16816(Wc[j + 1], ea, r[2], r[3]);
+        mma16816(Wc[j], ea, Kt[j / 2][0], Kt[j / 2][1]);
+        mma16816(Wc[j + 1], ea, Kt[j / 2][2], Kt[j / 2][3]);
       }
+    }
+    // Y^T += E^T P^T
+    {
+      const uint32_t ea[4] = {pack_bf16(E[0][0], E[0][1]), pack_bf16(E[0][2], E[0][3]),
+                              pack_bf16(E[1][0], E[1][1]), pack_bf16(E[1][2], E[1][3])};
+      mma16816(Y[0], ea, Pb[0][0], Pb[0][1]);
+      mma16816(Y[1], ea, Pb[1][0], Pb[1][1]);
     }
 
     // Output: stage Y^T -> [t][r] and store 16 rows x 32 bytes.
@@ -309,10 +313,10 @@ ttt_linear_bf16_kernel(const __grid_constant__ Params p) {
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
       const int t = 8 * nt + 2 * c4;
-      os[t][g] = __float2bfloat16_rn(Y[nt][0]);
-      os[t + 1][g] = __float2bfloat16_rn(Y[nt][1]);
-      os[t][g + 8] = __float2bfloat16_rn(Y[nt][2]);
-      os[t + 1][g + 8] = __float2bfloat16_rn(Y[nt][3]);
+      os[t][g] = __float2bfloat16_rn(Y[nt][0] + Y2[nt][0]);
+      os[t + 1][g] = __float2bfloat16_rn(Y[nt][1] + Y2[nt][1]);
+      os[t][g + 8] = __float2bfloat16_rn(Y[nt][2] + Y2[nt][2]);
+      os[t + 1][g + 8] = __float2bfloat16_rn(Y[nt][3] + Y2[nt][3]);
     }
     __syncwarp();
     {
@@ -325,7 +329,9 @@ ttt_linear_bf16_kernel(const __grid_constant__ Params p) {
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&sm.empty[st]);
-    if (p.loss == TTT_LOSS_MSE && chunk_end) refresh_start();
+    pack_cur();
+    if constexpr (LOSS == TTT_LOSS_MSE)
+      if (chunk_end) start_chunk();
     s += nb;
   }
 
@@ -375,10 +381,12 @@ cudaError_t launch(const LinearArgs& a, cudaStream_t s) {
   p.loss = a.loss;
   p.status = a.status;
   const size_t smem = sizeof(Smem<D>) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(ttt_linear_bf16_kernel<D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kernel = a.loss == TTT_LOSS_MSE ? ttt_linear_bf16_kernel<D, TTT_LOSS_MSE>
+                                       : ttt_linear_bf16_kernel<D, TTT_LOSS_NEG_DOT>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  ttt_linear_bf16_kernel<D><<<a.B * a.H, (D / 16 + 1) * 32, smem, s>>>(p);
+  kernel<<<a.B * a.H, (D / 16 + 1) * 32, smem, s>>>(p);
   return cudaGetLastError();
 }
 
