@@ -182,6 +182,42 @@ __device__ __forceinline__ void fill_rows(uint8_t* s, int lane, const uint8_t* s
   __syncwarp();
 }
 
+// Half-width staging: 32 rows x 64 bytes (2 KB), 16-byte chunk j (0..3) of row
+// r at r * 64 + ((j ^ ((r >> 1) & 3)) << 4) -- conflict-free for a lane writing
+// its row and for four lanes reading one row.
+__device__ __forceinline__ uint32_t sw64(int r, int j) {
+  return (uint32_t)(r * 64 + ((j ^ ((r >> 1) & 3)) << 4));
+}
+__device__ __forceinline__ void put_bf16_64(uint8_t* s, int lane, int p, const float (&v)[16],
+                                            bool lo) {
+  uint32_t w[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    float a = v[2 * u], b = v[2 * u + 1];
+    if (lo) {
+      a -= __bfloat162float(__float2bfloat16_rn(a));
+      b -= __bfloat162float(__float2bfloat16_rn(b));
+    }
+    w[u] = pack_bf16x2(a, b);
+  }
+  *reinterpret_cast<uint4*>(s + sw64(lane, 2 * p)) = make_uint4(w[0], w[1], w[2], w[3]);
+  *reinterpret_cast<uint4*>(s + sw64(lane, 2 * p + 1)) = make_uint4(w[4], w[5], w[6], w[7]);
+}
+// Staged rows r < nrows (64 bytes each) -> dst + r * ld: eight rows per store.
+__device__ __forceinline__ void flush_rows64(const uint8_t* s, int lane, uint8_t* dst, int64_t ld,
+                                             int nrows) {
+  __syncwarp();
+  uint4 x[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) x[i] = *reinterpret_cast<const uint4*>(s + sw64(8 * i + (lane >> 2), lane & 3));
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = 8 * i + (lane >> 2);
+    if (r < nrows) *reinterpret_cast<uint4*>(dst + r * ld + (lane & 3) * 16) = x[i];
+  }
+  __syncwarp();
+}
+
 // The staging buffer of one epilogue warp. Synchronous use (stage, then
 // flush_rows) needs no bookkeeping; a TMA add-reduction reads the buffer
 // asynchronously, so the buffer is rewritten only after that read is done.
@@ -247,6 +283,14 @@ __device__ __forceinline__ TileCoord decode_tile(const Params& P, int t) {
 // (relative error ~1e-7; 1 / inf = 0 for very negative x). A correctly rounded
 // reciprocal costs about ten times as much and dominated the epilogues.
 __device__ __forceinline__ float sigmoidf_(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
+// One special-function op instead of two: sigmoid(x) = (1 + tanh(x / 2)) / 2
+// with the hardware tanh approximation (absolute error about 2.5e-4 on the
+// result), used where the outputs are rounded to bf16 anyway.
+__device__ __forceinline__ float sigmoid_fast(float x) {
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
+  return fmaf(0.5f, t, 0.5f);
+}
 
 // Epilogue for 16 consecutive accumulator columns [c0, c0+16) of row `row` of
 // tile (m0, n0). For EPI_AQ / EPI_HK the tile's 128 columns hold 64 columns of
@@ -305,7 +349,8 @@ __device__ __forceinline__ void epilogue_tile(const Problem& pr, const TileCoord
         float h1[16], h3[16];
         tmem_ld2x16(tbase + c0 + 16 * p, tbase + c0 + kHid + 16 * p, h1, h3);
 #pragma unroll
-        for (int u = 0; u < 16; ++u) a[u] = h1[u] * sigmoidf_(h1[u]) * h3[u];
+        for (int u = 0; u < 16; ++u)
+          a[u] = h1[u] * (split ? sigmoidf_(h1[u]) : sigmoid_fast(h1[u])) * h3[u];
       };
       const int64_t off = (((int64_t)z * e.orows + row0) * e.ocols + hid) * 2;
       emit(static_cast<uint8_t*>(e.optr[0]) + off, ld, false, aq);
@@ -313,17 +358,22 @@ __device__ __forceinline__ void epilogue_tile(const Problem& pr, const TileCoord
       return;
     }
     // EPI_HKG: columns [0, 64) h1, [64, 128) h3, [128, 192) u of hidden units
-    // hid .. hid + 63. Warp half 0 writes ak and dh3, half 1 writes dh1.
-    const int hid = tc.n0 * kHid;
+    // hid .. hid + 63; this warp takes units [32ch, 32ch + 32). The sigmoid of
+    // each h1 is evaluated once and kept; outputs go through the two 2 KB
+    // halves of the staging buffer as 64-byte rows.
+    const int cw = ch * 32;
+    const int hid = tc.n0 * kHid + cw;
     const float eta_i = lane_ok ? eta_of(e, z, row0 + lane) : 0.f;
     auto dst = [&](int o) {
       return static_cast<uint8_t*>(e.optr[o]) + (((int64_t)z * e.orows + row0) * e.ocols + hid) * 2;
     };
+    uint8_t* const bA = buf;
+    uint8_t* const bB = buf + 2048;
     auto load3 = [&](int p, float (&h1)[16], float (&h3)[16], float (&gz)[16]) {
       uint32_t r1[16], r3[16], rg[16];
-      umma::tmem_ld16_async(tbase + 16 * p, r1);
-      umma::tmem_ld16_async(tbase + kHid + 16 * p, r3);
-      umma::tmem_ld16_async(tbase + 2 * kHid + 16 * p, rg);
+      umma::tmem_ld16_async(tbase + cw + 16 * p, r1);
+      umma::tmem_ld16_async(tbase + kHid + cw + 16 * p, r3);
+      umma::tmem_ld16_async(tbase + 2 * kHid + cw + 16 * p, rg);
       umma::tmem_wait_ld(r1);
       umma::tmem_wait_ld(r3);
       umma::tmem_wait_ld(rg);
@@ -334,37 +384,56 @@ __device__ __forceinline__ void epilogue_tile(const Problem& pr, const TileCoord
         gz[u] = -eta_i * __uint_as_float(rg[u]);
       }
     };
-    if (ch == 0) {
-      auto ak = [&](int p, float (&v)[16]) {  // eta * silu(h1) * h3
-        float h1[16], h3[16];
-        tmem_ld2x16(tbase + 16 * p, tbase + kHid + 16 * p, h1, h3);
+    float sgm[2][16];
+    // pass 1: ak = eta silu(h1) h3 (+ dh3 = gz silu(h1) when not split)
 #pragma unroll
-        for (int u = 0; u < 16; ++u) v[u] = eta_i * h1[u] * sigmoidf_(h1[u]) * h3[u];
-      };
-      auto dh3 = [&](int p, float (&v)[16]) {  // gz * silu(h1)
-        float h1[16], h3[16], gz[16];
-        load3(p, h1, h3, gz);
+    for (int p = 0; p < 2; ++p) {
+      float h1[16], h3[16], gz[16], a[16], d[16];
+      load3(p, h1, h3, gz);
 #pragma unroll
-        for (int u = 0; u < 16; ++u) v[u] = gz[u] * h1[u] * sigmoidf_(h1[u]);
-      };
-      emit(dst(0), ld, false, ak);
-      if (split) emit(dst(3), ld, true, ak);
-      emit(dst(2), ld, false, dh3);
-      if (split) emit(dst(5), ld, true, dh3);
-    } else {
-      // dh1 = gz * h3 * silu'(h1),  silu'(x) = sigmoid(x) (1 + x (1 - sigmoid(x)))
-      auto dh1 = [&](int p, float (&v)[16]) {
-        float h1[16], h3[16], gz[16];
-        load3(p, h1, h3, gz);
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const float sg1 = sigmoidf_(h1[u]);
-          v[u] = gz[u] * h3[u] * sg1 * (1.f + h1[u] * (1.f - sg1));
-        }
-      };
-      emit(dst(1), ld, false, dh1);
-      if (split) emit(dst(4), ld, true, dh1);
+      for (int u = 0; u < 16; ++u) {
+        sgm[p][u] = split ? sigmoidf_(h1[u]) : sigmoid_fast(h1[u]);
+        const float s1 = h1[u] * sgm[p][u];
+        a[u] = eta_i * s1 * h3[u];
+        d[u] = gz[u] * s1;
+      }
+      put_bf16_64(bA, lane, p, a, false);
+      if (split)
+        put_bf16_64(bB, lane, p, a, true);
+      else
+        put_bf16_64(bB, lane, p, d, false);
     }
+    flush_rows64(bA, lane, dst(0), ld, nrows);
+    flush_rows64(bB, lane, dst(split ? 3 : 2), ld, nrows);
+    if (split) {
+      // pass 2: dh3 hi / lo
+#pragma unroll
+      for (int p = 0; p < 2; ++p) {
+        float h1[16], h3[16], gz[16], d[16];
+        load3(p, h1, h3, gz);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) d[u] = gz[u] * h1[u] * sgm[p][u];
+        put_bf16_64(bA, lane, p, d, false);
+        put_bf16_64(bB, lane, p, d, true);
+      }
+      flush_rows64(bA, lane, dst(2), ld, nrows);
+      flush_rows64(bB, lane, dst(5), ld, nrows);
+    }
+    // last pass: dh1 = gz h3 silu'(h1),  silu'(x) = sigmoid(x) (1 + x (1 - sigmoid(x)))
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+      float h1[16], h3[16], gz[16], d[16];
+      load3(p, h1, h3, gz);
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const float sg1 = sgm[p][u];
+        d[u] = gz[u] * h3[u] * sg1 * (1.f + h1[u] * (1.f - sg1));
+      }
+      put_bf16_64(bA, lane, p, d, false);
+      if (split) put_bf16_64(bB, lane, p, d, true);
+    }
+    flush_rows64(bA, lane, dst(1), ld, nrows);
+    if (split) flush_rows64(bB, lane, dst(4), ld, nrows);
     return;
   }
 

@@ -22,6 +22,7 @@
 // Precision: GD uses bf16 operands with fp32 accumulation; Muon uses
 // split-bf16 operands (x = hi + lo, products hi*hi + lo*hi + hi*lo) because
 // the unit-step Muon scan amplifies per-chunk rounding across chunks.
+#include <cooperative_groups.h>
 #include <vector>
 
 #include "gemm_tc.cuh"
@@ -334,6 +335,186 @@ __global__ void __cluster_dims__(kNsCluster, 1, 1) __launch_bounds__(kNsThreads)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Newton-Schulz for 128 x 512 (or 512 x 128) gradients with every operand in
+// shared memory: a cluster of kNsCluster CTAs per matrix, CTA c owning the
+// 128 x 128 slab c of the long side. The slab X, the Gram matrix G and the
+// polynomial P live in shared memory as bf16 hi / lo pairs (x = hi + lo to
+// about 16 bits), so the split-bf16 products hi*hi + lo*hi + hi*lo read their
+// fragments straight from shared memory. Gram partials are summed across the
+// cluster through distributed shared memory: CTA c reduces rows [32c, 32c+32)
+// of G and writes them into every CTA's copy.
+// ---------------------------------------------------------------------------
+
+constexpr int kN5 = 128;          // slab side
+constexpr int kN5Ld = kN5 + 8;    // padded row (bf16): conflict-free ldmatrix
+constexpr int kN5Threads = 512;   // 16 warps, warp tile 32 x 32
+
+struct Ns128Smem {
+  __nv_bfloat16 x[2][kN5 * kN5Ld];  // hi, lo
+  __nv_bfloat16 g[2][kN5 * kN5Ld];
+  __nv_bfloat16 p[2][kN5 * kN5Ld];  // also holds the fp32 Gram partial [128][128]
+  float nrm;
+};
+
+__device__ __forceinline__ void split_store(__nv_bfloat16* hi, __nv_bfloat16* lo, int idx, float v) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(v);
+  hi[idx] = h;
+  lo[idx] = __float2bfloat16_rn(v - __bfloat162float(h));
+}
+
+// acc (warp tile rows 32wm + 16mt + {g, g+8}, columns 32wn + 8nt + 2c4 + {0,1})
+// = op(A) op(B) over k = 0..127 with split-bf16 products. TA: A is stored
+// [k][m] (A = S^T); TB: B is stored [k][n] (row-major); otherwise A is [m][k]
+// and B is stored [n][k].
+template <bool TA, bool TB>
+__device__ __forceinline__ void ns128_gemm(const __nv_bfloat16* const (&A)[2],
+                                           const __nv_bfloat16* const (&B)[2],
+                                           float (&acc)[2][4][4]) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wm = warp >> 2, wn = warp & 3, mi = lane >> 3, rr = lane & 7;
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[mt][nt][q] = 0.f;
+#pragma unroll 2
+  for (int k0 = 0; k0 < kN5; k0 += 16) {
+    uint32_t af[2][2][4], bf[2][4][2];  // [hi|lo][m-tile][4], [hi|lo][n-tile][2]
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        const int m0 = 32 * wm + 16 * mt;
+        if (TA)
+          ns_ldsm_x4_t(af[x][mt], A[x] + (k0 + rr + 8 * (mi >> 1)) * kN5Ld + m0 + 8 * (mi & 1));
+        else
+          ns_ldsm_x4(af[x][mt], A[x] + (m0 + rr + 8 * (mi & 1)) * kN5Ld + k0 + 8 * (mi >> 1));
+      }
+#pragma unroll
+      for (int np = 0; np < 2; ++np) {  // pairs of n-tiles
+        const int n0 = 32 * wn + 16 * np;
+        uint32_t r[4];
+        if (TB)
+          ns_ldsm_x4_t(r, B[x] + (k0 + rr + 8 * (mi & 1)) * kN5Ld + n0 + 8 * (mi >> 1));
+        else
+          ns_ldsm_x4(r, B[x] + (n0 + rr + 8 * (mi >> 1)) * kN5Ld + k0 + 8 * (mi & 1));
+        bf[x][2 * np][0] = r[0];
+        bf[x][2 * np][1] = r[1];
+        bf[x][2 * np + 1][0] = r[2];
+        bf[x][2 * np + 1][1] = r[3];
+      }
+    }
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) {
+        ns_mma(acc[mt][nt], af[0][mt], bf[0][nt][0], bf[0][nt][1]);  // hi * hi
+        ns_mma(acc[mt][nt], af[1][mt], bf[0][nt][0], bf[0][nt][1]);  // lo * hi
+        ns_mma(acc[mt][nt], af[0][mt], bf[1][nt][0], bf[1][nt][1]);  // hi * lo
+      }
+  }
+}
+
+// Visits the warp's accumulator elements: f(row, col, value).
+template <class F>
+__device__ __forceinline__ void ns128_each(const float (&acc)[2][4][4], F&& f) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wm = warp >> 2, wn = warp & 3, g = lane >> 2, c4 = lane & 3;
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        f(32 * wm + 16 * mt + g + 8 * (q >> 1), 32 * wn + 8 * nt + 2 * c4 + (q & 1), acc[mt][nt][q]);
+}
+
+__global__ void __cluster_dims__(kNsCluster, 1, 1) __launch_bounds__(kN5Threads, 1)
+    ns128_kernel(NsArgs a) {
+  extern __shared__ __align__(16) uint8_t ns_smem_raw[];
+  Ns128Smem& sm = *reinterpret_cast<Ns128Smem*>(ns_smem_raw);
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int mat = blockIdx.x / kNsCluster, c = (int)cluster.block_rank();
+  const int z = mat / 3, m = mat % 3;
+  const int R = a.rows[m], C = a.cols[m];
+  const bool tall = R >= C;
+  float* Xc = a.G[m] + (int64_t)z * R * C + (tall ? (int64_t)c * kN5 * C : (int64_t)c * kN5);
+  const int tid = threadIdx.x;
+
+  // Frobenius norm of the whole matrix (four slabs)
+  float ss = 0.f;
+  for (int e = tid; e < kN5 * kN5; e += kN5Threads) {
+    const float v = Xc[(int64_t)(e >> 7) * C + (e & 127)];
+    ss += v * v;
+  }
+  ss = block_sum(ss);
+  if (tid == 0) sm.nrm = ss;
+  cluster.sync();
+  float tot = 0.f;
+  for (int r = 0; r < kNsCluster; ++r) tot += *cluster.map_shared_rank(&sm.nrm, r);
+  const float inv = 1.f / (sqrtf(tot) + a.eps);
+  for (int e = tid; e < kN5 * kN5; e += kN5Threads) {
+    const int i = e >> 7, j = e & 127;
+    split_store(sm.x[0], sm.x[1], i * kN5Ld + j, Xc[(int64_t)i * C + j] * inv);
+  }
+  __syncthreads();
+
+  const __nv_bfloat16* const X2[2] = {sm.x[0], sm.x[1]};
+  const __nv_bfloat16* const G2[2] = {sm.g[0], sm.g[1]};
+  const __nv_bfloat16* const P2[2] = {sm.p[0], sm.p[1]};
+  float* part = reinterpret_cast<float*>(sm.p[0]);  // [128][128] fp32, spans p[0] and p[1]
+  float acc[2][4][4];
+  for (int it = 0; it < a.steps; ++it) {
+    // Gram partial of this slab: tall X^T X, wide X X^T
+    if (tall)
+      ns128_gemm<true, true>(X2, X2, acc);
+    else
+      ns128_gemm<false, false>(X2, X2, acc);
+    ns128_each(acc, [&](int i, int j, float v) { part[i * kN5 + j] = v; });
+    cluster.sync();
+    // rows [32c, 32c + 32) of G = sum of the four partials, into every CTA's G
+    for (int e = tid; e < 32 * kN5; e += kN5Threads) {
+      const int i = 32 * c + (e >> 7), j = e & 127;
+      float gsum = 0.f;
+      for (int r = 0; r < kNsCluster; ++r) gsum += cluster.map_shared_rank(part, r)[i * kN5 + j];
+      const __nv_bfloat16 h = __float2bfloat16_rn(gsum);
+      const __nv_bfloat16 l = __float2bfloat16_rn(gsum - __bfloat162float(h));
+      for (int r = 0; r < kNsCluster; ++r) {
+        cluster.map_shared_rank(sm.g[0], r)[i * kN5Ld + j] = h;
+        cluster.map_shared_rank(sm.g[1], r)[i * kN5Ld + j] = l;
+      }
+    }
+    cluster.sync();
+    // P = c G^2 + b G
+    ns128_gemm<false, true>(G2, G2, acc);
+    ns128_each(acc, [&](int i, int j, float v) {
+      const float gij = __bfloat162float(sm.g[0][i * kN5Ld + j]) + __bfloat162float(sm.g[1][i * kN5Ld + j]);
+      split_store(sm.p[0], sm.p[1], i * kN5Ld + j, a.c * v + a.b * gij);
+    });
+    __syncthreads();
+    // X <- a X + X P (tall) or a X + P X (wide)
+    if (tall)
+      ns128_gemm<false, true>(X2, P2, acc);
+    else
+      ns128_gemm<false, true>(P2, X2, acc);
+    __syncthreads();  // every warp is done reading X
+    const bool last = it + 1 == a.steps;
+    ns128_each(acc, [&](int i, int j, float v) {
+      const float xij = __bfloat162float(sm.x[0][i * kN5Ld + j]) + __bfloat162float(sm.x[1][i * kN5Ld + j]);
+      const float xn = a.a * xij + v;
+      if (last)
+        Xc[(int64_t)i * C + j] = xn;
+      else
+        split_store(sm.x[0], sm.x[1], i * kN5Ld + j, xn);
+    });
+    __syncthreads();
+  }
+  cluster.sync();  // no CTA leaves while another may still read its shared memory
+}
+
 __global__ void copy_kernel(float* dst, const float* src, int64_t n) {
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x)
@@ -640,6 +821,11 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
     na.steps = 5;
   }
 
+  // Gradients of 512 x 128 / 128 x 512 run the shared-memory-resident kernel.
+  const bool ns128 = split && dk == kN5 && dv == kN5 && dh == kNsCluster * kN5;
+  if (ns128)
+    check(cudaFuncSetAttribute(ns128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)sizeof(Ns128Smem)));
   const int* segW = split ? &kSegBsplit[0][0] : &kSegExact[0][0];
   const int nsegW = split ? 2 : 1;
 
@@ -794,7 +980,11 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
     }
     // L3 / L4: Muon orthogonalisation, update and row renormalisation
     if (split) {
-      ns_kernel<<<Z * 3 * kNsCluster, kNsThreads, 0, s>>>(na);
+      if (ns128) {
+        ns128_kernel<<<Z * 3 * kNsCluster, kN5Threads, sizeof(Ns128Smem), s>>>(na);
+      } else {
+        ns_kernel<<<Z * 3 * kNsCluster, kNsThreads, 0, s>>>(na);
+      }
       check(cudaGetLastError());
     }
     lact_rows_kernel<<<row_blocks, 256, 0, s>>>(ra);

@@ -42,8 +42,16 @@ def test_gd_non_causal():
 
 
 def test_muon_small():
+    """d = 128, hidden 512: the shared-memory-resident Newton-Schulz path."""
     w = synth.make_lact(1, 2, 1024, 128, 512, 256, synth.UPDATE_MUON, seed=5)
     compare(w, "muon")
+
+
+@pytest.mark.parametrize("d,dh", [(64, 128), (256, 512), (128, 256)])
+def test_muon_other_shapes(d, dh):
+    """Gradient shapes outside 128 x 512 take the general cluster Newton-Schulz."""
+    w = synth.make_lact(1, 2, 512, d, dh, 256, synth.UPDATE_MUON, seed=d + dh + 1)
+    compare(w, f"muon d{d} dh{dh}")
 
 
 def test_gd_full_size_workload():
