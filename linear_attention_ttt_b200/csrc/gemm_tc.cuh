@@ -24,6 +24,8 @@
 // add-reductions. All barrier waits are bounded.
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "tma.cuh"
 #include "umma.cuh"
@@ -121,14 +123,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 }
 
 // Row `lane` of the buffer, columns [16p, 16p + 16) as bf16 (chunks 2p, 2p+1):
-// bf16(v), or the residual v - bf16(v) when lo.
-__device__ __forceinline__ void put_bf16(uint8_t* s, int lane, int p, const float (&v)[16],
-                                         bool lo) {
+// bf16(v), or the residual v - bf16(v) for LO.
+template <bool LO>
+__device__ __forceinline__ void put_bf16(uint8_t* s, int lane, int p, const float (&v)[16]) {
   uint32_t w[8];
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
     float a = v[2 * u], b = v[2 * u + 1];
-    if (lo) {
+    if constexpr (LO) {
       a -= __bfloat162float(__float2bfloat16_rn(a));
       b -= __bfloat162float(__float2bfloat16_rn(b));
     }
@@ -188,13 +190,13 @@ __device__ __forceinline__ void fill_rows(uint8_t* s, int lane, const uint8_t* s
 __device__ __forceinline__ uint32_t sw64(int r, int j) {
   return (uint32_t)(r * 64 + ((j ^ ((r >> 1) & 3)) << 4));
 }
-__device__ __forceinline__ void put_bf16_64(uint8_t* s, int lane, int p, const float (&v)[16],
-                                            bool lo) {
+template <bool LO>
+__device__ __forceinline__ void put_bf16_64(uint8_t* s, int lane, int p, const float (&v)[16]) {
   uint32_t w[8];
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
     float a = v[2 * u], b = v[2 * u + 1];
-    if (lo) {
+    if constexpr (LO) {
       a -= __bfloat162float(__float2bfloat16_rn(a));
       b -= __bfloat162float(__float2bfloat16_rn(b));
     }
@@ -313,54 +315,53 @@ __device__ __forceinline__ void k_range(const Problem& pr, int ks, int& kb0, int
 // Epilogue of one accumulator tile, run by one warp: its 32 TMEM lanes (tile
 // rows quarter*32 ...) and the columns of half `ch` (0 or 1) of the tile.
 // Rows at or beyond min(M, rows_valid) are not written.
-template <int BN>
-__device__ __forceinline__ void epilogue_tile(const Problem& pr, const TileCoord& tc, int quarter,
-                                              uint32_t tbase, bool live_tile, int ch, Stage& sg) {
+template <int BN, int EPI, bool SPLIT>
+__device__ __forceinline__ void epilogue_body(const Problem& pr, const TileCoord& tc, int quarter,
+                                              uint32_t tbase, int ch, Stage& sg) {
   const EpiArgs& e = pr.e;
   const int z = tc.z, n0 = tc.n0 * pr.tn;
   const int row0 = tc.m0 + quarter * 32;  // first tile row of this warp
-  const int lim = min(pr.M, e.rows_valid);
-  if (!live_tile || row0 >= lim) return;   // warp-uniform
-  const int nrows = min(32, lim - row0);
+  const int nrows = min(32, min(pr.M, e.rows_valid) - row0);
   const int lane = sg.lane;
   const bool lane_ok = lane < nrows;       // this lane's row exists
   uint8_t* const buf = sg.buf;
   sg.drain();
   // 64 bf16 columns of this warp's rows: values of columns [16p, 16p + 16)
-  // from val(p, v), staged as bf16 (or residuals when lo), then written.
-  auto emit = [&](uint8_t* d, int64_t ld, bool lo, auto&& val) {
+  // from val(p, v), staged as bf16 (or as residuals for LO), then written.
+  auto emit = [&](uint8_t* d, int64_t ld, auto lo_c, auto&& val) {
+    constexpr bool LO = decltype(lo_c)::value;
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
       float v[16];
       val(p, v);
-      put_bf16(buf, lane, p, v, lo);
+      put_bf16<LO>(buf, lane, p, v);
     }
     flush_rows(buf, lane, d, ld, nrows);
   };
+  using Hi = std::false_type;
+  using Lo = std::true_type;
 
-  if (pr.epi == EPI_AQ || pr.epi == EPI_HKG) {
+  if constexpr (EPI == EPI_AQ) {
+    // tile columns [128ch, 128ch + 64) h1, [128ch + 64, 128ch + 128) h3
     const int64_t ld = (int64_t)e.ocols * 2;
-    const bool split = e.nsplit > 1;
-    if (pr.epi == EPI_AQ) {
-      // tile columns [128ch, 128ch + 64) h1, [128ch + 64, 128ch + 128) h3
-      const int c0 = ch * 2 * kHid;
-      const int hid = n0 / 2 + ch * kHid;
-      auto aq = [&](int p, float (&a)[16]) {
-        float h1[16], h3[16];
-        tmem_ld2x16(tbase + c0 + 16 * p, tbase + c0 + kHid + 16 * p, h1, h3);
+    const int c0 = ch * 2 * kHid;
+    const int hid = n0 / 2 + ch * kHid;
+    auto aq = [&](int p, float (&a)[16]) {
+      float h1[16], h3[16];
+      tmem_ld2x16(tbase + c0 + 16 * p, tbase + c0 + kHid + 16 * p, h1, h3);
 #pragma unroll
-        for (int u = 0; u < 16; ++u)
-          a[u] = h1[u] * (split ? sigmoidf_(h1[u]) : sigmoid_fast(h1[u])) * h3[u];
-      };
-      const int64_t off = (((int64_t)z * e.orows + row0) * e.ocols + hid) * 2;
-      emit(static_cast<uint8_t*>(e.optr[0]) + off, ld, false, aq);
-      if (split) emit(static_cast<uint8_t*>(e.optr[3]) + off, ld, true, aq);
-      return;
-    }
-    // EPI_HKG: columns [0, 64) h1, [64, 128) h3, [128, 192) u of hidden units
+      for (int u = 0; u < 16; ++u)
+        a[u] = h1[u] * (SPLIT ? sigmoidf_(h1[u]) : sigmoid_fast(h1[u])) * h3[u];
+    };
+    const int64_t off = (((int64_t)z * e.orows + row0) * e.ocols + hid) * 2;
+    emit(static_cast<uint8_t*>(e.optr[0]) + off, ld, Hi{}, aq);
+    if constexpr (SPLIT) emit(static_cast<uint8_t*>(e.optr[3]) + off, ld, Lo{}, aq);
+  } else if constexpr (EPI == EPI_HKG) {
+    // columns [0, 64) h1, [64, 128) h3, [128, 192) u of hidden units
     // hid .. hid + 63; this warp takes units [32ch, 32ch + 32). The sigmoid of
     // each h1 is evaluated once and kept; outputs go through the two 2 KB
     // halves of the staging buffer as 64-byte rows.
+    const int64_t ld = (int64_t)e.ocols * 2;
     const int cw = ch * 32;
     const int hid = tc.n0 * kHid + cw;
     const float eta_i = lane_ok ? eta_of(e, z, row0 + lane) : 0.f;
@@ -392,20 +393,20 @@ __device__ __forceinline__ void epilogue_tile(const Problem& pr, const TileCoord
       load3(p, h1, h3, gz);
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
-        sgm[p][u] = split ? sigmoidf_(h1[u]) : sigmoid_fast(h1[u]);
+        sgm[p][u] = SPLIT ? sigmoidf_(h1[u]) : sigmoid_fast(h1[u]);
         const float s1 = h1[u] * sgm[p][u];
         a[u] = eta_i * s1 * h3[u];
         d[u] = gz[u] * s1;
       }
-      put_bf16_64(bA, lane, p, a, false);
-      if (split)
-        put_bf16_64(bB, lane, p, a, true);
+      put_bf16_64<false>(bA, lane, p, a);
+      if constexpr (SPLIT)
+        put_bf16_64<true>(bB, lane, p, a);
       else
-        put_bf16_64(bB, lane, p, d, false);
+        put_bf16_64<false>(bB, lane, p, d);
     }
     flush_rows64(bA, lane, dst(0), ld, nrows);
-    flush_rows64(bB, lane, dst(split ? 3 : 2), ld, nrows);
-    if (split) {
+    flush_rows64(bB, lane, dst(SPLIT ? 3 : 2), ld, nrows);
+    if constexpr (SPLIT) {
       // pass 2: dh3 hi / lo
 #pragma unroll
       for (int p = 0; p < 2; ++p) {
@@ -413,8 +414,8 @@ __device__ __forceinline__ void epilogue_tile(const Problem& pr, const TileCoord
         load3(p, h1, h3, gz);
 #pragma unroll
         for (int u = 0; u < 16; ++u) d[u] = gz[u] * h1[u] * sgm[p][u];
-        put_bf16_64(bA, lane, p, d, false);
-        put_bf16_64(bB, lane, p, d, true);
+        put_bf16_64<false>(bA, lane, p, d);
+        put_bf16_64<true>(bB, lane, p, d);
       }
       flush_rows64(bA, lane, dst(2), ld, nrows);
       flush_rows64(bB, lane, dst(5), ld, nrows);
@@ -429,66 +430,90 @@ __device__ __forceinline__ void epilogue_tile(const Problem& pr, const TileCoord
         const float sg1 = sgm[p][u];
         d[u] = gz[u] * h3[u] * sg1 * (1.f + h1[u] * (1.f - sg1));
       }
-      put_bf16_64(bA, lane, p, d, false);
-      if (split) put_bf16_64(bB, lane, p, d, true);
+      put_bf16_64<false>(bA, lane, p, d);
+      if constexpr (SPLIT) put_bf16_64<true>(bB, lane, p, d);
     }
     flush_rows64(bA, lane, dst(1), ld, nrows);
-    if (split) flush_rows64(bB, lane, dst(4), ld, nrows);
-    return;
-  }
-
-  if (pr.epi == EPI_GRAD) {
+    if constexpr (SPLIT) flush_rows64(bB, lane, dst(4), ld, nrows);
+  } else if constexpr (EPI == EPI_GRAD) {
     const int oz2 = z % e.ozdiv, oz3 = z / e.ozdiv;
     for (int gi = 0; gi < pr.tn / 64; ++gi) {   // 32 fp32 columns per group
       const int gc = n0 + ch * (pr.tn / 2) + 32 * gi;
       if (gc >= pr.N) break;
       float v[16], w[16];
       tmem_ld2x16(tbase + gc - n0, tbase + gc - n0 + 16, v, w);
-      if (e.scale != 1.f)
+      const float sc = e.scale;
 #pragma unroll
-        for (int u = 0; u < 16; ++u) v[u] *= e.scale, w[u] *= e.scale;
+      for (int u = 0; u < 16; ++u) v[u] *= sc, w[u] *= sc;
       sg.drain();  // the previous reduction has read the buffer
       put_f32(buf, lane, 0, v);
       put_f32(buf, lane, 1, w);
       sg.reduce(&e.gmap, gc, row0, oz2, oz3);
     }
-    return;
-  }
-
-  const int b = z / e.H, h = z % e.H;
-  const int64_t es = e.out_bf16 ? 2 : 4;
-  uint8_t* base = static_cast<uint8_t*>(e.out.p) +
-                  ((int64_t)b * e.out.sb + (int64_t)h * e.out.sh +
-                   (int64_t)(e.orow0 + row0) * e.out.st) * es;
-  const int64_t ld = e.out.st * es;
-  if (!e.out_bf16) {
-    // EPI_Y, fp32 output tokens: 32 columns per group
-    for (int gi = 0; gi < pr.tn / 64; ++gi) {
-      const int gc = n0 + ch * (pr.tn / 2) + 32 * gi;
-      if (gc >= pr.N) break;
-      float v[16], w[16];
-      tmem_ld2x16(tbase + gc - n0, tbase + gc - n0 + 16, v, w);
-      put_f32(buf, lane, 0, v);
-      put_f32(buf, lane, 1, w);
-      flush_rows(buf, lane, base + (int64_t)gc * 4, ld, nrows);
-    }
-    return;
-  }
-  // EPI_Y, bf16 output tokens: 64 columns per group
-  for (int gi = 0; gi < pr.tn / 128; ++gi) {
-    const int gc = n0 + ch * (pr.tn / 2) + 64 * gi;
-    if (gc >= pr.N) break;
-    auto y = [&](int p, float (&v)[16]) {
-      uint32_t r[16];
-      umma::tmem_ld16_async(tbase + gc - n0 + 16 * p, r);
-      umma::tmem_wait_ld(r);
+  } else {  // EPI_Y
+    const int b = z / e.H, h = z % e.H;
+    constexpr int64_t es = SPLIT ? 4 : 2;  // SPLIT selects fp32 output tokens here
+    uint8_t* base = static_cast<uint8_t*>(e.out.p) +
+                    ((int64_t)b * e.out.sb + (int64_t)h * e.out.sh +
+                     (int64_t)(e.orow0 + row0) * e.out.st) * es;
+    const int64_t ld = e.out.st * es;
+    if constexpr (SPLIT) {
+      // fp32 output tokens: 32 columns per group
+      for (int gi = 0; gi < pr.tn / 64; ++gi) {
+        const int gc = n0 + ch * (pr.tn / 2) + 32 * gi;
+        if (gc >= pr.N) break;
+        float v[16], w[16];
+        tmem_ld2x16(tbase + gc - n0, tbase + gc - n0 + 16, v, w);
+        put_f32(buf, lane, 0, v);
+        put_f32(buf, lane, 1, w);
+        flush_rows(buf, lane, base + (int64_t)gc * 4, ld, nrows);
+      }
+    } else {
+      // bf16 output tokens: 64 columns per group
+      for (int gi = 0; gi < pr.tn / 128; ++gi) {
+        const int gc = n0 + ch * (pr.tn / 2) + 64 * gi;
+        if (gc >= pr.N) break;
+        auto y = [&](int p, float (&v)[16]) {
+          uint32_t r[16];
+          umma::tmem_ld16_async(tbase + gc - n0 + 16 * p, r);
+          umma::tmem_wait_ld(r);
 #pragma unroll
-      for (int u = 0; u < 16; ++u) v[u] = __uint_as_float(r[u]);
-    };
-    emit(base + (int64_t)gc * 2, ld, false, y);
+          for (int u = 0; u < 16; ++u) v[u] = __uint_as_float(r[u]);
+        };
+        emit(base + (int64_t)gc * 2, ld, Hi{}, y);
+      }
+    }
   }
 }
 
+// Epilogue of one accumulator tile, run by one warp: its 32 TMEM lanes (tile
+// rows quarter*32 ...) and the columns of half `ch` (0 or 1) of the tile.
+// Rows at or beyond min(M, rows_valid) are not written. Each (kind, precision)
+// pair is a separate straight-line instantiation.
+template <int BN>
+__device__ __forceinline__ void epilogue_tile(const Problem& pr, const TileCoord& tc, int quarter,
+                                              uint32_t tbase, bool live_tile, int ch, Stage& sg) {
+  const int row0 = tc.m0 + quarter * 32;
+  if (!live_tile || row0 >= min(pr.M, pr.e.rows_valid)) return;  // warp-uniform
+  const bool split = pr.e.nsplit > 1;
+  switch (pr.epi) {
+    case EPI_AQ:
+      if (split) epilogue_body<BN, EPI_AQ, true>(pr, tc, quarter, tbase, ch, sg);
+      else epilogue_body<BN, EPI_AQ, false>(pr, tc, quarter, tbase, ch, sg);
+      break;
+    case EPI_HKG:
+      if (split) epilogue_body<BN, EPI_HKG, true>(pr, tc, quarter, tbase, ch, sg);
+      else epilogue_body<BN, EPI_HKG, false>(pr, tc, quarter, tbase, ch, sg);
+      break;
+    case EPI_GRAD:
+      epilogue_body<BN, EPI_GRAD, false>(pr, tc, quarter, tbase, ch, sg);
+      break;
+    default:
+      if (pr.e.out_bf16) epilogue_body<BN, EPI_Y, false>(pr, tc, quarter, tbase, ch, sg);
+      else epilogue_body<BN, EPI_Y, true>(pr, tc, quarter, tbase, ch, sg);
+      break;
+  }
+}
 template <int BN>
 __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant__ Params P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
