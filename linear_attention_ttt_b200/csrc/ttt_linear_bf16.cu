@@ -396,6 +396,7 @@ cudaError_t launch_ttt_linear_bf16(const LinearArgs& a, cudaStream_t s, bool* su
   *supported = (a.dk == a.dv) && (a.dk == 64 || a.dk == 128);
   if (!*supported) return cudaSuccess;
   if (la_tc_supported(a)) return launch_la_tc(a, s);
+  if (ttt_linear_wy_supported(a)) return launch_ttt_linear_wy(a, s);
   return a.dk == 64 ? launch<64>(a, s) : launch<128>(a, s);
 }
 
