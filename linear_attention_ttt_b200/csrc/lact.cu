@@ -593,12 +593,25 @@ int num_sms() {
 }
 
 // Persistent launch: one CTA per SM (or fewer if there are fewer tiles).
+// The dynamic shared-memory limit of the GEMM kernel is raised once per device.
+cudaError_t gemm_attr_once() {
+  constexpr int kMaxDevices = 64;
+  static bool done[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  if (dev < kMaxDevices && done[dev]) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(gemm::gemm_kernel<BN>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)(sizeof(gemm::Smem<BN>) + 1024));
+  if (e == cudaSuccess && dev < kMaxDevices) done[dev] = true;
+  return e;
+}
+
 cudaError_t launch_gemm(Params& P, cudaStream_t s) {
   fill_problem_tiles(P);
   if (P.total_tiles == 0) return cudaSuccess;
   const size_t smem = sizeof(gemm::Smem<BN>) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(gemm::gemm_kernel<BN>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = gemm_attr_once();
   if (e != cudaSuccess) return e;
   const int grid = P.total_tiles < num_sms() ? P.total_tiles : num_sms();
   gemm::gemm_kernel<BN><<<grid, gemm::kThreads, smem, s>>>(P);
@@ -829,28 +842,48 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
   const int* segW = split ? &kSegBsplit[0][0] : &kSegExact[0][0];
   const int nsegW = split ? 2 : 1;
 
-  for (int s0 = 0; s0 < a.T && result == TTT_OK; s0 += chunk) {
-    const int bc = (a.T - s0) < chunk ? (a.T - s0) : chunk;
-    // shared operands for this chunk
-    Operand W13, W13h, W2mn, W2k, Qk, Kk, Vk, Kmn, Vmn, AQk, DH1mn, DH3mn, AKmn;
+  // Tensor maps do not depend on the chunk (token operands carry the chunk
+  // start as a row offset); the chunk-length activation maps are built once
+  // for full chunks and once more for a ragged last chunk.
+  Operand W13, W13h, W2mn, W2k, Qk0, Kk0, Vk0, Kmn0, Vmn0;
+  struct ActOps {
+    Operand AQk, DH1mn, DH3mn, AKmn;
+  } act_full, act_last;
+  CUtensorMap gmaps[3];
+  if (a.T > 0) {
     bool ok = true;
     ok &= buf_op(W13, sc.w13, Z, 2 * dh, 2 * dh, dk, 0, BN, split);
     ok &= buf_op(W13h, sc.w13, Z, 2 * dh, 2 * dh, dk, 0, 2 * gemm::kHid, split);
     ok &= buf_op(W2mn, sc.w2, Z, dv, dv, dh, 1, 64, split);
     ok &= buf_op(W2k, sc.w2, Z, dv, dv, dh, 0, BN, split);
-    ok &= tok_kmajor(Qk, a.q, a, dk, s0, gemm::BM);
-    ok &= tok_kmajor(Kk, a.k, a, dk, s0, gemm::BM);
-    ok &= tok_kmajor(Vk, a.v, a, dv, s0, gemm::BM);
-    ok &= tok_mnmajor(Kmn, a.k, a, dk, s0);
-    ok &= tok_mnmajor(Vmn, a.v, a, dv, s0);
-    ok &= buf_op(AQk, sc.aq, Z, bc, chunk, dh, 0, gemm::BM, split);
-    ok &= buf_op(DH1mn, sc.dh1, Z, bc, chunk, dh, 1, 64, split);
-    ok &= buf_op(DH3mn, sc.dh3, Z, bc, chunk, dh, 1, 64, split);
-    ok &= buf_op(AKmn, sc.ak, Z, bc, chunk, dh, 1, 64, split);
-    if (!ok) {
-      result = TTT_ERR_CUDA;
-      break;
-    }
+    ok &= tok_kmajor(Qk0, a.q, a, dk, 0, gemm::BM);
+    ok &= tok_kmajor(Kk0, a.k, a, dk, 0, gemm::BM);
+    ok &= tok_kmajor(Vk0, a.v, a, dv, 0, gemm::BM);
+    ok &= tok_mnmajor(Kmn0, a.k, a, dk, 0);
+    ok &= tok_mnmajor(Vmn0, a.v, a, dv, 0);
+    auto acts = [&](ActOps& o, int rows) {
+      return buf_op(o.AQk, sc.aq, Z, rows, chunk, dh, 0, gemm::BM, split) &&
+             buf_op(o.DH1mn, sc.dh1, Z, rows, chunk, dh, 1, 64, split) &&
+             buf_op(o.DH3mn, sc.dh3, Z, rows, chunk, dh, 1, 64, split) &&
+             buf_op(o.AKmn, sc.ak, Z, rows, chunk, dh, 1, 64, split);
+    };
+    ok &= acts(act_full, chunk);
+    const int last = a.T > 0 ? a.T - ((a.T - 1) / chunk) * chunk : chunk;
+    ok &= last == chunk ? true : acts(act_last, last);
+    if (last == chunk) act_last = act_full;
+    ok &= grad_map(&gmaps[0], sc.G[0], Z, dh, dk);
+    ok &= grad_map(&gmaps[1], sc.G[1], Z, dh, dk);
+    ok &= grad_map(&gmaps[2], sc.G[2], Z, dv, dh);
+    if (!ok) result = TTT_ERR_CUDA;
+  }
+
+  for (int s0 = 0; s0 < a.T && result == TTT_OK; s0 += chunk) {
+    const int bc = (a.T - s0) < chunk ? (a.T - s0) : chunk;
+    // operands of this chunk
+    Operand Qk = Qk0, Kk = Kk0, Vk = Vk0, Kmn = Kmn0, Vmn = Vmn0;
+    Qk.row0 = Kk.row0 = Vk.row0 = Kmn.row0 = Vmn.row0 = s0;
+    const ActOps& act = bc == chunk ? act_full : act_last;
+    const Operand &AQk = act.AQk, &DH1mn = act.DH1mn, &DH3mn = act.DH3mn, &AKmn = act.AKmn;
     bool okm = true;  // output maps built
     auto new_problem = [&](Params& P) -> Problem& {
       Problem& p = P.p[P.nprob++];
@@ -939,7 +972,7 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
             segs(p, 1, kSegExact);
           p.e = epi_base(a, s0, dh);
           p.e.ozdiv = Z;
-          okm &= grad_map(&p.e.gmap, g == 0 ? sc.G[0] : sc.G[1], Z, dh, dk);
+          p.e.gmap = gmaps[g];
         } else {
           p.a = Vmn;
           p.b = AKmn;
@@ -952,7 +985,7 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
           p.e = epi_base(a, s0, dv);
           p.e.ozdiv = Z;
           p.e.scale = -1.f;
-          okm &= grad_map(&p.e.gmap, sc.G[2], Z, dv, dh);
+          p.e.gmap = gmaps[2];
         }
       }
     };

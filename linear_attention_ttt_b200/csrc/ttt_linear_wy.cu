@@ -45,10 +45,28 @@ constexpr int kThreads = (kWarps + 1) * 32;
 constexpr int kTile = kG * D * 2;  // one [64 x 64] bf16 tile, 8 KB
 constexpr int kProducts = 16;      // 10 Q K^T blocks + 6 K K^T blocks
 
-// Product p = 4w + j: kind (0: S = Q_c K_c'^T, 1: M = K_c K_c'^T), c, c'.
-__device__ __constant__ int kProd[kProducts][3] = {
-    {0, 0, 0}, {0, 1, 0}, {0, 1, 1}, {0, 2, 0}, {0, 2, 1}, {0, 2, 2}, {0, 3, 0}, {0, 3, 1},
-    {0, 3, 2}, {0, 3, 3}, {1, 1, 0}, {1, 2, 0}, {1, 2, 1}, {1, 3, 0}, {1, 3, 1}, {1, 3, 2}};
+// Product p = 4w + j: kind (0: S = Q_c K_c'^T, 1: M = K_c K_c'^T), c, c',
+// as codes kind << 4 | c << 2 | c', one byte each in two 64-bit literals:
+//   S (0,0) (1,0) (1,1) (2,0) (2,1) (2,2) (3,0) (3,1) (3,2) (3,3),
+//   M (1,0) (2,0) (2,1) (3,0) (3,1) (3,2).
+__host__ __device__ constexpr int prod_code(int kind, int c, int cp) {
+  return (kind << 4) | (c << 2) | cp;
+}
+__host__ __device__ constexpr uint64_t prod_bits(int lo) {
+  const int codes[kProducts] = {prod_code(0, 0, 0), prod_code(0, 1, 0), prod_code(0, 1, 1),
+                                prod_code(0, 2, 0), prod_code(0, 2, 1), prod_code(0, 2, 2),
+                                prod_code(0, 3, 0), prod_code(0, 3, 1), prod_code(0, 3, 2),
+                                prod_code(0, 3, 3), prod_code(1, 1, 0), prod_code(1, 2, 0),
+                                prod_code(1, 2, 1), prod_code(1, 3, 0), prod_code(1, 3, 1),
+                                prod_code(1, 3, 2)};
+  uint64_t b = 0;
+  for (int i = 0; i < 8; ++i) b |= (uint64_t)codes[lo + i] << (8 * i);
+  return b;
+}
+__device__ __forceinline__ int prod_of(int pi) {
+  constexpr uint64_t kLo = prod_bits(0), kHi = prod_bits(8);
+  return (int)(((pi < 8 ? kLo : kHi) >> (8 * (pi & 7))) & 0x1f);
+}
 // Index of S block (c, c') and M block (c, c') in the table.
 __host__ __device__ constexpr int s_index(int c, int cp) { return c * (c + 1) / 2 + cp; }
 __host__ __device__ constexpr int m_index(int c, int cp) { return 10 + c * (c - 1) / 2 + cp; }
@@ -232,7 +250,8 @@ __global__ void __launch_bounds__(kThreads, 1) ttt_linear_wy_kernel(const __grid
 #pragma unroll
     for (int jj = 0; jj < 4; ++jj) {
       const int pi = 4 * warp + jj;
-      const int kind = kProd[pi][0], c = kProd[pi][1], cp = kProd[pi][2];
+      const int code = prod_of(pi);
+      const int kind = code >> 4, c = (code >> 2) & 3, cp = code & 3;
       float X[2][4] = {};
       const uint32_t abase = kind == 0 ? qa : ka;
 #pragma unroll
@@ -300,13 +319,15 @@ __global__ void __launch_bounds__(kThreads, 1) ttt_linear_wy_kernel(const __grid
 
     // 4) forward substitution: E_c -= sum over earlier sub-blocks of other chunks
     //    of (-N E_c')^T (K_c' K_c^T); As[c] = (-N_c E_c)^T as A fragments
-    auto chunk_of = [&](int c) { return (g0 + 16 * c) / p.chunk; };
+    int chunk_id[kSub];
+#pragma unroll
+    for (int c = 0; c < kSub; ++c) chunk_id[c] = (g0 + 16 * c) / p.chunk;
     uint32_t As[kSub][4], Ae[kSub][4];
 #pragma unroll
     for (int c = 0; c < kSub; ++c) {
 #pragma unroll
       for (int cp = 0; cp < c; ++cp) {
-        if (chunk_of(cp) == chunk_of(c)) continue;
+        if (chunk_id[cp] == chunk_id[c]) continue;
         const uint32_t* f = &sm.frag[fb][m_index(c, cp)][0][0][0];
         mma16816(E[c][0], As[cp], f[0 * 64 + 0 * 32 + lane], f[0 * 64 + 1 * 32 + lane]);
         mma16816(E[c][1], As[cp], f[1 * 64 + 0 * 32 + lane], f[1 * 64 + 1 * 32 + lane]);
