@@ -171,7 +171,11 @@ class Step:
         dt = d["q"].dtype
         self.out = torch.empty((w.B, w.H, w.T, w.dv), dtype=dt, device=d["q"].device)
         if w.variant == "lact":
-            self.launches = None
+            # prep rows kernel, then per chunk two GEMM launches and the rows
+            # kernel (+ Newton-Schulz for Muon, + two apply GEMMs when non-causal)
+            nch = -(-w.T // w.chunk) if w.T > 0 else 0
+            per = 3 + (1 if w.update_rule == synth.UPDATE_MUON else 0) + (0 if w.causal else 2)
+            self.launches = 1 + nch * per
         else:
             self.Wf = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=d["q"].device)
             self.launches = 1
@@ -217,6 +221,9 @@ KERNEL_SOURCES = {
                         "linear_attention_ttt_b200/csrc/tma.cuh"],
     "ttt_linear_f32": ["linear_attention_ttt_b200/csrc/ttt_linear_f32.cu",
                        "linear_attention_ttt_b200/csrc/common.cuh"],
+    "ttt_linear_wy": ["linear_attention_ttt_b200/csrc/ttt_linear_wy.cu",
+                      "linear_attention_ttt_b200/csrc/common.cuh",
+                      "linear_attention_ttt_b200/csrc/tma.cuh"],
 }
 
 
@@ -227,6 +234,9 @@ def kernel_key(w):
         return "ttt_linear_f32"
     if w.loss == synth.LOSS_NEG_DOT and w.dk == 128 and w.dv == 128:
         return "la_tc"
+    if (w.loss == synth.LOSS_MSE and w.dk == 64 and w.dv == 64
+            and (w.chunk in (16, 32) or w.chunk % 64 == 0)):
+        return "ttt_linear_wy"
     return "ttt_linear_bf16"
 
 

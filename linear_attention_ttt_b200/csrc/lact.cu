@@ -139,6 +139,7 @@ struct NsArgs {
   // xn [L*s], then kNsCluster partial squared norms
   float* scratch;
   int64_t scratch_stride;
+  int* status;  // device status word (bounded waits record a timeout here)
   float a, b, c, eps;
   int steps;
 };
@@ -335,106 +336,48 @@ __global__ void __cluster_dims__(kNsCluster, 1, 1) __launch_bounds__(kNsThreads)
   }
 }
 
+constexpr int kN5 = 128;          // slab side of the 128 x 512 Newton-Schulz kernel
+
 // ---------------------------------------------------------------------------
-// Newton-Schulz for 128 x 512 (or 512 x 128) gradients with every operand in
-// shared memory: a cluster of kNsCluster CTAs per matrix, CTA c owning the
-// 128 x 128 slab c of the long side. The slab X, the Gram matrix G and the
-// polynomial P live in shared memory as bf16 hi / lo pairs (x = hi + lo to
-// about 16 bits), so the split-bf16 products hi*hi + lo*hi + hi*lo read their
-// fragments straight from shared memory. Gram partials are summed across the
-// cluster through distributed shared memory: CTA c reduces rows [32c, 32c+32)
-// of G and writes them into every CTA's copy.
+// Newton-Schulz for 128 x 512 (or 512 x 128) gradients on the 5th-generation
+// tensor cores: a cluster of kNsCluster CTAs per matrix, CTA c owning the
+// 128 x 128 slab c of the long side; Gram partials are summed through
+// distributed shared memory (CTA c reduces rows [32c, 32c + 32) of G and writes
+// them into every CTA's copy). X, G and P stay in shared memory as bf16 hi / lo
+// (x = hi + lo to about 16 bits) in the 128-byte-swizzled layout of two
+// 64-column boxes [128 rows][128 B]; one storage serves as a K-major operand
+// (rows = M or N) and as an MN-major operand (rows = K). Each split product
+// hi*hi + lo*hi + hi*lo is 24 tcgen05.mma of 128 x 128 x 16 into one TMEM
+// accumulator, issued by one thread; 16 warps move accumulators out of TMEM.
 // ---------------------------------------------------------------------------
 
-constexpr int kN5 = 128;          // slab side
-constexpr int kN5Ld = kN5 + 8;    // padded row (bf16): conflict-free ldmatrix
-constexpr int kN5Threads = 512;   // 16 warps, warp tile 32 x 32
+constexpr int kT5Threads = 512;
+constexpr uint32_t kT5Box = 16384;  // one 64-column box of a 128 x 128 bf16 matrix
 
-struct Ns128Smem {
-  __nv_bfloat16 x[2][kN5 * kN5Ld];  // hi, lo
-  __nv_bfloat16 g[2][kN5 * kN5Ld];
-  __nv_bfloat16 p[2][kN5 * kN5Ld];  // also holds the fp32 Gram partial [128][128]
+struct Ns5Smem {
+  alignas(1024) uint8_t x[2][2 * kT5Box];  // [hi|lo]
+  alignas(1024) uint8_t g[2][2 * kT5Box];
+  alignas(1024) uint8_t p[2][2 * kT5Box];  // also the fp32 Gram partial [128][128]
+  uint64_t mma_done;
+  uint32_t tmem_base;
   float nrm;
 };
 
-__device__ __forceinline__ void split_store(__nv_bfloat16* hi, __nv_bfloat16* lo, int idx, float v) {
-  const __nv_bfloat16 h = __float2bfloat16_rn(v);
-  hi[idx] = h;
-  lo[idx] = __float2bfloat16_rn(v - __bfloat162float(h));
+// byte offset of bf16 element (r, c) of a 128 x 128 matrix in the box layout
+__device__ __forceinline__ uint32_t t5_off(int r, int c) {
+  return (uint32_t)((c >> 6) * kT5Box + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4) +
+                    ((c & 7) << 1));
+}
+// byte offset of 16-byte fp32 chunk j (columns 4j .. 4j+3) of row r of the partial
+__device__ __forceinline__ uint32_t t5_part(int r, int j) {
+  return (uint32_t)(r * 512 + ((j ^ (r & 7)) << 4));
 }
 
-// acc (warp tile rows 32wm + 16mt + {g, g+8}, columns 32wn + 8nt + 2c4 + {0,1})
-// = op(A) op(B) over k = 0..127 with split-bf16 products. TA: A is stored
-// [k][m] (A = S^T); TB: B is stored [k][n] (row-major); otherwise A is [m][k]
-// and B is stored [n][k].
-template <bool TA, bool TB>
-__device__ __forceinline__ void ns128_gemm(const __nv_bfloat16* const (&A)[2],
-                                           const __nv_bfloat16* const (&B)[2],
-                                           float (&acc)[2][4][4]) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int wm = warp >> 2, wn = warp & 3, mi = lane >> 3, rr = lane & 7;
-#pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-      for (int q = 0; q < 4; ++q) acc[mt][nt][q] = 0.f;
-#pragma unroll 2
-  for (int k0 = 0; k0 < kN5; k0 += 16) {
-    uint32_t af[2][2][4], bf[2][4][2];  // [hi|lo][m-tile][4], [hi|lo][n-tile][2]
-#pragma unroll
-    for (int x = 0; x < 2; ++x) {
-#pragma unroll
-      for (int mt = 0; mt < 2; ++mt) {
-        const int m0 = 32 * wm + 16 * mt;
-        if (TA)
-          ns_ldsm_x4_t(af[x][mt], A[x] + (k0 + rr + 8 * (mi >> 1)) * kN5Ld + m0 + 8 * (mi & 1));
-        else
-          ns_ldsm_x4(af[x][mt], A[x] + (m0 + rr + 8 * (mi & 1)) * kN5Ld + k0 + 8 * (mi >> 1));
-      }
-#pragma unroll
-      for (int np = 0; np < 2; ++np) {  // pairs of n-tiles
-        const int n0 = 32 * wn + 16 * np;
-        uint32_t r[4];
-        if (TB)
-          ns_ldsm_x4_t(r, B[x] + (k0 + rr + 8 * (mi & 1)) * kN5Ld + n0 + 8 * (mi >> 1));
-        else
-          ns_ldsm_x4(r, B[x] + (n0 + rr + 8 * (mi >> 1)) * kN5Ld + k0 + 8 * (mi & 1));
-        bf[x][2 * np][0] = r[0];
-        bf[x][2 * np][1] = r[1];
-        bf[x][2 * np + 1][0] = r[2];
-        bf[x][2 * np + 1][1] = r[3];
-      }
-    }
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int nt = 0; nt < 4; ++nt) {
-        ns_mma(acc[mt][nt], af[0][mt], bf[0][nt][0], bf[0][nt][1]);  // hi * hi
-        ns_mma(acc[mt][nt], af[1][mt], bf[0][nt][0], bf[0][nt][1]);  // lo * hi
-        ns_mma(acc[mt][nt], af[0][mt], bf[1][nt][0], bf[1][nt][1]);  // hi * lo
-      }
-  }
-}
-
-// Visits the warp's accumulator elements: f(row, col, value).
-template <class F>
-__device__ __forceinline__ void ns128_each(const float (&acc)[2][4][4], F&& f) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int wm = warp >> 2, wn = warp & 3, g = lane >> 2, c4 = lane & 3;
-#pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        f(32 * wm + 16 * mt + g + 8 * (q >> 1), 32 * wn + 8 * nt + 2 * c4 + (q & 1), acc[mt][nt][q]);
-}
-
-__global__ void __cluster_dims__(kNsCluster, 1, 1) __launch_bounds__(kN5Threads, 1)
-    ns128_kernel(NsArgs a) {
-  extern __shared__ __align__(16) uint8_t ns_smem_raw[];
-  Ns128Smem& sm = *reinterpret_cast<Ns128Smem*>(ns_smem_raw);
+__global__ void __cluster_dims__(kNsCluster, 1, 1) __launch_bounds__(kT5Threads, 1)
+    ns5_kernel(NsArgs a) {
+  extern __shared__ __align__(1024) uint8_t ns5_raw[];
+  Ns5Smem& sm = *reinterpret_cast<Ns5Smem*>((reinterpret_cast<uintptr_t>(ns5_raw) + 1023) &
+                                            ~uintptr_t(1023));
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
   const int mat = blockIdx.x / kNsCluster, c = (int)cluster.block_rank();
@@ -442,11 +385,21 @@ __global__ void __cluster_dims__(kNsCluster, 1, 1) __launch_bounds__(kN5Threads,
   const int R = a.rows[m], C = a.cols[m];
   const bool tall = R >= C;
   float* Xc = a.G[m] + (int64_t)z * R * C + (tall ? (int64_t)c * kN5 * C : (int64_t)c * kN5);
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  // Frobenius norm of the whole matrix (four slabs)
+  if (tid == 0) {
+    mbar_init(&sm.mma_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) umma::tmem_alloc(&sm.tmem_base, 128);
+  umma::fence_before();
+  __syncthreads();
+  umma::fence_after();
+  const uint32_t tmem = sm.tmem_base;
+
+  // Frobenius norm of the whole matrix (four slabs), then the scaled slab as hi / lo
   float ss = 0.f;
-  for (int e = tid; e < kN5 * kN5; e += kN5Threads) {
+  for (int e = tid; e < kN5 * kN5; e += kT5Threads) {
     const float v = Xc[(int64_t)(e >> 7) * C + (e & 127)];
     ss += v * v;
   }
@@ -456,63 +409,170 @@ __global__ void __cluster_dims__(kNsCluster, 1, 1) __launch_bounds__(kN5Threads,
   float tot = 0.f;
   for (int r = 0; r < kNsCluster; ++r) tot += *cluster.map_shared_rank(&sm.nrm, r);
   const float inv = 1.f / (sqrtf(tot) + a.eps);
-  for (int e = tid; e < kN5 * kN5; e += kN5Threads) {
-    const int i = e >> 7, j = e & 127;
-    split_store(sm.x[0], sm.x[1], i * kN5Ld + j, Xc[(int64_t)i * C + j] * inv);
+  for (int e = tid; e < kN5 * kN5 / 8; e += kT5Threads) {  // 8 columns per step
+    const int r = e >> 4, c0 = (e & 15) * 8;
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float v0 = Xc[(int64_t)r * C + c0 + 2 * u] * inv;
+      const float v1 = Xc[(int64_t)r * C + c0 + 2 * u + 1] * inv;
+      const __nv_bfloat16 h0 = __float2bfloat16_rn(v0), h1 = __float2bfloat16_rn(v1);
+      hi[u] = gemm::pack_bf16x2(__bfloat162float(h0), __bfloat162float(h1));
+      lo[u] = gemm::pack_bf16x2(v0 - __bfloat162float(h0), v1 - __bfloat162float(h1));
+    }
+    *reinterpret_cast<uint4*>(sm.x[0] + t5_off(r, c0)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(sm.x[1] + t5_off(r, c0)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
   }
+  umma::fence_proxy_async_smem();
   __syncthreads();
 
-  const __nv_bfloat16* const X2[2] = {sm.x[0], sm.x[1]};
-  const __nv_bfloat16* const G2[2] = {sm.g[0], sm.g[1]};
-  const __nv_bfloat16* const P2[2] = {sm.p[0], sm.p[1]};
-  float* part = reinterpret_cast<float*>(sm.p[0]);  // [128][128] fp32, spans p[0] and p[1]
-  float acc[2][4][4];
+  // One split product into the accumulator: A, B given as [hi, lo] storages and
+  // whether each is read MN-major (rows = K) or K-major (rows = M or N).
+  int phase = 0;
+  auto product = [&](uint8_t* const (&A)[2], bool a_mn, uint8_t* const (&B)[2], bool b_mn) {
+    if (tid == 0) {
+      umma::fence_after();
+      const uint32_t idesc = umma::instr_desc(1, kN5, kN5, a_mn, b_mn);
+      const int pa[3] = {0, 1, 0}, pb[3] = {0, 0, 1};
+      for (int pr = 0; pr < 3; ++pr) {
+        const uint32_t sa = smem_u32(A[pa[pr]]), sb = smem_u32(B[pb[pr]]);
+#pragma unroll
+        for (int kk = 0; kk < kN5 / 16; ++kk) {
+          const uint64_t ad = a_mn ? umma::smem_desc(sa + kk * 2048, kT5Box, 1024)
+                                   : umma::smem_desc(sa + (kk >> 2) * kT5Box + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = b_mn ? umma::smem_desc(sb + kk * 2048, kT5Box, 1024)
+                                   : umma::smem_desc(sb + (kk >> 2) * kT5Box + (kk & 3) * 32, 16, 1024);
+          umma::mma_bf16(tmem, ad, bd, idesc, (pr > 0 || kk > 0) ? 1u : 0u);
+        }
+      }
+      umma::commit(&sm.mma_done);
+    }
+    const bool ok = mbar_wait(&sm.mma_done, phase, a.status);
+    phase ^= 1;
+    umma::fence_after();
+    return ok;
+  };
+  // This thread's 32 accumulator values: row 32 (warp & 3) + lane, columns 32 (warp >> 2) ..
+  const int er = 32 * (warp & 3) + lane, ec = 32 * (warp >> 2);
+  const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + ec;
+  auto acc_load = [&](float (&v)[32]) {
+    uint32_t r0[16], r1[16];
+    umma::tmem_ld16_async(tl, r0);
+    umma::tmem_ld16_async(tl + 16, r1);
+    umma::tmem_wait_ld(r0);
+    umma::tmem_wait_ld(r1);
+#pragma unroll
+    for (int u = 0; u < 16; ++u) v[u] = __uint_as_float(r0[u]), v[16 + u] = __uint_as_float(r1[u]);
+  };
+  // value (hi + lo) of bf16 storage element (r, c)
+  auto val = [&](uint8_t* const (&S)[2], int r, int cc) {
+    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(S[0] + t5_off(r, cc))) +
+           __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(S[1] + t5_off(r, cc)));
+  };
+  // store 32 values of row r, columns cc .. cc+31, as hi / lo
+  auto put32 = [&](uint8_t* const (&S)[2], int r, int cc, const float (&v)[32]) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t hi[4], lo[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float v0 = v[8 * q + 2 * u], v1 = v[8 * q + 2 * u + 1];
+        const __nv_bfloat16 h0 = __float2bfloat16_rn(v0), h1 = __float2bfloat16_rn(v1);
+        hi[u] = gemm::pack_bf16x2(__bfloat162float(h0), __bfloat162float(h1));
+        lo[u] = gemm::pack_bf16x2(v0 - __bfloat162float(h0), v1 - __bfloat162float(h1));
+      }
+      *reinterpret_cast<uint4*>(S[0] + t5_off(r, cc + 8 * q)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      *reinterpret_cast<uint4*>(S[1] + t5_off(r, cc + 8 * q)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    }
+  };
+
+  uint8_t* const X2[2] = {sm.x[0], sm.x[1]};
+  uint8_t* const G2[2] = {sm.g[0], sm.g[1]};
+  uint8_t* const P2[2] = {sm.p[0], sm.p[1]};
+  uint8_t* const part = sm.p[0];  // 64 KB: p[0] and p[1] are contiguous
+  bool ok = true;
   for (int it = 0; it < a.steps; ++it) {
-    // Gram partial of this slab: tall X^T X, wide X X^T
-    if (tall)
-      ns128_gemm<true, true>(X2, X2, acc);
-    else
-      ns128_gemm<false, false>(X2, X2, acc);
-    ns128_each(acc, [&](int i, int j, float v) { part[i * kN5 + j] = v; });
+    // Gram partial: tall X^T X (both operands MN-major), wide X X^T (both K-major)
+    ok = product(X2, tall, X2, tall) && ok;
+    {
+      float v[32];
+      acc_load(v);
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        *reinterpret_cast<float4*>(part + t5_part(er, ec / 4 + q)) =
+            make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    }
+    umma::fence_before();
     cluster.sync();
-    // rows [32c, 32c + 32) of G = sum of the four partials, into every CTA's G
-    for (int e = tid; e < 32 * kN5; e += kN5Threads) {
-      const int i = 32 * c + (e >> 7), j = e & 127;
-      float gsum = 0.f;
-      for (int r = 0; r < kNsCluster; ++r) gsum += cluster.map_shared_rank(part, r)[i * kN5 + j];
-      const __nv_bfloat16 h = __float2bfloat16_rn(gsum);
-      const __nv_bfloat16 l = __float2bfloat16_rn(gsum - __bfloat162float(h));
-      for (int r = 0; r < kNsCluster; ++r) {
-        cluster.map_shared_rank(sm.g[0], r)[i * kN5Ld + j] = h;
-        cluster.map_shared_rank(sm.g[1], r)[i * kN5Ld + j] = l;
+    // rows [32c, 32c + 32) of G: sum of the four partials, into every CTA's G
+    {
+      const int r = 32 * c + (tid >> 4), c0 = (tid & 15) * 8;
+      float gsum[8] = {};
+      for (int rk = 0; rk < kNsCluster; ++rk) {
+        const uint8_t* rp = cluster.map_shared_rank(part, rk);
+        const float4 u0 = *reinterpret_cast<const float4*>(rp + t5_part(r, c0 / 4));
+        const float4 u1 = *reinterpret_cast<const float4*>(rp + t5_part(r, c0 / 4 + 1));
+        gsum[0] += u0.x, gsum[1] += u0.y, gsum[2] += u0.z, gsum[3] += u0.w;
+        gsum[4] += u1.x, gsum[5] += u1.y, gsum[6] += u1.z, gsum[7] += u1.w;
+      }
+      uint32_t hi[4], lo[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float v0 = gsum[2 * u], v1 = gsum[2 * u + 1];
+        const __nv_bfloat16 h0 = __float2bfloat16_rn(v0), h1 = __float2bfloat16_rn(v1);
+        hi[u] = gemm::pack_bf16x2(__bfloat162float(h0), __bfloat162float(h1));
+        lo[u] = gemm::pack_bf16x2(v0 - __bfloat162float(h0), v1 - __bfloat162float(h1));
+      }
+      for (int rk = 0; rk < kNsCluster; ++rk) {
+        *reinterpret_cast<uint4*>(cluster.map_shared_rank(sm.g[0], rk) + t5_off(r, c0)) =
+            make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(cluster.map_shared_rank(sm.g[1], rk) + t5_off(r, c0)) =
+            make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
     }
     cluster.sync();
-    // P = c G^2 + b G
-    ns128_gemm<false, true>(G2, G2, acc);
-    ns128_each(acc, [&](int i, int j, float v) {
-      const float gij = __bfloat162float(sm.g[0][i * kN5Ld + j]) + __bfloat162float(sm.g[1][i * kN5Ld + j]);
-      split_store(sm.p[0], sm.p[1], i * kN5Ld + j, a.c * v + a.b * gij);
-    });
+    umma::fence_proxy_async_smem();
     __syncthreads();
-    // X <- a X + X P (tall) or a X + P X (wide)
+    // P = c G^2 + b G   (A = G K-major, B = G MN-major)
+    ok = product(G2, false, G2, true) && ok;
+    {
+      float v[32];
+      acc_load(v);
+#pragma unroll
+      for (int u = 0; u < 32; ++u) v[u] = a.c * v[u] + a.b * val(G2, er, ec + u);
+      put32(P2, er, ec, v);
+    }
+    umma::fence_before();
+    umma::fence_proxy_async_smem();
+    __syncthreads();
+    // X <- a X + X P (tall) or a X + P X (wide)   (B MN-major)
     if (tall)
-      ns128_gemm<false, true>(X2, P2, acc);
+      ok = product(X2, false, P2, true) && ok;
     else
-      ns128_gemm<false, true>(P2, X2, acc);
-    __syncthreads();  // every warp is done reading X
-    const bool last = it + 1 == a.steps;
-    ns128_each(acc, [&](int i, int j, float v) {
-      const float xij = __bfloat162float(sm.x[0][i * kN5Ld + j]) + __bfloat162float(sm.x[1][i * kN5Ld + j]);
-      const float xn = a.a * xij + v;
-      if (last)
-        Xc[(int64_t)i * C + j] = xn;
-      else
-        split_store(sm.x[0], sm.x[1], i * kN5Ld + j, xn);
-    });
+      ok = product(P2, false, X2, true) && ok;
+    {
+      float v[32];
+      acc_load(v);
+#pragma unroll
+      for (int u = 0; u < 32; ++u) v[u] += a.a * val(X2, er, ec + u);
+      if (it + 1 == a.steps) {
+#pragma unroll
+        for (int u = 0; u < 32; ++u) Xc[(int64_t)er * C + ec + u] = v[u];
+      } else {
+        umma::fence_before();
+        __syncthreads();  // every thread has read its old X values
+        put32(X2, er, ec, v);
+      }
+    }
+    umma::fence_before();
+    umma::fence_proxy_async_smem();
     __syncthreads();
+    // A timed-out wait is recorded in the status word; the loop still runs to
+    // its end so that every CTA of the cluster meets the same cluster barriers.
   }
+  (void)ok;
   cluster.sync();  // no CTA leaves while another may still read its shared memory
+  if (warp == 0) umma::tmem_dealloc(tmem, 128);
 }
 
 __global__ void copy_kernel(float* dst, const float* src, int64_t n) {
@@ -826,6 +886,7 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
     na.rows[2] = dv;
     na.cols[2] = dh;
     na.scratch = sc.ns;
+    na.status = a.status;
     na.scratch_stride = ns_stride;
     na.a = 3.4445f;
     na.b = -4.7750f;
@@ -835,10 +896,10 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
   }
 
   // Gradients of 512 x 128 / 128 x 512 run the shared-memory-resident kernel.
-  const bool ns128 = split && dk == kN5 && dv == kN5 && dh == kNsCluster * kN5;
-  if (ns128)
-    check(cudaFuncSetAttribute(ns128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)sizeof(Ns128Smem)));
+  const bool ns_tc = split && dk == kN5 && dv == kN5 && dh == kNsCluster * kN5;
+  if (ns_tc)
+    check(cudaFuncSetAttribute(ns5_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)(sizeof(Ns5Smem) + 1024)));
   const int* segW = split ? &kSegBsplit[0][0] : &kSegExact[0][0];
   const int nsegW = split ? 2 : 1;
 
@@ -1013,8 +1074,8 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
     }
     // L3 / L4: Muon orthogonalisation, update and row renormalisation
     if (split) {
-      if (ns128) {
-        ns128_kernel<<<Z * 3 * kNsCluster, kN5Threads, sizeof(Ns128Smem), s>>>(na);
+      if (ns_tc) {
+        ns5_kernel<<<Z * 3 * kNsCluster, kT5Threads, sizeof(Ns5Smem) + 1024, s>>>(na);
       } else {
         ns_kernel<<<Z * 3 * kNsCluster, kNsThreads, 0, s>>>(na);
       }
