@@ -55,7 +55,7 @@ def peaks():
 
 
 # ---------------------------------------------------------------------------
-# Workload accounting (algorithmic bytes / flops per step, per DESIGN.md)
+# Workload accounting (algorithmic bytes / flops per step)
 # ---------------------------------------------------------------------------
 
 def linear_bytes(w):
@@ -240,10 +240,11 @@ def kernel_key(w):
     return "ttt_linear_bf16"
 
 
-def rank_workload(index, rank, chunk=None):
+def rank_workload(index, rank, chunk=None, seq_len=None):
     """Each rank runs its own replica: the same workload shape with an
-    independent draw of the inputs (weak scaling, no data-path collective)."""
-    return synth.config(index, chunk=chunk, replica=rank)
+    independent draw of the inputs (weak scaling, no data-path collective).
+    seq_len shortens the sequence (same distributions), e.g. for profiling."""
+    return synth.config(index, chunk=chunk, T=seq_len, replica=rank)
 
 
 def max_over_ranks(value, dist=None, device=None):
@@ -302,6 +303,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", type=int, default=2)
     ap.add_argument("--chunk", type=int, default=None)
+    ap.add_argument("--seq-len", type=int, default=None,
+                    help="shorter sequence of the same workload (profiling); the default "
+                         "line uses the workload's own length")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -310,7 +314,7 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
 
-    w = rank_workload(args.workload, rank, chunk=args.chunk)
+    w = rank_workload(args.workload, rank, chunk=args.chunk, seq_len=args.seq_len)
     tokens_per_step = w.B * w.T
     base_cfg = {"workload": w.name, "batch": w.B, "heads": w.H, "seq_len": w.T, "dk": w.dk,
                 "dv": w.dv, "chunk": w.chunk, "variant": w.variant,

@@ -76,7 +76,7 @@ typedef enum {
   TTT_ERR_SHAPE = -2,       /* sizes inconsistent across tensors, or ndim wrong */
   TTT_ERR_DTYPE = -3,       /* element type not allowed for this tensor */
   TTT_ERR_LAYOUT = -4,      /* stride or 16-byte alignment rule broken */
-  TTT_ERR_UNSUPPORTED = -5, /* valid request this build has no kernel for */
+  TTT_ERR_UNSUPPORTED = -5, /* valid request the library has no kernel for */
   TTT_ERR_CUDA = -6,        /* a CUDA runtime call failed (launch, memory) */
   TTT_ERR_TIMEOUT = -7,     /* a device-side bounded wait gave up */
   TTT_ERR_ALLOC = -8,       /* stream-ordered scratch allocation failed */
@@ -116,7 +116,8 @@ ttt_status ttt_linear_fwd(const ttt_tensor* q, const ttt_tensor* k, const ttt_te
 
 /*
  * LaCT SwiGLU layer forward.
- *  q, k [B,H,T,dk] bf16 or fp32; v, out [B,H,T,dv] (dk == dv for bf16)
+ *  q, k [B,H,T,dk], v, out [B,H,T,dv], bf16 with dk == dv (fp32 tokens
+ *       return TTT_ERR_UNSUPPORTED)
  *  eta  [B,H,T] fp32
  *  W1, W3 [H,dh,dk] or [B,H,dh,dk]; W2 [H,dv,dh] or [B,H,dv,dh]; fp32,
  *         contiguous, read-only (the scan works on private copies)

@@ -123,7 +123,7 @@ const char* ttt_status_string(int32_t s) {
     case TTT_ERR_SHAPE: return "tensor shapes are inconsistent or have the wrong rank";
     case TTT_ERR_DTYPE: return "element type not allowed for this tensor";
     case TTT_ERR_LAYOUT: return "stride or 16-byte alignment rule broken";
-    case TTT_ERR_UNSUPPORTED: return "no kernel in this build for these sizes/types";
+    case TTT_ERR_UNSUPPORTED: return "no kernel in this library for these sizes/types";
     case TTT_ERR_CUDA: return "a CUDA runtime call failed";
     case TTT_ERR_TIMEOUT: return "a device-side bounded wait gave up";
     case TTT_ERR_ALLOC: return "stream-ordered scratch allocation failed";

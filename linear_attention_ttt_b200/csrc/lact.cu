@@ -398,10 +398,18 @@ __global__ void __cluster_dims__(kNsCluster, 1, 1) __launch_bounds__(kT5Threads,
   const uint32_t tmem = sm.tmem_base;
 
   // Frobenius norm of the whole matrix (four slabs), then the scaled slab as hi / lo
+  // the slab as 8-column pieces (two float4 each), 4 per thread, kept in registers
+  float4 xs[4][2];
   float ss = 0.f;
-  for (int e = tid; e < kN5 * kN5; e += kT5Threads) {
-    const float v = Xc[(int64_t)(e >> 7) * C + (e & 127)];
-    ss += v * v;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int e = tid + i * kT5Threads, r = e >> 4, c0 = (e & 15) * 8;
+    const float4* src = reinterpret_cast<const float4*>(Xc + (int64_t)r * C + c0);
+    xs[i][0] = src[0];
+    xs[i][1] = src[1];
+    ss += xs[i][0].x * xs[i][0].x + xs[i][0].y * xs[i][0].y + xs[i][0].z * xs[i][0].z +
+          xs[i][0].w * xs[i][0].w + xs[i][1].x * xs[i][1].x + xs[i][1].y * xs[i][1].y +
+          xs[i][1].z * xs[i][1].z + xs[i][1].w * xs[i][1].w;
   }
   ss = block_sum(ss);
   if (tid == 0) sm.nrm = ss;
@@ -409,13 +417,16 @@ __global__ void __cluster_dims__(kNsCluster, 1, 1) __launch_bounds__(kT5Threads,
   float tot = 0.f;
   for (int r = 0; r < kNsCluster; ++r) tot += *cluster.map_shared_rank(&sm.nrm, r);
   const float inv = 1.f / (sqrtf(tot) + a.eps);
-  for (int e = tid; e < kN5 * kN5 / 8; e += kT5Threads) {  // 8 columns per step
-    const int r = e >> 4, c0 = (e & 15) * 8;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int e = tid + i * kT5Threads, r = e >> 4, c0 = (e & 15) * 8;
+    const float xv[8] = {xs[i][0].x, xs[i][0].y, xs[i][0].z, xs[i][0].w,
+                         xs[i][1].x, xs[i][1].y, xs[i][1].z, xs[i][1].w};
     uint32_t hi[4], lo[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const float v0 = Xc[(int64_t)r * C + c0 + 2 * u] * inv;
-      const float v1 = Xc[(int64_t)r * C + c0 + 2 * u + 1] * inv;
+      const float v0 = xv[2 * u] * inv;
+      const float v1 = xv[2 * u + 1] * inv;
       const __nv_bfloat16 h0 = __float2bfloat16_rn(v0), h1 = __float2bfloat16_rn(v1);
       hi[u] = gemm::pack_bf16x2(__bfloat162float(h0), __bfloat162float(h1));
       lo[u] = gemm::pack_bf16x2(v0 - __bfloat162float(h0), v1 - __bfloat162float(h1));
@@ -464,10 +475,21 @@ __global__ void __cluster_dims__(kNsCluster, 1, 1) __launch_bounds__(kT5Threads,
 #pragma unroll
     for (int u = 0; u < 16; ++u) v[u] = __uint_as_float(r0[u]), v[16 + u] = __uint_as_float(r1[u]);
   };
-  // value (hi + lo) of bf16 storage element (r, c)
-  auto val = [&](uint8_t* const (&S)[2], int r, int cc) {
-    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(S[0] + t5_off(r, cc))) +
-           __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(S[1] + t5_off(r, cc)));
+  // values (hi + lo) of bf16 storage elements (r, cc .. cc+31), 16-byte reads
+  auto val32 = [&](uint8_t* const (&S)[2], int r, int cc, float (&o)[32]) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 h = *reinterpret_cast<const uint4*>(S[0] + t5_off(r, cc + 8 * q));
+      const uint4 l = *reinterpret_cast<const uint4*>(S[1] + t5_off(r, cc + 8 * q));
+      const uint32_t hw[4] = {h.x, h.y, h.z, h.w}, lw[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const __nv_bfloat162 hb = *reinterpret_cast<const __nv_bfloat162*>(&hw[u]);
+        const __nv_bfloat162 lb = *reinterpret_cast<const __nv_bfloat162*>(&lw[u]);
+        o[8 * q + 2 * u] = __low2float(hb) + __low2float(lb);
+        o[8 * q + 2 * u + 1] = __high2float(hb) + __high2float(lb);
+      }
+    }
   };
   // store 32 values of row r, columns cc .. cc+31, as hi / lo
   auto put32 = [&](uint8_t* const (&S)[2], int r, int cc, const float (&v)[32]) {
@@ -536,10 +558,11 @@ __global__ void __cluster_dims__(kNsCluster, 1, 1) __launch_bounds__(kT5Threads,
     // P = c G^2 + b G   (A = G K-major, B = G MN-major)
     ok = product(G2, false, G2, true) && ok;
     {
-      float v[32];
+      float v[32], gv[32];
       acc_load(v);
+      val32(G2, er, ec, gv);
 #pragma unroll
-      for (int u = 0; u < 32; ++u) v[u] = a.c * v[u] + a.b * val(G2, er, ec + u);
+      for (int u = 0; u < 32; ++u) v[u] = a.c * v[u] + a.b * gv[u];
       put32(P2, er, ec, v);
     }
     umma::fence_before();
@@ -551,13 +574,16 @@ __global__ void __cluster_dims__(kNsCluster, 1, 1) __launch_bounds__(kT5Threads,
     else
       ok = product(P2, false, X2, true) && ok;
     {
-      float v[32];
+      float v[32], xv[32];
       acc_load(v);
+      val32(X2, er, ec, xv);
 #pragma unroll
-      for (int u = 0; u < 32; ++u) v[u] += a.a * val(X2, er, ec + u);
+      for (int u = 0; u < 32; ++u) v[u] += a.a * xv[u];
       if (it + 1 == a.steps) {
+        float4* dst = reinterpret_cast<float4*>(Xc + (int64_t)er * C + ec);
 #pragma unroll
-        for (int u = 0; u < 32; ++u) Xc[(int64_t)er * C + ec + u] = v[u];
+        for (int q = 0; q < 8; ++q)
+          dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
       } else {
         umma::fence_before();
         __syncthreads();  // every thread has read its old X values

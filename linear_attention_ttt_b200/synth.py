@@ -181,6 +181,7 @@ def config(index: int, chunk: Optional[int] = None, T: Optional[int] = None,
         w = make_lact(B or 1, H or 8, T or 131072, 128, 512, chunk or 4096, UPDATE_MUON, seed)
     else:
         raise ValueError(f"no workload {index}")
-    w.name = CONFIG_NAMES[index] + ("" if chunk is None else f"_chunk{chunk}")
+    w.name = (CONFIG_NAMES[index] + ("" if chunk is None else f"_chunk{chunk}") +
+              ("" if T is None else f"_T{T}"))
     w.meta["config"] = index
     return w
