@@ -122,8 +122,10 @@ ttt_status ttt_linear_fwd(const ttt_tensor* q, const ttt_tensor* k, const ttt_te
  *  W1, W3 [H,dh,dk] or [B,H,dh,dk]; W2 [H,dv,dh] or [B,H,dv,dh]; fp32,
  *         contiguous, read-only (the scan works on private copies)
  *  chunk  >= 1; update_rule LACT_UPDATE_GD or LACT_UPDATE_MUON; causal 0/1
- * Scratch is taken stream-ordered from the device's default memory pool
- * (cudaMallocAsync / cudaFreeAsync on `stream`); failure -> TTT_ERR_ALLOC.
+ * Scratch is taken stream-ordered (cudaMallocFromPoolAsync / cudaFreeAsync on
+ * `stream`) from a memory pool the library creates per device and keeps for
+ * the process lifetime, so repeated calls reuse the same mapped memory; the
+ * device's default pool is not touched. Failure -> TTT_ERR_ALLOC.
  */
 ttt_status lact_swiglu_fwd(const ttt_tensor* q, const ttt_tensor* k, const ttt_tensor* v,
                            const ttt_tensor* eta, const ttt_tensor* W1, const ttt_tensor* W2,

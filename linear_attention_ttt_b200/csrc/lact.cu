@@ -23,6 +23,9 @@
 // split-bf16 operands (x = hi + lo, products hi*hi + lo*hi + hi*lo) because
 // the unit-step Muon scan amplifies per-chunk rounding across chunks.
 #include <cooperative_groups.h>
+
+#include <cstdint>
+#include <mutex>
 #include <vector>
 
 #include "gemm_tc.cuh"
@@ -73,33 +76,12 @@ __global__ void __launch_bounds__(256) lact_rows_kernel(RowArgs a) {
   const int nrows = (m == 2) ? a.dv : a.dh;
   float* W = a.Wm[m] + ((int64_t)z * nrows + r) * len;
   float* G = a.G[m] + ((int64_t)z * nrows + r) * len;
-  float v[32];
-  float ss = 0.f;
-  const int per = len / 32;  // len is a multiple of 32
+  const float* src = nullptr;
   if (a.prep) {
     const int zin = a.win_sz[m] ? z : z % a.H;
-    const float* src = a.Win[m] + ((int64_t)zin * nrows + r) * len;
-    for (int i = 0; i < per; ++i) {
-      v[i] = src[lane + 32 * i];
-      ss += v[i] * v[i];
-    }
-  } else {
-    for (int i = 0; i < per; ++i) {
-      v[i] = W[lane + 32 * i] - G[lane + 32 * i];
-      ss += v[i] * v[i];
-    }
+    src = a.Win[m] + ((int64_t)zin * nrows + r) * len;
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  const float nrm = sqrtf(ss);
   float* rho = a.rho[m] + (int64_t)z * nrows + r;
-  if (a.prep) {
-    if (lane == 0) *rho = nrm;
-  } else {
-    const float target = *rho;
-    const float s = nrm > 0.f ? target / nrm : 1.f;
-    for (int i = 0; i < per; ++i) v[i] *= s;
-  }
   __nv_bfloat16 *hi, *lo;
   int64_t orow;
   if (m == 2) {
@@ -112,13 +94,86 @@ __global__ void __launch_bounds__(256) lact_rows_kernel(RowArgs a) {
     orow = (int64_t)z * 2 * a.dh + (r / gemm::kHid) * 2 * gemm::kHid + (m == 1 ? gemm::kHid : 0) +
            (r % gemm::kHid);
   }
+  hi += orow * len;
+  if (a.split) lo += orow * len;
+
+  // new row = (W - G) (or the input row), then rescaled to its initial norm
+  auto finish = [&](float ss, float& s) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float nrm = sqrtf(ss);
+    if (a.prep) {
+      if (lane == 0) *rho = nrm;
+      s = 1.f;
+    } else {
+      const float target = *rho;
+      s = nrm > 0.f ? target / nrm : 1.f;
+    }
+  };
+  if (len % 128 == 0) {
+    // 4 consecutive columns per lane: 16-byte loads and stores, all issued
+    // before the row reduction
+    constexpr int kMaxV = 8;  // len <= 1024
+    const int per = len / 128;
+    float4 v[kMaxV];
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < kMaxV; ++i) {
+      if (i >= per) break;
+      const int c = 4 * (lane + 32 * i);
+      if (a.prep) {
+        v[i] = *reinterpret_cast<const float4*>(src + c);
+      } else {
+        const float4 w = *reinterpret_cast<const float4*>(W + c);
+        const float4 g = *reinterpret_cast<const float4*>(G + c);
+        v[i] = make_float4(w.x - g.x, w.y - g.y, w.z - g.z, w.w - g.w);
+      }
+      ss += v[i].x * v[i].x + v[i].y * v[i].y + v[i].z * v[i].z + v[i].w * v[i].w;
+    }
+    float s;
+    finish(ss, s);
+#pragma unroll
+    for (int i = 0; i < kMaxV; ++i) {
+      if (i >= per) break;
+      const int c = 4 * (lane + 32 * i);
+      const float4 x = make_float4(v[i].x * s, v[i].y * s, v[i].z * s, v[i].w * s);
+      *reinterpret_cast<float4*>(W + c) = x;
+      *reinterpret_cast<float4*>(G + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+      const __nv_bfloat16 h0 = __float2bfloat16_rn(x.x), h1 = __float2bfloat16_rn(x.y);
+      const __nv_bfloat16 h2 = __float2bfloat16_rn(x.z), h3 = __float2bfloat16_rn(x.w);
+      __nv_bfloat162 p0, p1;
+      p0.x = h0, p0.y = h1, p1.x = h2, p1.y = h3;
+      *reinterpret_cast<uint2*>(hi + c) =
+          make_uint2(*reinterpret_cast<uint32_t*>(&p0), *reinterpret_cast<uint32_t*>(&p1));
+      if (a.split) {
+        __nv_bfloat162 q0 = __floats2bfloat162_rn(x.x - __bfloat162float(h0), x.y - __bfloat162float(h1));
+        __nv_bfloat162 q1 = __floats2bfloat162_rn(x.z - __bfloat162float(h2), x.w - __bfloat162float(h3));
+        *reinterpret_cast<uint2*>(lo + c) =
+            make_uint2(*reinterpret_cast<uint32_t*>(&q0), *reinterpret_cast<uint32_t*>(&q1));
+      }
+    }
+    return;
+  }
+  // rows of 32 or 64 columns: one value per lane per step
+  float v[2];
+  float ss = 0.f;
+  const int per = len / 32;  // 1 or 2: the supported sizes give len 64 or a multiple of 128
+  if (per > 2) return;
   for (int i = 0; i < per; ++i) {
     const int c = lane + 32 * i;
-    W[c] = v[i];
+    v[i] = a.prep ? src[c] : W[c] - G[c];
+    ss += v[i] * v[i];
+  }
+  float s;
+  finish(ss, s);
+  for (int i = 0; i < per; ++i) {
+    const int c = lane + 32 * i;
+    const float x = v[i] * s;
+    W[c] = x;
     G[c] = 0.f;
-    const __nv_bfloat16 h = __float2bfloat16_rn(v[i]);
-    hi[orow * len + c] = h;
-    if (a.split) lo[orow * len + c] = __float2bfloat16_rn(v[i] - __bfloat162float(h));
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    hi[c] = h;
+    if (a.split) lo[c] = __float2bfloat16_rn(x - __bfloat162float(h));
   }
 }
 
@@ -770,6 +825,13 @@ int pick_ksplit(int kblocks, int tiles) {
 
 namespace {
 
+// Muon gradients of 128 x 512 / 512 x 128 run the tensor-core Newton-Schulz
+// kernel, which keeps every operand on chip and needs no scratch.
+bool ns_on_chip(const LactArgs& a) {
+  return a.update_rule == LACT_UPDATE_MUON && a.dk == kN5 && a.dv == kN5 &&
+         a.dh == kNsCluster * kN5;
+}
+
 struct Sizes {
   bool ok;
   int Z, chunk;
@@ -796,7 +858,9 @@ Sizes lact_sizes(const LactArgs& a) {
   z.ns_stride = 2 * kNsCluster * (int64_t)s_max * s_max +
                 kNsCluster * 2 * (int64_t)s_max * s_max + (int64_t)dh * dk + 64;
   for (int m = 0; m < 3; ++m) z.f32n += (size_t)z.Z * (2 * z.nW[m] + z.nrows[m]);
-  if (z.split) z.f32n += (size_t)z.Z * 3 * z.ns_stride;  // Newton-Schulz scratch
+  // Newton-Schulz scratch: only the general-shape kernel needs it (the
+  // tensor-core kernel for 128 x 512 gradients keeps everything on chip)
+  if (z.split && !ns_on_chip(a)) z.f32n += (size_t)z.Z * 3 * z.ns_stride;
   z.bfn = (size_t)z.Z * (2 * dh * dk + dv * dh) * (z.split ? 2 : 1);
   z.bfn += (size_t)z.Z * z.chunk * dh * 4 * (z.split ? 2 : 1);
   z.bytes = z.f32n * 4 + z.bfn * 2 + 4096;
@@ -810,11 +874,44 @@ size_t lact_scratch_bytes(const LactArgs& a) {
   return z.ok ? z.bytes : 0;
 }
 
+// The library's own stream-ordered memory pool on the current device. Its
+// release threshold keeps freed scratch mapped, so back-to-back calls reuse it
+// instead of mapping it again after every synchronisation (the device's
+// default pool, and with it the caller's, is left untouched).
+cudaMemPool_t scratch_pool() {
+  constexpr int kMaxDevices = 64;
+  static cudaMemPool_t pools[kMaxDevices] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!pools[dev]) {
+    cudaMemPoolProps props;
+    memset(&props, 0, sizeof(props));
+    props.allocType = cudaMemAllocationTypePinned;
+    props.handleTypes = cudaMemHandleTypeNone;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool = nullptr;
+    if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    uint64_t keep = UINT64_MAX;
+    cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    pools[dev] = pool;
+  }
+  return pools[dev];
+}
+
 ttt_status lact_forward(const LactArgs& a, cudaStream_t s) {
   const Sizes z = lact_sizes(a);
   if (!z.ok) return TTT_ERR_UNSUPPORTED;
   void* base = nullptr;
-  if (cudaMallocAsync(&base, z.bytes, s) != cudaSuccess) {
+  cudaMemPool_t pool = scratch_pool();
+  const cudaError_t ae = pool ? cudaMallocFromPoolAsync(&base, z.bytes, pool, s)
+                              : cudaMallocAsync(&base, z.bytes, s);
+  if (ae != cudaSuccess) {
     cudaGetLastError();
     return TTT_ERR_ALLOC;
   }
@@ -844,8 +941,9 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
       sc.rho[m] = f;
       f += Z * nrows[m];
     }
-    sc.ns = split ? f : nullptr;
-    if (split) f += (size_t)Z * 3 * ns_stride;
+    const bool ns_scratch = split && !ns_on_chip(a);
+    sc.ns = ns_scratch ? f : nullptr;
+    if (ns_scratch) f += (size_t)Z * 3 * ns_stride;
     uintptr_t up = (reinterpret_cast<uintptr_t>(f) + 255) & ~uintptr_t(255);
     __nv_bfloat16* b = reinterpret_cast<__nv_bfloat16*>(up);
     auto take = [&](size_t n) {
@@ -922,7 +1020,7 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
   }
 
   // Gradients of 512 x 128 / 128 x 512 run the shared-memory-resident kernel.
-  const bool ns_tc = split && dk == kN5 && dv == kN5 && dh == kNsCluster * kN5;
+  const bool ns_tc = ns_on_chip(a);
   if (ns_tc)
     check(cudaFuncSetAttribute(ns5_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)(sizeof(Ns5Smem) + 1024)));
