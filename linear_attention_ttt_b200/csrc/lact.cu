@@ -20,8 +20,10 @@
 // Non-causal (update, then apply): L1 without Aq, L2 without Y, L3, L4, then
 // Aq and Y with the updated weights.
 // Precision: GD uses bf16 operands with fp32 accumulation; Muon uses
-// split-bf16 operands (x = hi + lo, products hi*hi + lo*hi + hi*lo) because
-// the unit-step Muon scan amplifies per-chunk rounding across chunks.
+// split-bf16 operands (x = hi + lo, products hi*hi + lo*hi + hi*lo) on the
+// update path because the unit-step Muon scan amplifies per-chunk rounding
+// across chunks. The apply path (Aq, Y) feeds only the output: there the
+// weights keep hi / lo and Aq is plain bf16.
 #include <cooperative_groups.h>
 
 #include <cstdint>
@@ -796,7 +798,6 @@ void segs(Problem& p, int n, const int (*ab)[2]) {
 const int kSegExact[1][2] = {{0, 0}};
 const int kSegBsplit[2][2] = {{0, 0}, {0, 1}};
 const int kSegAsplit[2][2] = {{0, 0}, {1, 0}};
-const int kSegBoth[3][2] = {{0, 0}, {1, 0}, {0, 1}};
 
 gemm::EpiArgs epi_base(const LactArgs& a, int s0, int rows_valid) {
   gemm::EpiArgs e;
@@ -1088,9 +1089,10 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
       segs(p, nsegW, reinterpret_cast<const int(*)[2]>(segW));
       p.epi = gemm::EPI_AQ;
       p.e = epi_base(a, s0, bc);
-      p.e.nsplit = split ? 2 : 1;
+      // The apply path produces only the layer output, so Aq is stored as
+      // plain bf16 even under Muon (the weights keep their hi / lo parts).
+      p.e.nsplit = 1;
       p.e.optr[0] = sc.aq[0];
-      p.e.optr[3] = sc.aq[1];
       p.e.orows = chunk;
       p.e.ocols = dh;
     };
@@ -1102,7 +1104,7 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
       p.N = dv;
       p.K = dh;
       if (split)
-        segs(p, 3, kSegBoth);
+        segs(p, 2, kSegBsplit);  // Aq (bf16) x W2 hi + Aq x W2 lo
       else
         segs(p, 1, kSegExact);
       p.epi = gemm::EPI_Y;
