@@ -20,7 +20,13 @@
 // The A operands come from tensor memory, so the only shared-memory operands
 // are Q, K (from TMA) and P (written by the score warps).
 //
-// One CTA per (batch, head), 16 warps:
+// Each (batch, head) runs on two CTAs that split the sequence at tile `mid`.
+// CTA 0 handles tiles [0, mid). CTA 1 first builds the state after tile mid-1
+// with MMAs only: per tile, K scaled by eta in place and
+// S^T += V^T (diag(eta) K) with both operands in shared memory. It then
+// handles tiles [mid, end) with the full loop below and writes W_final.
+//
+// Per CTA, 16 warps:
 //   warp 0      TMA producer: Q, K, V tiles into a 4-stage ring (plus L2
 //               prefetch further ahead); eta to smem
 //   warp 1      TMEM owner; one thread issues all tcgen05.mma
@@ -63,6 +69,7 @@ struct Smem {
   float eta[kStages][TT];
   uint64_t full[kStages], stage_free[kStages];
   uint64_t sc_full[2], p_ready[2], vt_ready[2], y_full[2], y_free[2], s_ready, done;
+  uint64_t k_scaled[2], p1_done;  // state-only prefix (second CTA of a head)
   uint32_t tmem_base;
 };
 
@@ -121,8 +128,11 @@ __global__ void __launch_bounds__(kThreads, 1) la_tc_kernel(const __grid_constan
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                       ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.x, b = bh / p.H, h = bh % p.H;
-  const int ntiles = (p.T + TT - 1) / TT;
+  const int bh = blockIdx.x >> 1, seg = blockIdx.x & 1, b = bh / p.H, h = bh % p.H;
+  const int ntot = (p.T + TT - 1) / TT, mid = (ntot + 1) / 2;
+  // tiles [0, p1) build the state only; tiles [p1, tend) run the full loop
+  const int p1 = seg ? mid : 0, tend = seg ? ntot : mid, n2 = tend - p1;
+  const int s0 = seg ? 1 : 0;  // s_ready phase of the first full tile
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -138,6 +148,9 @@ __global__ void __launch_bounds__(kThreads, 1) la_tc_kernel(const __grid_constan
     }
     mbar_init(&sm.s_ready, 4);
     mbar_init(&sm.done, 1);
+    mbar_init(&sm.k_scaled[0], 4);
+    mbar_init(&sm.k_scaled[1], 4);
+    mbar_init(&sm.p1_done, 1);
     fence_mbar_init();
   }
   if (warp == 1) umma::tmem_alloc(&sm.tmem_base, kTmemCols);
@@ -169,9 +182,9 @@ __global__ void __launch_bounds__(kThreads, 1) la_tc_kernel(const __grid_constan
       prefetch_tmap(&p.tq);
       prefetch_tmap(&p.tk);
       prefetch_tmap(&p.tv);
-      for (int j = 0; j < kL2Ahead && j < ntiles; ++j)
+      for (int j = 0; j < kL2Ahead && j < tend; ++j)
         for (int x = 0; x < 2; ++x) {
-          tma_prefetch_l2_4d(&p.tq, 64 * x, j * TT, h, b);
+          if (j >= p1) tma_prefetch_l2_4d(&p.tq, 64 * x, j * TT, h, b);
           tma_prefetch_l2_4d(&p.tk, 64 * x, j * TT, h, b);
           tma_prefetch_l2_4d(&p.tv, 64 * x, j * TT, h, b);
         }
@@ -182,8 +195,8 @@ __global__ void __launch_bounds__(kThreads, 1) la_tc_kernel(const __grid_constan
     const float* eta = p.eta.p + b * p.eta.sb + h * p.eta.sh;
     auto load_eta = [&](int j, float& e0, float& e1) {
       const int t = j * TT + lane;
-      e0 = (j < ntiles && t < p.T) ? eta[(int64_t)t * p.eta.st] : 0.f;
-      e1 = (j < ntiles && t + 32 < p.T) ? eta[(int64_t)(t + 32) * p.eta.st] : 0.f;
+      e0 = (j < tend && t < p.T) ? eta[(int64_t)t * p.eta.st] : 0.f;
+      e1 = (j < tend && t + 32 < p.T) ? eta[(int64_t)(t + 32) * p.eta.st] : 0.f;
     };
     float r0a, r0b, r1a, r1b, r2a, r2b, r3a, r3b;
     load_eta(0, r0a, r0b);
@@ -192,11 +205,12 @@ __global__ void __launch_bounds__(kThreads, 1) la_tc_kernel(const __grid_constan
     load_eta(3, r3a, r3b);
     int j = 0;
     auto issue = [&](float& ea, float& eb) -> bool {
-      if (j >= ntiles) return false;
+      if (j >= tend) return false;
       const int s = j % kStages;
-      if (lane == 0 && j + kL2Ahead < ntiles)
+      const bool full_tile = j >= p1;  // state-only tiles need no Q
+      if (lane == 0 && j + kL2Ahead < tend)
         for (int x = 0; x < 2; ++x) {
-          tma_prefetch_l2_4d(&p.tq, 64 * x, (j + kL2Ahead) * TT, h, b);
+          if (j + kL2Ahead >= p1) tma_prefetch_l2_4d(&p.tq, 64 * x, (j + kL2Ahead) * TT, h, b);
           tma_prefetch_l2_4d(&p.tk, 64 * x, (j + kL2Ahead) * TT, h, b);
           tma_prefetch_l2_4d(&p.tv, 64 * x, (j + kL2Ahead) * TT, h, b);
         }
@@ -207,9 +221,9 @@ __global__ void __launch_bounds__(kThreads, 1) la_tc_kernel(const __grid_constan
       sm.eta[s][lane + 32] = eb;
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive_expect_tx(&sm.full[s], 3 * kTileBytes);
+        mbar_arrive_expect_tx(&sm.full[s], (full_tile ? 3 : 2) * kTileBytes);
         for (int x = 0; x < 2; ++x) {
-          tma_load_4d(sm.q[s] + x * 8192, &p.tq, &sm.full[s], 64 * x, t0, h, b);
+          if (full_tile) tma_load_4d(sm.q[s] + x * 8192, &p.tq, &sm.full[s], 64 * x, t0, h, b);
           tma_load_4d(sm.k[s] + x * 8192, &p.tk, &sm.full[s], 64 * x, t0, h, b);
           tma_load_4d(sm.v[s] + x * 8192, &p.tv, &sm.full[s], 64 * x, t0, h, b);
         }
@@ -227,10 +241,10 @@ __global__ void __launch_bounds__(kThreads, 1) la_tc_kernel(const __grid_constan
       const uint32_t id_y = umma::instr_desc(1, D, TT, 0, 0);     // S^T Q^T, Vt^T P^T (A in TMEM)
       const uint32_t id_ds = umma::instr_desc(1, D, D, 0, 1);     // Vt^T K           (A in TMEM)
       auto issue_scores = [&](int j, bool block) -> int {  // 1 issued, 0 not ready, -1 timeout
-        const int s = j % kStages;
+        const int g = p1 + j, s = g % kStages;              // g: tile index in the sequence
         if (block) {
-          if (!mbar_wait(&sm.full[s], (j / kStages) & 1, p.status)) return -1;
-        } else if (!mbar_try_wait(&sm.full[s], (j / kStages) & 1)) {
+          if (!mbar_wait(&sm.full[s], (g / kStages) & 1, p.status)) return -1;
+        } else if (!mbar_try_wait(&sm.full[s], (g / kStages) & 1)) {
           return 0;
         }
         umma::fence_after();
@@ -245,18 +259,37 @@ __global__ void __launch_bounds__(kThreads, 1) la_tc_kernel(const __grid_constan
         return 1;
       };
       bool ok = true;
-      int issued = 0;  // score tiles issued so far
-      for (int j = 0; j < ntiles && ok; ++j) {
-        const int s = j % kStages, x = j & 1;
+      // state-only prefix: S^T += V^T (diag(eta) K), both operands MN-major
+      if (p1 > 0) {
+        const uint32_t id_p1 = umma::instr_desc(1, D, D, 1, 1);
+        ok = mbar_wait(&sm.s_ready, 0, p.status);  // S^T holds W0^T
+        for (int j = 0; j < p1 && ok; ++j) {
+          const int s = j % kStages;
+          ok = mbar_wait(&sm.full[s], (j / kStages) & 1, p.status) &&
+               mbar_wait(&sm.k_scaled[j & 1], (j >> 1) & 1, p.status);
+          if (!ok) break;
+          umma::fence_after();
+          const uint32_t va = smem_u32(sm.v[s]), ka = smem_u32(sm.k[s]);
+#pragma unroll
+          for (int kk = 0; kk < TT / 16; ++kk)
+            umma::mma_bf16(tmem + kColS, umma::smem_desc(va + kk * 2048, 8192, 1024),
+                           umma::smem_desc(ka + kk * 2048, 8192, 1024), id_p1, 1);
+          umma::commit(&sm.stage_free[s]);
+        }
+        umma::commit(&sm.p1_done);
+      }
+      int issued = 0;  // score tiles issued so far (counted from p1)
+      for (int j = 0; j < n2 && ok; ++j) {
+        const int g = p1 + j, s = g % kStages, x = j & 1;
         // the score epilogue needs the scores of tiles j and j+1 in flight
-        while (ok && issued < j + 2 && issued < ntiles) {
+        while (ok && issued < j + 2 && issued < n2) {
           ok = issue_scores(issued, true) > 0;
           ++issued;
         }
         if (!ok) break;
         ok = mbar_wait(&sm.p_ready[x], (j >> 1) & 1, p.status) &&
              mbar_wait(&sm.vt_ready[x], (j >> 1) & 1, p.status) &&
-             mbar_wait(&sm.s_ready, j & 1, p.status) &&
+             mbar_wait(&sm.s_ready, (s0 + j) & 1, p.status) &&
              (j < 2 || mbar_wait(&sm.y_free[x], ((j - 2) >> 1) & 1, p.status));
         if (!ok) break;
         umma::fence_after();
@@ -280,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1) la_tc_kernel(const __grid_constan
                                 umma::smem_desc(ka + kk * 2048, 8192, 1024), id_ds, 1);
         umma::commit(&sm.y_full[x]);
         umma::commit(&sm.stage_free[s]);
-        if (issued == j + 2 && issued < ntiles) {
+        if (issued == j + 2 && issued < n2) {
           const int r = issue_scores(issued, false);
           if (r < 0) ok = false;
           issued += r > 0;
@@ -294,9 +327,38 @@ __global__ void __launch_bounds__(kThreads, 1) la_tc_kernel(const __grid_constan
     const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
     // column r of the V tile: box r / 64, 16-byte chunk (r % 64) / 8, byte 2 * (r % 8)
     const uint32_t box = (uint32_t)(r >> 6) * 8192, chunk = (r & 63) >> 3, byte = (r & 7) * 2;
-    for (int j = 0; j < ntiles; ++j) {
-      const int s = j % kStages, x = j & 1;
+    // state-only prefix: K rows scaled by eta in place (8 x 16 bytes per thread)
+    const int ti = threadIdx.x - 32 * kVtWarp0;  // 0..127
+    for (int j = 0; j < p1; ++j) {
+      const int s = j % kStages;
       if (!mbar_wait(&sm.full[s], (j / kStages) & 1, p.status)) return;
+      // k_scaled[j & 1] is free again once tile j-2's MMAs have completed
+      // (they released that tile's stage)
+      if (j >= 2 && !mbar_wait(&sm.stage_free[(j - 2) % kStages], ((j - 2) / kStages) & 1, p.status))
+        return;
+      const float* et = sm.eta[s];
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const int c = ti + 128 * m;                 // 16-byte chunk of the K tile
+        const int t = (c & 511) >> 3;               // its row (token)
+        uint4* ptr = reinterpret_cast<uint4*>(sm.k[s] + (c >> 9) * 8192 + t * 128 + (c & 7) * 16);
+        uint4 u = *ptr;
+        uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+        const float e = et[t];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const __nv_bfloat162 x2 = *reinterpret_cast<const __nv_bfloat162*>(&w[q]);
+          w[q] = pack2(e * __low2float(x2), e * __high2float(x2));
+        }
+        *ptr = u;
+      }
+      umma::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.k_scaled[j & 1]);
+    }
+    for (int j = 0; j < n2; ++j) {
+      const int g = p1 + j, s = g % kStages, x = j & 1;
+      if (!mbar_wait(&sm.full[s], (g / kStages) & 1, p.status)) return;
       // the Vt^T buffer of tile j-2 is free once that tile's MMAs are done
       if (j >= 2 && !mbar_wait(&sm.y_full[x], ((j - 2) >> 1) & 1, p.status)) return;
       const uint8_t* vb = sm.v[s] + box + byte;
@@ -318,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1) la_tc_kernel(const __grid_constan
     // ------------------------------------------------------------ score epilogue
     const int q4 = warp & 3;
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
-    for (int j = 0; j < ntiles; ++j) {
+    for (int j = 0; j < n2; ++j) {
       const int x = j & 1;
       if (!mbar_wait(&sm.sc_full[x], (j >> 1) & 1, p.status)) return;
       umma::fence_after();
@@ -348,20 +410,29 @@ __global__ void __launch_bounds__(kThreads, 1) la_tc_kernel(const __grid_constan
     const int q4 = warp & 3;
     const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
     const int r = q4 * 32 + lane;  // dv row
-    for (int j = 0; j < ntiles; ++j) {
+    if (p1 > 0) {
+      // the state after the prefix, copied to bf16 for the first full tile
+      if (!mbar_wait(&sm.p1_done, 0, p.status)) return;
+      umma::fence_after();
+      refresh_state_copy(tl);
+      umma::fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.s_ready);  // phase 1
+    }
+    for (int j = 0; j < n2; ++j) {
       const int x = j & 1;
       // On a timeout the warp still takes part in both named barriers below.
       const bool ok = mbar_wait(&sm.y_full[x], (j >> 1) & 1, p.status);
       umma::fence_after();
       // 1) bf16 copy of the updated state for the next tile's S^T Q^T
-      if (ok && j + 1 < ntiles) {
+      if (ok && j + 1 < n2) {
         refresh_state_copy(tl);
         umma::fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.s_ready);
       }
       // 2) Y^T tile -> [t][dv] bf16 staging -> 16-byte row pieces
-      const int t0 = j * TT;
+      const int t0 = (p1 + j) * TT;
       __nv_bfloat16* st = sm.ystage;
       for (int c = 0; c < TT && ok; c += 16) {
         float v[16];
@@ -384,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1) la_tc_kernel(const __grid_constan
       if (!ok) return;
     }
     // final state
-    if (p.W_final) {
+    if (p.W_final && seg == 1) {
       if (!mbar_wait(&sm.done, 0, p.status)) return;
       umma::fence_after();
       float* Wf = p.W_final + (int64_t)bh * D * D;
@@ -437,7 +508,7 @@ cudaError_t launch_la_tc(const LinearArgs& a, cudaStream_t s) {
   cudaError_t e =
       cudaFuncSetAttribute(la_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  la_tc_kernel<<<a.B * a.H, kThreads, smem, s>>>(p);
+  la_tc_kernel<<<a.B * a.H * 2, kThreads, smem, s>>>(p);
   return cudaGetLastError();
 }
 
