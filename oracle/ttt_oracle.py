@@ -45,7 +45,9 @@ Layouts: q, k [B,H,T,dk]; v [B,H,T,dv]; eta [B,H,T]; TTT-Linear W0 [H,dk,dv]
 (or with a leading B). Outputs y [B,H,T,dv].
 
 Parity status: every function below is pinned by the ``-m "not gpu"`` tests in
-``tests/test_oracle_pins.py`` except where its docstring says otherwise.
+``tests/test_oracle_pins.py`` (the forward pass) and
+``tests/test_oracle_backward.py`` (the TTT-Linear backward pass) except where
+its docstring says otherwise.
 """
 from __future__ import annotations
 
@@ -190,6 +192,83 @@ def linear_attention(q, k, v, eta, S0):
         S = S + eta[:, :, t, None, None] * np.einsum("zha,zhc->zhac", k[:, :, t], v[:, :, t])
         y[:, :, t] = np.einsum("zha,zhac->zhc", q[:, :, t], S)
     return y, S
+
+
+# ----------------------------------------------------------------------------
+# TTT-Linear backward: the reverse chunk scan (training).
+# ----------------------------------------------------------------------------
+
+def ttt_linear_minibatch_bwd(q, k, v, eta, W0, chunk, loss, dy, dW_final=None):
+    """Gradients of a scalar objective through ``ttt_linear_minibatch``, given
+    dL/dy [B,H,T,dv] and dL/dW_final [B,H,dk,dv] (None means zero).
+
+    The chain rule written out for the mini-batch rule ([TTT] "병렬화:
+    Mini-batch Gradient Descent"). In a chunk with start weights W, token t
+    uses W_t = W - sum_{i<=t} eta_i g_i(W) and y_t = q_t W_t, and the chunk's
+    last W_t starts the next chunk. With U_t = dL/dW_t = q_t^T dy_t (plus, at
+    the chunk's last token, the gradient of the next chunk's start) and
+    R_i = sum of U_t over t >= i in the chunk:
+      dq_t    = dy_t W_t^T
+      deta_i  = -<R_i, g_i(W)>
+      and Gamma_i = -eta_i R_i flows into g_i:
+        MSE, g_i = k_i^T e_i with e_i = k_i W - v_i:
+          de_i = k_i Gamma_i,  dk_i = e_i Gamma_i^T + de_i W^T,
+          dv_i = -de_i,        dL/dW gains k_i^T de_i;
+        inner product, g_i = -k_i^T v_i:
+          dk_i = -v_i Gamma_i^T,  dv_i = -k_i Gamma_i.
+      dL/dW (the chunk start) = sum_t U_t (+ the MSE terms), carried back to
+      the previous chunk.
+    Returns (dq, dk, dv, deta, dW0); dW0 is summed over the batch when W0 is
+    shared by it ([H,dk,dv])."""
+    q, k, v, eta, dy = map(_f64, (q, k, v, eta, dy))
+    B, H, T, _ = q.shape
+    if chunk < 1:
+        raise ValueError("chunk must be >= 1")
+    if loss not in (LOSS_MSE, LOSS_NEG_DOT):
+        raise ValueError(loss)
+    # forward: the start weights of every chunk
+    W = _broadcast_state(W0, B)
+    starts = list(range(0, T, chunk))
+    W_start = []
+    for s in starts:
+        W_start.append(W.copy())
+        for i in range(s, min(s + chunk, T)):
+            W = W - eta[:, :, i, None, None] * loss_grad(W_start[-1], k[:, :, i], v[:, :, i], loss)
+    G = np.zeros_like(W) if dW_final is None else _f64(dW_final).copy()
+    dq, dk, dv, deta = (np.zeros_like(x) for x in (q, k, v, eta))
+    for ci in reversed(range(len(starts))):
+        s, Ws = starts[ci], W_start[ci]
+        e = min(s + chunk, T)
+        g, Wt, acc = [], [], np.zeros_like(Ws)
+        for i in range(s, e):
+            g.append(loss_grad(Ws, k[:, :, i], v[:, :, i], loss))
+            acc = acc + eta[:, :, i, None, None] * g[-1]
+            Wt.append(Ws - acc)
+        R = np.zeros_like(Ws)
+        dWs = np.zeros_like(Ws)
+        for idx in reversed(range(e - s)):
+            t = s + idx
+            U = np.einsum("zha,zhc->zhac", q[:, :, t], dy[:, :, t])
+            if t == e - 1:
+                U = U + G
+            dq[:, :, t] = np.einsum("zhc,zhac->zha", dy[:, :, t], Wt[idx])
+            R = R + U
+            dWs = dWs + U
+            deta[:, :, t] = -np.einsum("zhac,zhac->zh", R, g[idx])
+            Gam = -eta[:, :, t, None, None] * R
+            if loss == LOSS_MSE:
+                err = np.einsum("zha,zhac->zhc", k[:, :, t], Ws) - v[:, :, t]
+                de = np.einsum("zha,zhac->zhc", k[:, :, t], Gam)
+                dk[:, :, t] = (np.einsum("zhac,zhc->zha", Gam, err) +
+                               np.einsum("zhc,zhac->zha", de, Ws))
+                dv[:, :, t] = -de
+                dWs = dWs + np.einsum("zha,zhc->zhac", k[:, :, t], de)
+            else:
+                dk[:, :, t] = -np.einsum("zhac,zhc->zha", Gam, v[:, :, t])
+                dv[:, :, t] = -np.einsum("zha,zhac->zhc", k[:, :, t], Gam)
+        G = dWs
+    dW0 = G.sum(axis=0) if _f64(W0).ndim == 3 else G
+    return dq, dk, dv, deta, dW0
 
 
 def arithmetic_intensity(b, h):
