@@ -58,7 +58,8 @@
  *    allowed); dk, dv in [1, 256] for fp32 tensors. bf16 kernels take
  *    dk = dv in {64, 128} for TTT-Linear and d in {64, 128, 256},
  *    dh a multiple of 128 up to 1024 for LaCT; other sizes return
- *    TTT_ERR_UNSUPPORTED.
+ *    TTT_ERR_UNSUPPORTED, and so do T > 2^30 tokens and B*H > 2^24
+ *    (the kernels index tokens and (batch, head) pairs with 32-bit integers).
  */
 #ifndef TTT_B200_H
 #define TTT_B200_H

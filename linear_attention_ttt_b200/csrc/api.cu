@@ -28,6 +28,12 @@ int* device_status_ptr() {
 
 size_t elem_size(int32_t dtype) { return dtype == TTT_BF16 ? 2 : 4; }
 
+// Sizes the kernels index with 32-bit integers: tokens per sequence (tile
+// starts plus one tile stay below 2^31) and (batch, head) pairs (grids of a
+// few CTAs per pair).
+constexpr int64_t kMaxT = (int64_t)1 << 30;
+constexpr int64_t kMaxHeads = (int64_t)1 << 24;
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Byte range [lo, hi) touched by a strided tensor (non-negative strides).
@@ -157,7 +163,7 @@ ttt_status ttt_linear_fwd(const ttt_tensor* q, const ttt_tensor* k, const ttt_te
   const int64_t B = q->shape[0], H = q->shape[1], T = q->shape[2], dk = q->shape[3];
   const int64_t dv = v->shape[3];
   if (B < 1 || H < 1 || T < 0 || dk < 1 || dv < 1) return TTT_ERR_SHAPE;
-  if (dk > 256 || dv > 256 || T > (int64_t)1 << 31 || B * H > (1 << 30)) return TTT_ERR_UNSUPPORTED;
+  if (dk > 256 || dv > 256 || T > kMaxT || B * H > kMaxHeads) return TTT_ERR_UNSUPPORTED;
   const int32_t dt = q->dtype;
   if (dt != TTT_F32 && dt != TTT_BF16) return TTT_ERR_DTYPE;
   ttt_status st;
@@ -249,6 +255,8 @@ ttt_status lact_build_args(const ttt_tensor* q, const ttt_tensor* k, const ttt_t
   const int64_t dv = v->shape[3];
   const int64_t dh = W1->shape[W1->ndim - 2];
   if (B < 1 || H < 1 || T < 0 || dk < 1 || dv < 1 || dh < 1) return TTT_ERR_SHAPE;
+  if (dk > 256 || dv > 256 || dh > 4096 || T > kMaxT || B * H > kMaxHeads)
+    return TTT_ERR_UNSUPPORTED;
   const int32_t dt = q->dtype;
   if (dt != TTT_F32 && dt != TTT_BF16) return TTT_ERR_DTYPE;
   ttt_status st;

@@ -163,6 +163,23 @@ def test_rejects_oversized_heads(lib):
     assert c.call(lib) == ERR["TTT_ERR_UNSUPPORTED"]
 
 
+def test_rejects_sizes_beyond_32_bit_indexing(lib):
+    """More than 2^30 tokens or 2^24 (batch, head) pairs: refused before any
+    descriptor is read further (the kernels index with 32-bit integers)."""
+    c = Case(T=(1 << 30) + 1)
+    assert c.call(lib) == ERR["TTT_ERR_UNSUPPORTED"]
+    c = Case(B=1 << 12, H=(1 << 12) + 1)
+    assert c.call(lib) == ERR["TTT_ERR_UNSUPPORTED"]
+
+    def long_seq(ts):
+        T = (1 << 30) + 1
+        for n in ("q", "k", "v", "out"):
+            ts[n] = tok(1, 2, T, 128, base=ts[n].data)
+        ts["eta"] = dense((1, 2, T), ts["eta"].data)
+    assert lact_call(lib, mutate=long_seq) == ERR["TTT_ERR_UNSUPPORTED"]
+    assert lact_call(lib, dh=8192) == ERR["TTT_ERR_UNSUPPORTED"]
+
+
 def lact_call(lib, rule=0, causal=1, dh=512, mutate=None):
     gap = 1 << 28
     Bs, H, T, d = 1, 2, 64, 128
