@@ -368,9 +368,12 @@ def main():
         if dist is not None:
             dist.barrier()
 
+    nvtx = torch.cuda.nvtx  # named ranges for profilers (no effect without one)
+    nvtx.range_push("warmup")
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
+    nvtx.range_pop()
 
     # ---- device-resident timing (whole step == the kernel launches) ----
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -379,6 +382,7 @@ def main():
     torch.cuda.synchronize()
     sampler = ClockSampler(device.index if world == 1 else local)
     with sampler:
+        nvtx.range_push("timed")
         t_wall = time.perf_counter()
         for i in range(args.steps):
             if flush is not None:
@@ -388,6 +392,7 @@ def main():
             ev[i][1].record(stream)
         torch.cuda.synchronize()
         t_wall = time.perf_counter() - t_wall
+        nvtx.range_pop()
     barrier()
     per = [a.elapsed_time(b) for a, b in ev]
     total_ms = max_over_ranks(sum(per), dist, device)
@@ -408,6 +413,7 @@ def main():
     torch.cuda.synchronize()
     barrier()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    nvtx.range_push("e2e")
     a.record(stream)
     for _ in range(e2e_steps):
         for k2, v2 in host.items():
@@ -416,6 +422,7 @@ def main():
         host_out.copy_(step.out, non_blocking=True)
     b.record(stream)
     torch.cuda.synchronize()
+    nvtx.range_pop()
     e2e_ms = max_over_ranks(a.elapsed_time(b) / e2e_steps, dist, device)
     e2e_value = job_throughput(tokens_per_step, world, e2e_ms)
 

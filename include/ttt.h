@@ -183,6 +183,15 @@ ttt_status ttt_get_device_status(void* stream);
 /* Library version, as major*10000 + minor*100 + patch. */
 int32_t ttt_version(void);
 
+/*
+ * Self-test of the failure detection: enqueues one CTA that waits on a
+ * barrier nothing arrives at. The bounded wait gives up after its limit
+ * (about 2 s), records TTT_ERR_TIMEOUT in the device status word and the
+ * kernel returns, leaving the context usable; ttt_get_device_status() then
+ * returns TTT_ERR_TIMEOUT (and clears it). Returns TTT_OK once launched.
+ */
+ttt_status ttt_selftest_wait_timeout(void* stream);
+
 #ifdef __cplusplus
 }
 #endif

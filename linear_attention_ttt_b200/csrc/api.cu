@@ -116,11 +116,31 @@ ttt_status lact_check_final(const ttt_tensor* W, int64_t B, int64_t H, int64_t r
   return TTT_OK;
 }
 
+// Failure-detection self-test: one thread waits on a barrier that nothing
+// arrives at. The bounded wait gives up after its time limit, records the
+// timeout in the status word and the kernel returns (no trap, no hang).
+__global__ void selftest_wait_kernel(int* status) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    ttt::mbar_init(&bar, 1);
+    ttt::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) ttt::mbar_wait(&bar, 0, status);
+}
+
 }  // namespace
 
 extern "C" {
 
 int32_t ttt_version(void) { return 100; }
+
+ttt_status ttt_selftest_wait_timeout(void* stream) {
+  int* p = device_status_ptr();
+  if (!p) return TTT_ERR_CUDA;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  return cudaGetLastError() == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
+}
 
 const char* ttt_status_string(int32_t s) {
   switch (s) {

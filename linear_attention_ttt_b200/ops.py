@@ -59,6 +59,7 @@ SIGNATURES = {
     "ttt_status_string": ([ctypes.c_int32], ctypes.c_char_p),
     "ttt_get_device_status": ([ctypes.c_void_p], ctypes.c_int32),
     "ttt_version": ([], ctypes.c_int32),
+    "ttt_selftest_wait_timeout": ([ctypes.c_void_p], ctypes.c_int32),
 }
 
 
@@ -177,6 +178,12 @@ def lact_swiglu_fwd_noalloc(q, k, v, eta, W1, W2, W3, chunk: int,
                                           r[8], r[9], r[10], _stream(stream))
     _check(code, "lact_swiglu_fwd_noalloc")
     return (out, *F) if finals else out
+
+
+def selftest_wait_timeout(stream=None) -> None:
+    """Enqueue the failure-detection self-test (a bounded wait that runs out);
+    device_status() afterwards returns TTT_ERR_TIMEOUT."""
+    _check(load().ttt_selftest_wait_timeout(_stream(stream)), "ttt_selftest_wait_timeout")
 
 
 def device_status(stream=None) -> int:
