@@ -271,6 +271,75 @@ def ttt_linear_minibatch_bwd(q, k, v, eta, W0, chunk, loss, dy, dW_final=None):
     return dq, dk, dv, deta, dW0
 
 
+# ----------------------------------------------------------------------------
+# TTT-MLP (the scope table's "next" row f3): a two-layer ReLU MLP fast weight.
+# ----------------------------------------------------------------------------
+
+def mlp_apply(W1, b1, W2, b2, x):
+    """f(x) = W2 ReLU(W1 x + b1) + b2 ([TTT] "TTT-MLP"), for the rows x of X
+    [n, dk]; W1 [dh, dk], b1 [dh], W2 [dv, dh], b2 [dv]. Returns [n, dv]."""
+    x = _f64(x)
+    return np.maximum(x @ _f64(W1).T + _f64(b1), 0.0) @ _f64(W2).T + _f64(b2)
+
+
+def mlp_loss(W1, b1, W2, b2, k, v):
+    """Per-token loss 1/2 ||f(k) - v||^2 (the MSE reading of TTT-Linear,
+    applied to the MLP fast weight)."""
+    r = mlp_apply(W1, b1, W2, b2, _f64(k)[None])[0] - _f64(v)
+    return 0.5 * float(r @ r)
+
+
+def mlp_grads(W1, b1, W2, b2, k, v):
+    """Gradients of ``mlp_loss`` for one token: with h = W1 k + b1,
+    a = ReLU(h), r = W2 a + b2 - v: db2 = r, dW2 = r a^T, dh = (W2^T r) [h > 0]
+    (derivative 0 at h = 0), db1 = dh, dW1 = dh k^T."""
+    W1, b1, W2, b2, k, v = map(_f64, (W1, b1, W2, b2, k, v))
+    h = W1 @ k + b1
+    a = np.maximum(h, 0.0)
+    r = W2 @ a + b2 - v
+    dh = (W2.T @ r) * (h > 0)
+    return np.outer(dh, k), dh, np.outer(r, a), r
+
+
+def ttt_mlp_token_recurrence(q, k, v, eta, W1, b1, W2, b2):
+    """One gradient step per token ([TTT] "TTT 정의" with the MLP of
+    "TTT-MLP"): W_t = W_{t-1} - eta_t grad(W_{t-1}; k_t, v_t), y_t = f(q_t; W_t),
+    for all four parameters. Single sequence: q, k [T, dk], v [T, dv], eta [T].
+    Returns (y [T, dv], (W1, b1, W2, b2) after the last token)."""
+    P = [_f64(x).copy() for x in (W1, b1, W2, b2)]
+    q, k, v, eta = map(_f64, (q, k, v, eta))
+    y = np.zeros((q.shape[0], v.shape[1]))
+    for t in range(q.shape[0]):
+        g = mlp_grads(*P, k[t], v[t])
+        P = [p - eta[t] * gi for p, gi in zip(P, g)]
+        y[t] = mlp_apply(*P, q[t][None])[0]
+    return y, tuple(P)
+
+
+def ttt_mlp_minibatch(q, k, v, eta, W1, b1, W2, b2, chunk):
+    """Mini-batch gradient descent on the MLP fast weight, the rule of
+    [TTT] "병렬화: Mini-batch Gradient Descent" for every parameter: with t'
+    the chunk start, P_t = P_{t'} - sum_{i=t'}^{t} eta_i grad(P_{t'}; k_i, v_i)
+    and y_t = f(q_t; P_t). Single sequence, as ``ttt_mlp_token_recurrence``.
+    Parity unpinned against the pages' numbers (they print none); pinned by
+    the tests in ``tests/test_oracle_ttt_mlp.py``."""
+    if chunk < 1:
+        raise ValueError("chunk must be >= 1")
+    P = [_f64(x).copy() for x in (W1, b1, W2, b2)]
+    q, k, v, eta = map(_f64, (q, k, v, eta))
+    T = q.shape[0]
+    y = np.zeros((T, v.shape[1]))
+    for s in range(0, T, chunk):
+        start = [p.copy() for p in P]
+        acc = [np.zeros_like(p) for p in P]
+        for t in range(s, min(s + chunk, T)):
+            g = mlp_grads(*start, k[t], v[t])
+            acc = [a + eta[t] * gi for a, gi in zip(acc, g)]
+            P = [p0 - a for p0, a in zip(start, acc)]
+            y[t] = mlp_apply(*P, q[t][None])[0]
+    return y, tuple(P)
+
+
 def arithmetic_intensity(b, h):
     """[TTT] "Arithmetic Intensity 분석": fast weight h x h, chunk input b x h,
     r = 2 h^2 b / (2 h^2 + 4 h b)  (= b / (1 + 2b/h), bounded by min(h/2, b))."""
