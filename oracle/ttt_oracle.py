@@ -321,8 +321,8 @@ def ttt_mlp_minibatch(q, k, v, eta, W1, b1, W2, b2, chunk):
     [TTT] "병렬화: Mini-batch Gradient Descent" for every parameter: with t'
     the chunk start, P_t = P_{t'} - sum_{i=t'}^{t} eta_i grad(P_{t'}; k_i, v_i)
     and y_t = f(q_t; P_t). Single sequence, as ``ttt_mlp_token_recurrence``.
-    Parity unpinned against the pages' numbers (they print none); pinned by
-    the tests in ``tests/test_oracle_ttt_mlp.py``."""
+    The pages print no numbers for TTT-MLP; the pins are the closed forms,
+    invariants and derivative checks of ``tests/test_oracle_ttt_mlp.py``."""
     if chunk < 1:
         raise ValueError("chunk must be >= 1")
     P = [_f64(x).copy() for x in (W1, b1, W2, b2)]
