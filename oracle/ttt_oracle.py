@@ -340,6 +340,39 @@ def ttt_mlp_minibatch(q, k, v, eta, W1, b1, W2, b2, chunk):
     return y, tuple(P)
 
 
+# ----------------------------------------------------------------------------
+# Sliding-window attention beside LaCT (the scope table's "next" row f4).
+# ----------------------------------------------------------------------------
+
+def sliding_window_attention(q, k, v, window):
+    """Causal softmax attention over the last `window` tokens ([LaCT] 3.1:
+    window attention computes the relations between tokens within a fixed
+    range): y_t = sum_{t-window < i <= t} softmax_i(q_t . k_i / sqrt(d)) v_i.
+    Single sequence: q, k [T, d], v [T, dv]. Returns [T, dv]."""
+    q, k, v = map(_f64, (q, k, v))
+    if window < 1:
+        raise ValueError("window must be >= 1")
+    T, d = q.shape
+    y = np.zeros((T, v.shape[1]))
+    for t in range(T):
+        lo = max(0, t - window + 1)
+        s = k[lo:t + 1] @ q[t] / np.sqrt(d)
+        p = np.exp(s - s.max())
+        y[t] = (p / p.sum()) @ v[lo:t + 1]
+    return y
+
+
+def lact_with_window_attention(q, k, v, eta, W1, W2, W3, chunk, update_rule, window):
+    """The LaCT layer with window attention beside it, both on the same q, k,
+    v ([LaCT] 4: attention and TTT share Q, K, V and their outputs are
+    combined), combined by summing the two outputs (causal order).
+    Single sequence, weights [dh, d] / [d, dh]. Returns [T, dv]."""
+    y, *_ = lact_swiglu(_f64(q)[None, None], _f64(k)[None, None], _f64(v)[None, None],
+                        _f64(eta)[None, None], _f64(W1)[None], _f64(W2)[None], _f64(W3)[None],
+                        chunk, update_rule, 1)
+    return y[0, 0] + sliding_window_attention(q, k, v, window)
+
+
 def arithmetic_intensity(b, h):
     """[TTT] "Arithmetic Intensity 분석": fast weight h x h, chunk input b x h,
     r = 2 h^2 b / (2 h^2 + 4 h b)  (= b / (1 + 2b/h), bounded by min(h/2, b))."""
