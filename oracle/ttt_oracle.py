@@ -57,6 +57,7 @@ LOSS_MSE = 0
 LOSS_NEG_DOT = 1
 UPDATE_GD = 0
 UPDATE_MUON = 1
+UPDATE_MOMENTUM = 2
 
 # Newton-Schulz quintic coefficients (a, b, c) and the normalisation epsilon.
 NS_COEFFS = (3.4445, -4.7750, 2.0315)
@@ -487,6 +488,42 @@ def lact_swiglu(q, k, v, eta, W1, W2, W3, chunk, update_rule=UPDATE_GD, causal=1
                     y[bi, h, s:e] = swiglu(w1, w2, w3, q[bi, h, s:e])
             Ws[0][bi, h], Ws[1][bi, h], Ws[2][bi, h] = w1, w2, w3
     return y, Ws[0], Ws[1], Ws[2]
+
+
+def lact_swiglu_momentum(q, k, v, eta, W1, W2, W3, chunk, beta, causal=1, M0=None):
+    """LaCT with the momentum update ([LaCT] 3.3 names GD, momentum and Muon
+    as the compared update rules, and prints no formula for momentum). The
+    reading taken is heavy-ball momentum over chunk gradients, per matrix:
+      M <- beta * M + G,   W <- renorm(W - M),   M = 0 before the first chunk
+    (or M0), with G the eta-weighted summed gradient of ``lact_swiglu`` and
+    the same apply/update order and row renormalisation. beta = 0 is GD.
+    Returns (y, W1_final, W2_final, W3_final, (M1, M2, M3)), all [B,H,...]."""
+    q, k, v, eta = map(_f64, (q, k, v, eta))
+    B, H, T, _ = q.shape
+    if chunk < 1:
+        raise ValueError("chunk must be >= 1")
+    Ws = [_broadcast_state(W, B) for W in (W1, W2, W3)]
+    Ms = [np.zeros_like(W) for W in Ws] if M0 is None else [_broadcast_state(M, B) for M in M0]
+    y = np.zeros((B, H, T, v.shape[-1]))
+    for bi in range(B):
+        for h in range(H):
+            w = [W[bi, h].copy() for W in Ws]
+            m = [M[bi, h].copy() for M in Ms]
+            rho = [row_norms(x) for x in w]
+            for s in range(0, T, chunk):
+                e = min(s + chunk, T)
+                if causal:
+                    y[bi, h, s:e] = swiglu(*w, q[bi, h, s:e])
+                g = lact_grads(*w, k[bi, h, s:e], v[bi, h, s:e], eta[bi, h, s:e])
+                for i in range(3):
+                    m[i] = beta * m[i] + g[i]
+                    w[i] = renorm_rows(w[i] - m[i], rho[i])
+                if not causal:
+                    y[bi, h, s:e] = swiglu(*w, q[bi, h, s:e])
+            for i in range(3):
+                Ws[i][bi, h] = w[i]
+                Ms[i][bi, h] = m[i]
+    return y, Ws[0], Ws[1], Ws[2], tuple(Ms)
 
 
 def lact_swiglu_prefix(q, k, v, eta, W1, W2, W3, chunk, update_rule, n_chunks, bh):
