@@ -377,3 +377,60 @@ def test_oracle_matches_stored_golden_values():
         got = compute(name)
         for key, val in stored[name].items():
             assert np.allclose(np.asarray(got[key]), np.asarray(val), rtol=1e-12, atol=1e-14), (name, key)
+
+
+# --------------------------------------------------------------------------
+# The Muon branch of the LaCT scan, composed by hand from pinned pieces:
+# lact_grads (finite differences), the Newton-Schulz polynomial evaluated on
+# numpy's SVD, and the row renorm written out as a scale per row.
+# ("Test-Time Training Done Right" review 3.3: the summed gradient is
+# orthogonalised by Newton-Schulz, then the step, then L2 normalisation.)
+# --------------------------------------------------------------------------
+
+def _ns5_by_svd(G):
+    U, S, Vt = np.linalg.svd(G, full_matrices=False)
+    s = S / (np.sqrt(np.sum(G * G)) + 1e-7)
+    a, b, c = 3.4445, -4.7750, 2.0315
+    for _ in range(5):
+        s = a * s + b * s ** 3 + c * s ** 5
+    return (U * s) @ Vt
+
+
+def _rescale_rows(W, W_init):
+    target = np.sqrt(np.sum(W_init * W_init, axis=1))
+    return W * (target / np.sqrt(np.sum(W * W, axis=1)))[:, None]
+
+
+def _swiglu_by_hand(W1, W2, W3, X):
+    h1 = X @ W1.T
+    return ((h1 / (1.0 + np.exp(-h1))) * (X @ W3.T)) @ W2.T
+
+
+def _muon_chunk_by_hand(Ws, W_init, K, V, eta):
+    G = O.lact_grads(*Ws, K, V, eta)
+    return [_rescale_rows(W - _ns5_by_svd(g), Wi) for W, g, Wi in zip(Ws, G, W_init)]
+
+
+@pytest.mark.parametrize("causal", [1, 0])
+def test_lact_muon_scan_is_svd_polynomial_step_then_renorm(causal):
+    """Two chunks (the second ragged) of one (batch, head) under Muon: the
+    weights after each chunk are renorm(W - U p5(S/(||G||_F+eps)) V^T) with G
+    taken at the renormalised weights of the previous chunk, and the outputs
+    are f of the weights before (causal) or after (non-causal) the chunk's
+    update. A scan that skipped Newton-Schulz, used the raw weights for the
+    second gradient, or renormalised to the previous chunk's norms fails."""
+    w = synth.make_lact(1, 1, 11, 3, 5, 6, O.UPDATE_MUON, 21, dtype=synth.F32, eta_scale=0.2)
+    q, k, v, eta = (np.float64(x[0, 0]) for x in (w.q, w.k, w.v, w.eta))
+    W_init = [np.float64(W[0]) for W in (w.W1, w.W2, w.W3)]
+    y, F1, F2, F3 = O.lact_swiglu(w.q, w.k, w.v, w.eta, w.W1, w.W2, w.W3, 6, O.UPDATE_MUON, causal)
+    W_a = _muon_chunk_by_hand(W_init, W_init, k[:6], v[:6], eta[:6])
+    W_b = _muon_chunk_by_hand(W_a, W_init, k[6:], v[6:], eta[6:])
+    for F, ref in zip((F1, F2, F3), W_b):
+        assert relerr(F[0, 0], ref) < 1e-10
+    y_ref = np.concatenate([_swiglu_by_hand(*(W_init if causal else W_a), q[:6]),
+                            _swiglu_by_hand(*(W_a if causal else W_b), q[6:])])
+    assert relerr(y[0, 0], y_ref) < 1e-10
+    # the step is not a plain gradient step: Newton-Schulz changed the weights
+    W_gd = [_rescale_rows(W - g, Wi) for W, g, Wi in
+            zip(W_init, O.lact_grads(*W_init, k[:6], v[:6], eta[:6]), W_init)]
+    assert max(relerr(a, b) for a, b in zip(W_a, W_gd)) > 1e-3
