@@ -1,22 +1,26 @@
 """Benchmark of the chunked TTT-layer forward on B200 (one JSON line on rank 0).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 2] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 5] [--also 2,3,3:256,4]
+                    [--impl ours|reference]
 
 A step is one forward pass of the layer over one batch of synthetic inputs
 (seeded, shaped like the pages' workloads; see linear_attention_ttt_b200.synth).
-Default workload: the inner-product-loss layer (chunked causal linear
-attention), batch 4, 16 heads, T=4096, d=128, chunk 64, bf16 tokens, fp32
-state. Workloads 1-5 can be selected with --workload.
+Headline workload (the JSON line's own value): LaCT SwiGLU with the Muon
+update, batch 1, 8 heads, T=131072, d=128, hidden 512, chunk 4096, bf16
+tokens, fp32 fast weights -- the largest single-GPU workload. The same run
+also measures the inner-product layer (B4 H16 T4096 d128 b64), small-chunk
+TTT-Linear MSE (B8 H16 T8192 d64, chunks 16 and 256) and LaCT GD (B2 H4
+T32768 d256 dh512 b2048) and reports them under "workloads" (--also).
 
 Multi-GPU: one process per GPU (torchrun). (batch, head) pairs are
 independent, so every rank runs its own replica of the workload with no
 collective on the data path (weak scaling); timing is the max over ranks.
 
-Timing: W untimed warm-up steps, then K steps between CUDA events on the
-launching stream, bracketed by a barrier and device synchronisation. Inputs
-of the default workload (q, k, v: 201 MB) exceed the 126 MB L2, so no flush is
-needed between steps; smaller workloads flush L2 by writing a 256 MB buffer
-before every step, outside the events of the kernel timing (see "l2").
+Timing: W untimed warm-up steps, then K steps, each between CUDA events on
+the launching stream, bracketed by a barrier and device synchronisation.
+Before every step L2 is flushed by reading a 256 MB buffer (outside the
+events): the read evicts the previous step's lines and writes back its dirty
+ones, so no write-back of earlier work lands inside a timed step.
 """
 from __future__ import annotations
 
@@ -296,13 +300,163 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
+def parse_extra(spec):
+    """'2,3,3:256,4' -> [(2, None), (3, None), (3, 256), (4, None)]"""
+    out = []
+    for item in filter(None, (x.strip() for x in spec.split(","))):
+        idx, _, ch = item.partition(":")
+        out.append((int(idx), int(ch) if ch else None))
+    return out
+
+
+def roofline(w, ms_per_launch, pk):
+    """Roofline entry of the kernel (TTT-Linear: the one launch of a step) or
+    of the whole step (LaCT: every launch of the chunk loop, so the figure is
+    a lower bound on the GEMM kernel's own fraction)."""
+    key = kernel_key(w)
+    if w.variant == "lact":
+        flops = lact_flops(w)
+        peak = pk["bf16_tflops"]
+        achieved = flops / (ms_per_launch / 1e3) / 1e12
+        return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None,
+                "peak_source": pk["_source"] + " bf16_tflops (burst: a step of a few ms timed alone)",
+                "kernel": "lact step (all launches)", "algorithmic_flops_per_step": flops}
+    byts = linear_bytes(w)
+    achieved = byts / (ms_per_launch / 1e3) / 1e9
+    sha = source_sha(KERNEL_SOURCES[key])
+    return {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / pk["hbm_gbs"], "traffic": recorded_traffic(key, sha),
+            "peak_source": pk["_source"] + " hbm_gbs", "kernel": key,
+            "algorithmic_bytes_per_launch": byts, "kernel_source_sha": sha}
+
+
+def cpu_baseline(w):
+    n = cpu_sample_heads(w)
+    dt, toks = cpu_oracle_step(w, n)
+    return {"value": toks / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"fp64 numpy oracle (dual form / LaCT scan) on {n} of {w.B * w.H} "
+                      f"(batch, head) sequences, {dt:.1f} s"}
+
+
+def workload_cfg(w, world):
+    cfg = {"workload": w.name, "batch": w.B, "heads": w.H, "seq_len": w.T, "dk": w.dk,
+           "dv": w.dv, "chunk": w.chunk, "variant": w.variant,
+           "loss": ("mse" if w.loss == 0 else "neg_dot") if w.variant != "lact" else "neg_dot_swiglu",
+           "parallelism": f"replicas{world}"}
+    if w.variant == "lact":
+        cfg.update(dh=w.dh, update_rule="muon" if w.update_rule else "gd", causal=w.causal)
+    return cfg
+
+
+class Runner:
+    """Times workloads on this rank's GPU (device-resident inputs; CUDA events
+    on the launching stream; L2 flushed by a read before every timed step)."""
+
+    def __init__(self, args, dist, device):
+        self.args, self.dist, self.device = args, dist, device
+        # 256 MB > L2: reading it evicts every line the previous step left,
+        # and dirty lines are written back during the read, outside the timing.
+        self.flush = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device=device)
+        self.stream = torch.cuda.current_stream()
+
+    def barrier(self):
+        if self.dist is not None:
+            self.dist.barrier()
+
+    def l2_flush(self):
+        torch.sum(self.flush)
+
+    def device_timing(self, step):
+        args = self.args
+        nvtx = torch.cuda.nvtx  # named ranges for profilers (no effect without one)
+        nvtx.range_push("warmup")
+        for _ in range(args.warmup):
+            self.l2_flush()
+            step()
+        torch.cuda.synchronize()
+        nvtx.range_pop()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        self.barrier()
+        torch.cuda.synchronize()
+        sampler = ClockSampler(self.device.index)
+        with sampler:
+            nvtx.range_push("timed")
+            t_wall = time.perf_counter()
+            for i in range(args.steps):
+                self.l2_flush()
+                ev[i][0].record(self.stream)
+                step()
+                ev[i][1].record(self.stream)
+            torch.cuda.synchronize()
+            t_wall = time.perf_counter() - t_wall
+            nvtx.range_pop()
+        self.barrier()
+        per = [a.elapsed_time(b) for a, b in ev]
+        ms = max_over_ranks(sum(per), self.dist, self.device) / args.steps
+        return ms, sampler.summary(), t_wall
+
+    def e2e(self, w, d, step):
+        """Same metric through the public API with host buffers: every step
+        copies its inputs from pinned host memory and reads back its results
+        (y, and W_final for TTT-Linear) inside the timed region."""
+        host = {k: v.to("cpu").pin_memory() for k, v in d.items()}
+        results = [step.out] + ([step.Wf] if getattr(step, "Wf", None) is not None else [])
+        host_res = [torch.empty(r.shape, dtype=r.dtype).pin_memory() for r in results]
+        h2d = sum(v.numel() * v.element_size() for v in host.values())
+        d2h = sum(r.numel() * r.element_size() for r in host_res)
+        n = max(3, min(self.args.steps, 20))
+
+        def one():
+            for k2, v2 in host.items():
+                d[k2].copy_(v2, non_blocking=True)
+            step()
+            for hr, r in zip(host_res, results):
+                hr.copy_(r, non_blocking=True)
+        for _ in range(2):
+            one()
+        torch.cuda.synchronize()
+        self.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.nvtx.range_push("e2e")
+        a.record(self.stream)
+        for _ in range(n):
+            one()
+        b.record(self.stream)
+        torch.cuda.synchronize()
+        torch.cuda.nvtx.range_pop()
+        ms = max_over_ranks(a.elapsed_time(b) / n, self.dist, self.device)
+        return ms, h2d, d2h
+
+    def measure(self, w, world, with_e2e):
+        d = upload(w, self.device)
+        step = Step(w, d)
+        ms, clocks, t_wall = self.device_timing(step)
+        res = {"ms_per_step": ms, "value": job_throughput(w.B * w.T, world, ms),
+               "roofline": roofline(w, ms, peaks()),
+               "gpu_launches": (step.launches or 0) * self.args.steps,
+               "clocks": clocks, "wall_s_timed": t_wall}
+        if with_e2e:
+            e_ms, h2d, d2h = self.e2e(w, d, step)
+            res["e2e"] = {"value": job_throughput(w.B * w.T, world, e_ms), "unit": "tokens/s",
+                          "h2d_bytes_per_step": h2d * world, "d2h_bytes_per_step": d2h * world}
+        del step, d
+        torch.cuda.empty_cache()
+        return res
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", type=int, default=2)
+    ap.add_argument("--workload", type=int, default=5,
+                    help="headline workload (default 5: LaCT Muon, the largest single-GPU one)")
     ap.add_argument("--chunk", type=int, default=None)
+    ap.add_argument("--also", default="2,3,3:256,4",
+                    help="workloads measured in the same run and reported under 'workloads' "
+                         "(index[:chunk], comma separated; '' for none)")
     ap.add_argument("--seq-len", type=int, default=None,
                     help="shorter sequence of the same workload (profiling); the default "
                          "line uses the workload's own length")
@@ -315,14 +469,7 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
 
     w = rank_workload(args.workload, rank, chunk=args.chunk, seq_len=args.seq_len)
-    tokens_per_step = w.B * w.T
-    base_cfg = {"workload": w.name, "batch": w.B, "heads": w.H, "seq_len": w.T, "dk": w.dk,
-                "dv": w.dv, "chunk": w.chunk, "variant": w.variant,
-                "loss": ("mse" if w.loss == 0 else "neg_dot") if w.variant != "lact" else "neg_dot_swiglu",
-                "parallelism": f"replicas{world}"}
-    if w.variant == "lact":
-        base_cfg.update(dh=w.dh, update_rule="muon" if w.update_rule else "gd",
-                        causal=w.causal)
+    base_cfg = workload_cfg(w, world)
 
     if args.impl == "reference":
         if rank != 0:
@@ -356,115 +503,39 @@ def main():
         torch.cuda.set_device(0)
     device = torch.device("cuda", torch.cuda.current_device())
     ops.load()
+    runner = Runner(args, dist, device)
+    want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
 
-    d = upload(w, device)
-    step = Step(w, d)
-    in_bytes = sum(x.numel() * x.element_size() for x in d.values())
-    l2_flush = in_bytes < 2 * L2_BYTES
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device) if l2_flush else None
-    stream = torch.cuda.current_stream()
-
-    def barrier():
-        if dist is not None:
-            dist.barrier()
-
-    nvtx = torch.cuda.nvtx  # named ranges for profilers (no effect without one)
-    nvtx.range_push("warmup")
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    nvtx.range_pop()
-
-    # ---- device-resident timing (whole step == the kernel launches) ----
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-    barrier()
-    torch.cuda.synchronize()
-    sampler = ClockSampler(device.index if world == 1 else local)
-    with sampler:
-        nvtx.range_push("timed")
-        t_wall = time.perf_counter()
-        for i in range(args.steps):
-            if flush is not None:
-                flush.zero_()
-            ev[i][0].record(stream)
-            step()
-            ev[i][1].record(stream)
-        torch.cuda.synchronize()
-        t_wall = time.perf_counter() - t_wall
-        nvtx.range_pop()
-    barrier()
-    per = [a.elapsed_time(b) for a, b in ev]
-    total_ms = max_over_ranks(sum(per), dist, device)
-    ms_per_step = total_ms / args.steps
-    value = job_throughput(tokens_per_step, world, ms_per_step)
-
-    # ---- end to end through the public API with host buffers ----
-    host = {k: v.to("cpu").pin_memory() for k, v in d.items()}
-    host_out = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
-    h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = host_out.numel() * host_out.element_size()
-    e2e_steps = max(3, min(args.steps, 20))
-    for _ in range(2):
-        for k2, v2 in host.items():
-            d[k2].copy_(v2, non_blocking=True)
-        step()
-        host_out.copy_(step.out, non_blocking=True)
-    torch.cuda.synchronize()
-    barrier()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    nvtx.range_push("e2e")
-    a.record(stream)
-    for _ in range(e2e_steps):
-        for k2, v2 in host.items():
-            d[k2].copy_(v2, non_blocking=True)
-        step()
-        host_out.copy_(step.out, non_blocking=True)
-    b.record(stream)
-    torch.cuda.synchronize()
-    nvtx.range_pop()
-    e2e_ms = max_over_ranks(a.elapsed_time(b) / e2e_steps, dist, device)
-    e2e_value = job_throughput(tokens_per_step, world, e2e_ms)
-
-    pk = peaks()
-    key = kernel_key(w)
-    if w.variant == "lact":
-        flops = lact_flops(w)
-        peak = pk["bf16_tflops_sustained"] if "bf16_tflops_sustained" in pk else pk["bf16_tflops"]
-        achieved = flops / (ms_per_step / 1e3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": None,
-                "peak_source": pk["_source"] + " bf16 (sustained)", "kernel": "lact step"}
-    else:
-        byts = linear_bytes(w)
-        launch_ms = ms_per_step  # one launch per step
-        achieved = byts / (launch_ms / 1e3) / 1e9
-        sha = source_sha(KERNEL_SOURCES[key])
-        roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / pk["hbm_gbs"], "traffic": recorded_traffic(key, sha),
-                "peak_source": pk["_source"] + " hbm_gbs", "kernel": key,
-                "algorithmic_bytes_per_launch": byts, "kernel_source_sha": sha}
-
+    head = runner.measure(w, world, with_e2e=True)
     cfg = dict(base_cfg)
-    cfg["l2"] = ("flushed (256 MB write) before every timed step" if l2_flush
-                 else f"inputs {in_bytes / 1e6:.0f} MB > L2 126 MB, no flush")
-    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+    cfg["l2"] = "flushed before every timed step (256 MB read, outside the timed events)"
+    line = {"metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if w.dtype == synth.BF16 else "f32", "data": "synthetic",
-            "config": cfg, "roofline": roof,
-            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d * world,
-                    "d2h_bytes_per_step": d2h * world},
-            "gpu_launches": (step.launches or 0) * args.steps,
-            "clocks": sampler.summary(), "wall_s_timed": t_wall}
+            "config": cfg, "roofline": head["roofline"], "e2e": head["e2e"],
+            "gpu_launches": head["gpu_launches"], "clocks": head["clocks"],
+            "wall_s_timed": head["wall_s_timed"]}
+    if want_cpu:
+        line["cpu_baseline"] = cpu_baseline(w)
 
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n = cpu_sample_heads(w)
-        dt, toks = cpu_oracle_step(w, n)
-        line["cpu_baseline"] = {"value": toks / dt, "unit": "tokens/s", "cores": blas_threads(),
-                                "kind": "oracle",
-                                "sample": f"fp64 numpy oracle (dual form / LaCT scan) on {n} of "
-                                          f"{w.B * w.H} (batch, head) sequences, {dt:.1f} s"}
+    extras = []
+    for idx, ch in parse_extra(args.also):
+        wx = rank_workload(idx, rank, chunk=ch, seq_len=args.seq_len)
+        r = runner.measure(wx, world, with_e2e=False)
+        item = {"config": workload_cfg(wx, world), "ms_per_step": r["ms_per_step"],
+                "value": r["value"], "unit": "tokens/s",
+                "dtype": "bf16" if wx.dtype == synth.BF16 else "f32",
+                "roofline": r["roofline"], "gpu_launches": r["gpu_launches"],
+                "clocks": r["clocks"]}
+        if want_cpu:
+            item["cpu_baseline"] = cpu_baseline(wx)
+        extras.append(item)
+        del wx
+    if extras:
+        line["workloads"] = extras
+        line["gpu_launches"] += sum(x["gpu_launches"] for x in extras)
+
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:

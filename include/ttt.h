@@ -53,6 +53,11 @@
  *  - Device-side errors: kernels that wait on a barrier give up after a
  *    bounded number of polls and record TTT_ERR_TIMEOUT in a device status
  *    word instead of hanging; ttt_get_device_status() reads and clears it.
+ *  - Device state: the status word, the LaCT scratch pool and the
+ *    no-allocation array are set up once per device and kept for the life of
+ *    the process. Resetting the device (cudaDeviceReset) or tearing down its
+ *    primary context invalidates them; calling the library afterwards in the
+ *    same process is not supported.
  *  - Supported sizes: B, H, T >= 1 (T = 0 is accepted and does nothing
  *    except copying W0 to W_final); chunk >= 1 (a shorter last chunk is
  *    allowed); dk, dv in [1, 256] for fp32 tensors. bf16 kernels take
@@ -156,11 +161,20 @@ ttt_status lact_swiglu_fwd_ex(const ttt_tensor* q, const ttt_tensor* k, const tt
  * Scratch: a fixed 32 MiB device array inside the library (each device that
  * loads the library holds it until the process exits). A problem whose
  * scratch need exceeds it is rejected with TTT_ERR_SCRATCH before anything
- * is launched. The need is about, per (batch, head), 4 bytes x (3 x 2 x
- * weight elements + chunk x dh) + 2 bytes x (weight elements + 4 x chunk x
- * dh), doubled for the bf16 parts under Muon.
+ * is launched. The need per (batch, head), with E = 2*dh*dk + dv*dh weight
+ * elements, R = 2*dh + dv weight rows and c = min(chunk, T), is
+ *   4 bytes x (2*E + R)  +  2 bytes x (E + 4*c*dh) x (2 under Muon),
+ * plus, under Muon when the gradients are not 128 x 512 (dk = dv = 128 and
+ * dh = 512 keep Newton-Schulz on chip), 4 bytes x 3 x (16*s*s + dh*dk + 64)
+ * with s = min(dk, dh); the sum over all (batch, head) pairs gets 4096
+ * bytes of alignment slack. Example: dk = dv = 128, dh = 512, chunk 1024,
+ * GD: 1,577,472 + 4,587,520 = 6,164,992 bytes per (batch, head), so up to
+ * five (batch, head) pairs fit.
  * The first call on a device looks up the array's device address with that
- * device current; make that first call before any stream capture.
+ * device current and keeps it for the life of the process; make that first
+ * call before any stream capture. A cudaDeviceReset (or any teardown of the
+ * device's primary context) invalidates the kept address, so this library
+ * must not be called again in that process afterwards.
  * All calls share the one array: calls whose GPU work overlaps (on
  * different streams, or from different host threads) race on it and give
  * wrong results; serialise them. What a previous call left in the array does

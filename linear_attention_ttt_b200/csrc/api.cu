@@ -332,9 +332,13 @@ ttt_status lact_build_args(const ttt_tensor* q, const ttt_tensor* k, const ttt_t
   a.update_rule = update_rule;
   a.causal = causal;
   a.dtype = dt;
-  a.status = device_status_ptr();
-  if (!a.status) return TTT_ERR_CUDA;
+  a.status = nullptr;
   return TTT_OK;
+}
+
+ttt_status lact_attach_status(LactArgs* a) {
+  a->status = device_status_ptr();
+  return a->status ? TTT_OK : TTT_ERR_CUDA;
 }
 
 }  // namespace ttt
@@ -351,6 +355,7 @@ ttt_status lact_swiglu_fwd_ex(const ttt_tensor* q, const ttt_tensor* k, const tt
   ttt_status st = ttt::lact_build_args(q, k, v, eta, W1, W2, W3, chunk, update_rule, causal, out,
                                        W1_final, W2_final, W3_final, &a);
   if (st != TTT_OK) return st;
+  if ((st = ttt::lact_attach_status(&a)) != TTT_OK) return st;
   return ttt::lact_forward(a, static_cast<cudaStream_t>(stream));
 }
 

@@ -27,11 +27,16 @@ size_t lact_scratch_bytes(const LactArgs& a);
 // 256-byte aligned. Allocates nothing.
 ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* scratch, size_t bytes);
 
-// Validates the C-ABI arguments of lact_swiglu_fwd_ex and fills `a`.
+// Validates the C-ABI arguments of lact_swiglu_fwd_ex and fills `a`, except
+// its status pointer. Makes no CUDA call.
 ttt_status lact_build_args(const ttt_tensor* q, const ttt_tensor* k, const ttt_tensor* v,
                            const ttt_tensor* eta, const ttt_tensor* W1, const ttt_tensor* W2,
                            const ttt_tensor* W3, int32_t chunk, int32_t update_rule,
                            int32_t causal, const ttt_tensor* out, const ttt_tensor* W1_final,
                            const ttt_tensor* W2_final, const ttt_tensor* W3_final, LactArgs* a);
+
+// Sets a->status to the current device's status word (TTT_ERR_CUDA if the
+// device or the symbol cannot be queried).
+ttt_status lact_attach_status(LactArgs* a);
 
 }  // namespace ttt

@@ -57,6 +57,7 @@ extern "C" ttt_status lact_swiglu_fwd_noalloc(
   const size_t need = ttt::lact_scratch_bytes(a);
   if (need == 0) return TTT_ERR_UNSUPPORTED;
   if (need > kLactPoolBytes) return TTT_ERR_SCRATCH;
+  if ((st = ttt::lact_attach_status(&a)) != TTT_OK) return st;
   void* pool = pool_ptr();
   if (!pool) return TTT_ERR_CUDA;
   // Every buffer the scan reads is written earlier in the same call (the

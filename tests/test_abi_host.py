@@ -209,3 +209,44 @@ def test_lact_rejects_bad_arguments(lib):
     def alias(ts):
         ts["out"].data = ts["q"].data
     assert lact_call(lib, mutate=alias) == ERR["TTT_ERR_ARG"]
+
+
+def noalloc_call(lib, H, T, d, dh, chunk, rule):
+    gap = 1 << 36
+    ts = [tok(1, H, T, d, base=FAKE), tok(1, H, T, d, base=FAKE + gap),
+          tok(1, H, T, d, base=FAKE + 2 * gap), dense((1, H, T), FAKE + 3 * gap),
+          dense((H, dh, d), FAKE + 4 * gap), dense((H, d, dh), FAKE + 5 * gap),
+          dense((H, dh, d), FAKE + 6 * gap), tok(1, H, T, d, base=FAKE + 7 * gap)]
+    r = ctypes.byref
+    return lib.lact_swiglu_fwd_noalloc(*(r(t) for t in ts[:7]), chunk, rule, 1, r(ts[7]),
+                                       None, None, None, None)
+
+
+def documented_scratch_per_pair(d, dh, chunk, T, muon):
+    """The per-(batch, head) scratch need as include/ttt.h states it for
+    lact_swiglu_fwd_noalloc."""
+    E, R, c = 2 * dh * d + d * dh, 2 * dh + d, min(chunk, T)
+    need = 4 * (2 * E + R) + 2 * (E + 4 * c * dh) * (2 if muon else 1)
+    if muon and not (d == 128 and dh == 512):
+        s = min(d, dh)
+        need += 4 * 3 * (16 * s * s + dh * d + 64)
+    return need
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(),
+                    reason="fake pointers: on a GPU a call that fits would launch")
+@pytest.mark.parametrize("d,dh,chunk,T,rule", [(128, 512, 1024, 4096, 0), (128, 512, 256, 4096, 1),
+                                               (64, 256, 512, 2048, 1), (256, 512, 128, 512, 0),
+                                               (256, 1024, 64, 100, 1)])
+def test_noalloc_scratch_limit_is_the_documented_formula(lib, d, dh, chunk, T, rule):
+    """The largest number of (batch, head) pairs the 32 MiB array accepts is
+    the one the header's formula (and its worked example) predicts: that many
+    pairs pass the size check (and, with no GPU, stop at the CUDA lookup),
+    one more returns TTT_ERR_SCRATCH before any CUDA call."""
+    per = documented_scratch_per_pair(d, dh, chunk, T, rule == 1)
+    n_max = ((32 << 20) - 4096) // per
+    if (d, dh, chunk, rule) == (128, 512, 1024, 0):
+        assert per == 6164992 and n_max == 5      # the header's worked example
+    assert n_max >= 1
+    assert noalloc_call(lib, n_max, T, d, dh, chunk, rule) == ERR["TTT_ERR_CUDA"]
+    assert noalloc_call(lib, n_max + 1, T, d, dh, chunk, rule) == ERR["TTT_ERR_SCRATCH"]
