@@ -96,6 +96,11 @@ typedef enum { TTT_LOSS_MSE = 0, TTT_LOSS_NEG_DOT = 1 } ttt_loss;
 
 typedef enum { LACT_UPDATE_GD = 0, LACT_UPDATE_MUON = 1 } lact_update_rule;
 
+/* Gradient exchange of lact_swiglu_fwd_cp: must enqueue on `stream` an
+ * in-place sum over all ranks of the n fp32 values at `grads` (device
+ * memory), and return 0 (anything else aborts the call with TTT_ERR_CUDA). */
+typedef int32_t (*lact_grad_reduce_fn)(float* grads, size_t n, void* stream, void* user);
+
 typedef struct {
   void* data;          /* device pointer, 16-byte aligned */
   int32_t dtype;       /* ttt_dtype */
@@ -119,6 +124,65 @@ ttt_status ttt_linear_fwd(const ttt_tensor* q, const ttt_tensor* k, const ttt_te
                           const ttt_tensor* eta, const ttt_tensor* W0, int32_t chunk,
                           int32_t loss, const ttt_tensor* out, const ttt_tensor* W_final,
                           void* stream);
+
+/*
+ * TTT-Linear / inner-product layer backward (training): the gradients of a
+ * scalar objective through ttt_linear_fwd, given dL/dy and dL/dW_final.
+ * Same page and sections as ttt_linear_fwd; differentiating the mini-batch
+ * rule token by token, with U_t = q_t^T dy_t and R_t = G + sum of U over the
+ * tokens t..end of t's chunk (G = dL/dW at the chunk end):
+ *   dq_t = dy_t W_t^T,  deta_t = -<R_t, g_t>,
+ *   MSE (g_t = k_t^T e_t, e_t = k_t W_s - v_t): de_t = -eta_t k_t R_t,
+ *     dk_t = -eta_t R_t e_t^T + de_t W_s^T, dv_t = -de_t,
+ *     dL/dW_s = R_s + sum_t k_t^T de_t;
+ *   inner product (g_t = -k_t^T v_t): dk_t = eta_t R_t v_t^T,
+ *     dv_t = eta_t k_t R_t, dL/dW_s = R_s;
+ * dL/dW_s of a chunk is G of the chunk before it; that of the first chunk is
+ * dL/dW0.
+ *  q, k, v, eta, W0, chunk, loss   as in ttt_linear_fwd
+ *  dy       [B,H,T,dv]  same type as q
+ *  dW_final NULL (zero) or [B,H,dk,dv] fp32 contiguous
+ *  dq, dk   [B,H,T,dk], dv [B,H,T,dv]: same type as q
+ *  deta     [B,H,T] fp32 contiguous
+ *  dW0      W0's shape, fp32 contiguous; for a W0 shared over the batch
+ *           ([H,dk,dv]) the gradient is summed over the batch
+ * dk, dv <= 128 (TTT_ERR_UNSUPPORTED otherwise). Arithmetic is fp32 on the
+ * CUDA cores, one CTA per (batch, head). The MSE path keeps the start
+ * weights of every chunk in a stream-ordered workspace of
+ * B*H*ceil(T/chunk)*dk*dv*4 bytes (plus B*H*dk*dv*4 for a shared W0) from
+ * the library's pool; failure -> TTT_ERR_ALLOC.
+ */
+ttt_status ttt_linear_bwd(const ttt_tensor* q, const ttt_tensor* k, const ttt_tensor* v,
+                          const ttt_tensor* eta, const ttt_tensor* W0, int32_t chunk,
+                          int32_t loss, const ttt_tensor* dy, const ttt_tensor* dW_final,
+                          const ttt_tensor* dq, const ttt_tensor* dk, const ttt_tensor* dv,
+                          const ttt_tensor* deta, const ttt_tensor* dW0, void* stream);
+
+/*
+ * TTT-MLP layer forward: a two-layer ReLU MLP fast weight,
+ *   f(x) = W2 ReLU(W1 x + b1) + b2,
+ * trained per chunk by the mini-batch rule of ttt_linear_fwd on the loss
+ * 1/2 ||f(k_i) - v_i||^2 ("Test-Time Training (TTT)" summary, sections
+ * "TTT-MLP" and "병렬화: Mini-batch Gradient Descent"): all four parameters
+ * are fast weights, every gradient of a chunk is taken at the chunk-start
+ * parameters, token t's query sees the updates of tokens <= t of its chunk,
+ * and the ReLU derivative at 0 is taken as 0.
+ *  q, k [B,H,T,dk], v, out [B,H,T,dv]: fp32 or bf16 (one type for all four)
+ *  eta  [B,H,T] fp32
+ *  W1 [H,dh,dk], b1 [H,dh], W2 [H,dv,dh], b2 [H,dv] (shared over the batch)
+ *     or with a leading B (per sequence); fp32 contiguous, read-only
+ *  *_final NULL or [B,H,...] fp32 contiguous: parameters after the last token
+ * dk, dv <= 256 and dh <= 512 (TTT_ERR_UNSUPPORTED otherwise). Arithmetic is
+ * fp32 on the CUDA cores, one CTA per (batch, head), with a stream-ordered
+ * workspace of 2 copies of the parameters per (batch, head) from the
+ * library's pool (failure -> TTT_ERR_ALLOC).
+ */
+ttt_status ttt_mlp_fwd(const ttt_tensor* q, const ttt_tensor* k, const ttt_tensor* v,
+                       const ttt_tensor* eta, const ttt_tensor* W1, const ttt_tensor* b1,
+                       const ttt_tensor* W2, const ttt_tensor* b2, int32_t chunk,
+                       const ttt_tensor* out, const ttt_tensor* W1_final,
+                       const ttt_tensor* b1_final, const ttt_tensor* W2_final,
+                       const ttt_tensor* b2_final, void* stream);
 
 /*
  * LaCT SwiGLU layer forward.
@@ -146,6 +210,59 @@ ttt_status lact_swiglu_fwd_ex(const ttt_tensor* q, const ttt_tensor* k, const tt
                               int32_t causal, const ttt_tensor* out,
                               const ttt_tensor* W1_final, const ttt_tensor* W2_final,
                               const ttt_tensor* W3_final, void* stream);
+
+/*
+ * LaCT SwiGLU layer forward with the momentum update rule.
+ *  "Test-Time Training Done Right" review, section 3.3, lists GD, momentum
+ *  and Muon as the compared fast-weight update rules and prints no formula
+ *  for momentum. This library takes heavy-ball momentum on each matrix's
+ *  eta-weighted chunk gradient G (the gradient of lact_swiglu_fwd):
+ *      M <- beta * M + G,    W <- W - M,    then the row renorm,
+ *  with M = M0 before the first chunk (zero when M?_0 is NULL). beta = 0 is
+ *  plain GD. Apply/update order, precision (bf16 operands, fp32 state) and
+ *  every other argument are those of lact_swiglu_fwd_ex with update_rule =
+ *  LACT_UPDATE_GD.
+ *  beta   any finite float (NaN or infinite -> TTT_ERR_ARG)
+ *  M1_0, M3_0 [H,dh,dk] or [B,H,dh,dk]; M2_0 [H,dv,dh] or [B,H,dv,dh]; fp32
+ *         contiguous, NULLable (zero initial momentum)
+ *  M1_final, M3_final [B,H,dh,dk], M2_final [B,H,dv,dh]: fp32 contiguous,
+ *         NULLable; the momentum after the last chunk (pass it back as M?_0,
+ *         with the *_final weights as W?, to resume on a chunk boundary)
+ * Scratch as for lact_swiglu_fwd, plus one fp32 momentum matrix per weight.
+ */
+ttt_status lact_swiglu_fwd_momentum(const ttt_tensor* q, const ttt_tensor* k,
+                                    const ttt_tensor* v, const ttt_tensor* eta,
+                                    const ttt_tensor* W1, const ttt_tensor* W2,
+                                    const ttt_tensor* W3, int32_t chunk, float beta,
+                                    int32_t causal, const ttt_tensor* M1_0,
+                                    const ttt_tensor* M2_0, const ttt_tensor* M3_0,
+                                    const ttt_tensor* out, const ttt_tensor* W1_final,
+                                    const ttt_tensor* W2_final, const ttt_tensor* W3_final,
+                                    const ttt_tensor* M1_final, const ttt_tensor* M2_final,
+                                    const ttt_tensor* M3_final, void* stream);
+
+/*
+ * Context-parallel LaCT forward ("Test-Time Training Done Right" review,
+ * section 8: the tokens of a large chunk are split over devices, each
+ * computes the update gradient of its share, and the shares are summed).
+ * Each rank passes its own token shard: for a global chunk of C tokens
+ * split over R ranks, rank r holds sub-block r (C/R tokens) of every chunk,
+ * so its q, k, v, eta, out are [B,H,T/R,d] and `chunk` is C/R. The chunk
+ * loop is that of lact_swiglu_fwd_ex; after each chunk's gradient GEMMs the
+ * library calls `reduce` (on the calling host thread, in chunk order) to
+ * sum the gradients over the ranks before Newton-Schulz, the step and the
+ * renorm, which every rank then runs on identical data, so the weights stay
+ * identical across ranks. `reduce` NULL means one rank (no exchange).
+ * Every rank must make the same sequence of calls with the same B, H,
+ * chunk count, d, dh and update rule. Scratch as lact_swiglu_fwd.
+ */
+ttt_status lact_swiglu_fwd_cp(const ttt_tensor* q, const ttt_tensor* k, const ttt_tensor* v,
+                              const ttt_tensor* eta, const ttt_tensor* W1, const ttt_tensor* W2,
+                              const ttt_tensor* W3, int32_t chunk, int32_t update_rule,
+                              int32_t causal, const ttt_tensor* out,
+                              const ttt_tensor* W1_final, const ttt_tensor* W2_final,
+                              const ttt_tensor* W3_final, lact_grad_reduce_fn reduce,
+                              void* reduce_user, void* stream);
 
 /*
  * lact_swiglu_fwd_ex without any device memory allocation. (The pages have
@@ -187,12 +304,46 @@ ttt_status lact_swiglu_fwd_noalloc(const ttt_tensor* q, const ttt_tensor* k, con
                                    const ttt_tensor* W1_final, const ttt_tensor* W2_final,
                                    const ttt_tensor* W3_final, void* stream);
 
+/*
+ * Sliding-window causal softmax attention ("Test-Time Training Done Right"
+ * review, section 3.1: window attention models the relations between tokens
+ * within a fixed range; the pages give windows of 2K and 4K tokens):
+ *   y_t = sum_{t-window < i <= t} softmax_i(q_t . k_i / sqrt(d)) v_i.
+ *  q, k [B,H,T,d], v, out [B,H,T,d]: bf16, d in {64, 128, 256}
+ *  window >= 1 (a window of T or more is plain causal attention)
+ *  accumulate 0: out = y; 1: out = out + y (summed in fp32, rounded once)
+ * mma.sync tensor-core tiles (bf16 operands, fp32 accumulation) with an
+ * online softmax; fp32 tokens or other sizes -> TTT_ERR_UNSUPPORTED.
+ */
+ttt_status window_attention_fwd(const ttt_tensor* q, const ttt_tensor* k, const ttt_tensor* v,
+                                int32_t window, int32_t accumulate, const ttt_tensor* out,
+                                void* stream);
+
+/*
+ * LaCT's hybrid block: the LaCT layer (causal, lact_swiglu_fwd) and window
+ * attention on the same q, k, v, outputs summed (review, section 4: the
+ * attention and the TTT layer share Q, K and V and their outputs are
+ * combined; this library takes the sum). Arguments as lact_swiglu_fwd plus
+ * `window`; bf16 with d in {64, 128, 256}.
+ */
+ttt_status lact_swiglu_window_fwd(const ttt_tensor* q, const ttt_tensor* k, const ttt_tensor* v,
+                                  const ttt_tensor* eta, const ttt_tensor* W1,
+                                  const ttt_tensor* W2, const ttt_tensor* W3, int32_t chunk,
+                                  int32_t update_rule, int32_t window, const ttt_tensor* out,
+                                  void* stream);
+
 /* Static description of a status code (never NULL). */
 const char* ttt_status_string(int32_t status);
 
 /* Synchronises `stream`, returns the first device-side error recorded since
  * the last call (TTT_OK if none) and clears it. */
 ttt_status ttt_get_device_status(void* stream);
+
+/* Test hook of the failure handling: the next n stream-ordered scratch
+ * allocations of the library (LaCT, the TTT-Linear backward, TTT-MLP) fail
+ * as if the device were out of memory, so the calls return TTT_ERR_ALLOC
+ * without launching anything. n = 0 turns it off. No GPU fault is involved. */
+void ttt_test_fail_allocations(int32_t n);
 
 /* Library version, as major*10000 + minor*100 + patch. */
 int32_t ttt_version(void);

@@ -133,7 +133,9 @@ __global__ void selftest_wait_kernel(int* status) {
 
 extern "C" {
 
-int32_t ttt_version(void) { return 100; }
+int32_t ttt_version(void) { return 200; }
+
+void ttt_test_fail_allocations(int32_t n) { ttt::set_failing_allocs(n); }
 
 ttt_status ttt_selftest_wait_timeout(void* stream) {
   int* p = device_status_ptr();
@@ -333,6 +335,15 @@ ttt_status lact_build_args(const ttt_tensor* q, const ttt_tensor* k, const ttt_t
   a.causal = causal;
   a.dtype = dt;
   a.status = nullptr;
+  a.momentum = 0;
+  a.beta = 0.f;
+  a.reduce = nullptr;
+  a.reduce_user = nullptr;
+  for (int m = 0; m < 3; ++m) {
+    a.M0[m] = nullptr;
+    a.m0_sb[m] = 0;
+    a.M_final[m] = nullptr;
+  }
   return TTT_OK;
 }
 
@@ -365,6 +376,359 @@ ttt_status lact_swiglu_fwd(const ttt_tensor* q, const ttt_tensor* k, const ttt_t
                            int32_t causal, const ttt_tensor* out, void* stream) {
   return lact_swiglu_fwd_ex(q, k, v, eta, W1, W2, W3, chunk, update_rule, causal, out, nullptr,
                             nullptr, nullptr, stream);
+}
+
+}  // extern "C"
+
+extern "C" {
+
+ttt_status lact_swiglu_fwd_momentum(const ttt_tensor* q, const ttt_tensor* k,
+                                    const ttt_tensor* v, const ttt_tensor* eta,
+                                    const ttt_tensor* W1, const ttt_tensor* W2,
+                                    const ttt_tensor* W3, int32_t chunk, float beta,
+                                    int32_t causal, const ttt_tensor* M1_0,
+                                    const ttt_tensor* M2_0, const ttt_tensor* M3_0,
+                                    const ttt_tensor* out, const ttt_tensor* W1_final,
+                                    const ttt_tensor* W2_final, const ttt_tensor* W3_final,
+                                    const ttt_tensor* M1_final, const ttt_tensor* M2_final,
+                                    const ttt_tensor* M3_final, void* stream) {
+  ttt::LactArgs a;
+  ttt_status st = ttt::lact_build_args(q, k, v, eta, W1, W2, W3, chunk, LACT_UPDATE_GD, causal,
+                                       out, W1_final, W2_final, W3_final, &a);
+  if (st != TTT_OK) return st;
+  if (!(beta == beta) || beta < -1e30f || beta > 1e30f) return TTT_ERR_ARG;  // finite
+  const int64_t B = a.B, H = a.H, dk = a.dk, dv = a.dv, dh = a.dh;
+  const ttt_tensor* M0[3] = {M1_0, M2_0, M3_0};
+  const ttt_tensor* Mf[3] = {M1_final, M2_final, M3_final};
+  const int64_t rows[3] = {dh, dv, dh}, cols[3] = {dk, dh, dk};
+  for (int m = 0; m < 3; ++m) {
+    if (M0[m]) {
+      int64_t sb = 0;
+      if ((st = lact_check_weight(M0[m], B, H, rows[m], cols[m], &sb)) != TTT_OK) return st;
+      a.M0[m] = static_cast<const float*>(M0[m]->data);
+      a.m0_sb[m] = sb;
+    }
+    if ((st = lact_check_final(Mf[m], B, H, rows[m], cols[m])) != TTT_OK) return st;
+    a.M_final[m] = Mf[m] ? static_cast<float*>(Mf[m]->data) : nullptr;
+  }
+  // outputs overlap no input and no other output
+  const ttt_tensor* ins[] = {q, k, v, eta, W1, W2, W3, M1_0, M2_0, M3_0};
+  const ttt_tensor* outs[] = {out, W1_final, W2_final, W3_final, M1_final, M2_final, M3_final};
+  for (const ttt_tensor* o : outs) {
+    for (const ttt_tensor* in : ins)
+      if (overlaps(o, in)) return TTT_ERR_ARG;
+    for (const ttt_tensor* o2 : outs)
+      if (o != o2 && overlaps(o, o2)) return TTT_ERR_ARG;
+  }
+  a.momentum = 1;
+  a.beta = beta;
+  if ((st = ttt::lact_attach_status(&a)) != TTT_OK) return st;
+  return ttt::lact_forward(a, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"
+
+extern "C" {
+
+ttt_status ttt_linear_bwd(const ttt_tensor* q, const ttt_tensor* k, const ttt_tensor* v,
+                          const ttt_tensor* eta, const ttt_tensor* W0, int32_t chunk,
+                          int32_t loss, const ttt_tensor* dy, const ttt_tensor* dW_final,
+                          const ttt_tensor* dq, const ttt_tensor* dk, const ttt_tensor* dv,
+                          const ttt_tensor* deta, const ttt_tensor* dW0, void* stream) {
+  if (!q || !k || !v || !eta || !W0 || !dy || !dq || !dk || !dv || !deta || !dW0)
+    return TTT_ERR_NULL;
+  if (chunk < 1) return TTT_ERR_ARG;
+  if (loss != TTT_LOSS_MSE && loss != TTT_LOSS_NEG_DOT) return TTT_ERR_ARG;
+  if (q->ndim != 4 || v->ndim != 4) return TTT_ERR_SHAPE;
+  const int64_t B = q->shape[0], H = q->shape[1], T = q->shape[2], dK = q->shape[3];
+  const int64_t dV = v->shape[3];
+  if (B < 1 || H < 1 || T < 0 || dK < 1 || dV < 1) return TTT_ERR_SHAPE;
+  if (T > kMaxT || B * H > kMaxHeads || !ttt::ttt_linear_bwd_supported((int)dK, (int)dV))
+    return TTT_ERR_UNSUPPORTED;
+  const int32_t dt = q->dtype;
+  if (dt != TTT_F32 && dt != TTT_BF16) return TTT_ERR_DTYPE;
+  ttt_status st;
+  if ((st = check_tokens(q, B, H, T, dK, dt)) != TTT_OK) return st;
+  if ((st = check_tokens(k, B, H, T, dK, dt)) != TTT_OK) return st;
+  if ((st = check_tokens(v, B, H, T, dV, dt)) != TTT_OK) return st;
+  if ((st = check_tokens(dy, B, H, T, dV, dt)) != TTT_OK) return st;
+  if ((st = check_tokens(dq, B, H, T, dK, dt)) != TTT_OK) return st;
+  if ((st = check_tokens(dk, B, H, T, dK, dt)) != TTT_OK) return st;
+  if ((st = check_tokens(dv, B, H, T, dV, dt)) != TTT_OK) return st;
+  auto check_eta = [&](const ttt_tensor* e, bool contig) -> ttt_status {
+    if (e->ndim != 3 || e->shape[0] != B || e->shape[1] != H || e->shape[2] != T)
+      return TTT_ERR_SHAPE;
+    if (e->dtype != TTT_F32) return TTT_ERR_DTYPE;
+    if (!e->data && T > 0) return TTT_ERR_NULL;
+    for (int i = 0; i < 3; ++i)
+      if (e->stride[i] < 0 && T > 0) return TTT_ERR_LAYOUT;
+    if (contig && T > 0 && !contiguous(e)) return TTT_ERR_LAYOUT;
+    if (!aligned16(e->data)) return TTT_ERR_LAYOUT;
+    return TTT_OK;
+  };
+  if ((st = check_eta(eta, false)) != TTT_OK) return st;
+  if ((st = check_eta(deta, true)) != TTT_OK) return st;
+  // W0 and dW0: [H,dk,dv] (shared over the batch) or [B,H,dk,dv], fp32 contiguous
+  auto check_w = [&](const ttt_tensor* w, int64_t* sb) -> ttt_status {
+    if (!w->data) return TTT_ERR_NULL;
+    if (w->dtype != TTT_F32) return TTT_ERR_DTYPE;
+    if (w->ndim == 3) {
+      if (w->shape[0] != H || w->shape[1] != dK || w->shape[2] != dV) return TTT_ERR_SHAPE;
+      *sb = 0;
+    } else if (w->ndim == 4) {
+      if (w->shape[0] != B || w->shape[1] != H || w->shape[2] != dK || w->shape[3] != dV)
+        return TTT_ERR_SHAPE;
+      *sb = H * dK * dV;
+    } else {
+      return TTT_ERR_SHAPE;
+    }
+    if (!contiguous(w) || !aligned16(w->data)) return TTT_ERR_LAYOUT;
+    return TTT_OK;
+  };
+  int64_t w0_sb = 0, dw0_sb = 0;
+  if ((st = check_w(W0, &w0_sb)) != TTT_OK) return st;
+  if ((st = check_w(dW0, &dw0_sb)) != TTT_OK) return st;
+  if (W0->ndim != dW0->ndim) return TTT_ERR_SHAPE;
+  if (dW_final) {
+    if (!dW_final->data) return TTT_ERR_NULL;
+    if (dW_final->dtype != TTT_F32) return TTT_ERR_DTYPE;
+    if (dW_final->ndim != 4 || dW_final->shape[0] != B || dW_final->shape[1] != H ||
+        dW_final->shape[2] != dK || dW_final->shape[3] != dV)
+      return TTT_ERR_SHAPE;
+    if (!contiguous(dW_final) || !aligned16(dW_final->data)) return TTT_ERR_LAYOUT;
+  }
+  const ttt_tensor* ins[] = {q, k, v, eta, W0, dy, dW_final};
+  const ttt_tensor* outs[] = {dq, dk, dv, deta, dW0};
+  for (const ttt_tensor* o : outs) {
+    for (const ttt_tensor* in : ins)
+      if (overlaps(o, in)) return TTT_ERR_ARG;
+    for (const ttt_tensor* o2 : outs)
+      if (o != o2 && overlaps(o, o2)) return TTT_ERR_ARG;
+  }
+
+  ttt::LinearBwdArgs a;
+  a.q = view(q);
+  a.k = view(k);
+  a.v = view(v);
+  a.dy = view(dy);
+  a.eta = {static_cast<const float*>(eta->data), eta->stride[0], eta->stride[1], eta->stride[2]};
+  a.W0 = static_cast<const float*>(W0->data);
+  a.w0_sb = w0_sb;
+  a.dWf = dW_final ? static_cast<const float*>(dW_final->data) : nullptr;
+  a.gq = {dq->data, dq->stride[0], dq->stride[1], dq->stride[2]};
+  a.gk = {dk->data, dk->stride[0], dk->stride[1], dk->stride[2]};
+  a.gv = {dv->data, dv->stride[0], dv->stride[1], dv->stride[2]};
+  a.deta = static_cast<float*>(deta->data);
+  a.dW = nullptr;
+  a.ckpt = nullptr;
+  a.B = (int)B;
+  a.H = (int)H;
+  a.T = (int)T;
+  a.dk = (int)dK;
+  a.dv = (int)dV;
+  a.chunk = chunk;
+  a.loss = loss;
+  a.nchunks = (int)((T + chunk - 1) / chunk);
+  a.status = device_status_ptr();
+  if (!a.status) return TTT_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool shared = W0->ndim == 3;
+  const size_t bytes = ttt::ttt_linear_bwd_workspace(a, shared);
+  void* ws = nullptr;
+  if (bytes && ttt::scratch_alloc(&ws, bytes, s) != cudaSuccess) return TTT_ERR_ALLOC;
+  cudaError_t e = ttt::launch_ttt_linear_bwd(a, dt == TTT_BF16, shared,
+                                             static_cast<float*>(dW0->data), ws, s);
+  if (ws && cudaFreeAsync(ws, s) != cudaSuccess && e == cudaSuccess) e = cudaErrorUnknown;
+  return e == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
+}
+
+}  // extern "C"
+
+namespace {
+
+// Parameter tensor of per-head shape `inner` (1 or 2 dims): [H, inner...] shared
+// over the batch, or [B, H, inner...]; fp32 contiguous. *per_seq = 1 for the latter.
+ttt_status check_param(const ttt_tensor* t, int64_t B, int64_t H, int nin, const int64_t* inner,
+                       int64_t* per_seq) {
+  if (!t->data) return TTT_ERR_NULL;
+  if (t->dtype != TTT_F32) return TTT_ERR_DTYPE;
+  int off;
+  if (t->ndim == nin + 1) {
+    if (t->shape[0] != H) return TTT_ERR_SHAPE;
+    off = 1;
+    *per_seq = 0;
+  } else if (t->ndim == nin + 2) {
+    if (t->shape[0] != B || t->shape[1] != H) return TTT_ERR_SHAPE;
+    off = 2;
+    *per_seq = 1;
+  } else {
+    return TTT_ERR_SHAPE;
+  }
+  for (int i = 0; i < nin; ++i)
+    if (t->shape[off + i] != inner[i]) return TTT_ERR_SHAPE;
+  if (!contiguous(t) || !aligned16(t->data)) return TTT_ERR_LAYOUT;
+  return TTT_OK;
+}
+
+ttt_status check_final_param(const ttt_tensor* t, int64_t B, int64_t H, int nin,
+                             const int64_t* inner) {
+  if (!t) return TTT_OK;
+  int64_t per = 0;
+  ttt_status st = check_param(t, B, H, nin, inner, &per);
+  if (st != TTT_OK) return st;
+  return per ? TTT_OK : TTT_ERR_SHAPE;
+}
+
+}  // namespace
+
+extern "C" {
+
+ttt_status ttt_mlp_fwd(const ttt_tensor* q, const ttt_tensor* k, const ttt_tensor* v,
+                       const ttt_tensor* eta, const ttt_tensor* W1, const ttt_tensor* b1,
+                       const ttt_tensor* W2, const ttt_tensor* b2, int32_t chunk,
+                       const ttt_tensor* out, const ttt_tensor* W1_final,
+                       const ttt_tensor* b1_final, const ttt_tensor* W2_final,
+                       const ttt_tensor* b2_final, void* stream) {
+  if (!q || !k || !v || !eta || !W1 || !b1 || !W2 || !b2 || !out) return TTT_ERR_NULL;
+  if (chunk < 1) return TTT_ERR_ARG;
+  if (q->ndim != 4 || v->ndim != 4 || W1->ndim < 3) return TTT_ERR_SHAPE;
+  const int64_t B = q->shape[0], H = q->shape[1], T = q->shape[2], dK = q->shape[3];
+  const int64_t dV = v->shape[3], dH = W1->shape[W1->ndim - 2];
+  if (B < 1 || H < 1 || T < 0 || dK < 1 || dV < 1 || dH < 1) return TTT_ERR_SHAPE;
+  if (T > kMaxT || B * H > kMaxHeads || !ttt::ttt_mlp_supported((int)dK, (int)dV, (int)dH))
+    return TTT_ERR_UNSUPPORTED;
+  const int32_t dt = q->dtype;
+  if (dt != TTT_F32 && dt != TTT_BF16) return TTT_ERR_DTYPE;
+  ttt_status st;
+  if ((st = check_tokens(q, B, H, T, dK, dt)) != TTT_OK) return st;
+  if ((st = check_tokens(k, B, H, T, dK, dt)) != TTT_OK) return st;
+  if ((st = check_tokens(v, B, H, T, dV, dt)) != TTT_OK) return st;
+  if ((st = check_tokens(out, B, H, T, dV, dt)) != TTT_OK) return st;
+  if (eta->ndim != 3 || eta->shape[0] != B || eta->shape[1] != H || eta->shape[2] != T)
+    return TTT_ERR_SHAPE;
+  if (eta->dtype != TTT_F32) return TTT_ERR_DTYPE;
+  if (!eta->data && T > 0) return TTT_ERR_NULL;
+  for (int i = 0; i < 3; ++i)
+    if (eta->stride[i] < 0) return TTT_ERR_LAYOUT;
+  if (!aligned16(eta->data)) return TTT_ERR_LAYOUT;
+  const int64_t sW1[2] = {dH, dK}, sb1[1] = {dH}, sW2[2] = {dV, dH}, sb2[1] = {dV};
+  const ttt_tensor* P[4] = {W1, b1, W2, b2};
+  const ttt_tensor* F[4] = {W1_final, b1_final, W2_final, b2_final};
+  const int64_t* inner[4] = {sW1, sb1, sW2, sb2};
+  const int nin[4] = {2, 1, 2, 1};
+  int64_t per[4];
+  for (int m = 0; m < 4; ++m) {
+    if ((st = check_param(P[m], B, H, nin[m], inner[m], &per[m])) != TTT_OK) return st;
+    if ((st = check_final_param(F[m], B, H, nin[m], inner[m])) != TTT_OK) return st;
+  }
+  const ttt_tensor* ins[] = {q, k, v, eta, W1, b1, W2, b2};
+  const ttt_tensor* outs[] = {out, W1_final, b1_final, W2_final, b2_final};
+  for (const ttt_tensor* o : outs) {
+    for (const ttt_tensor* in : ins)
+      if (overlaps(o, in)) return TTT_ERR_ARG;
+    for (const ttt_tensor* o2 : outs)
+      if (o != o2 && overlaps(o, o2)) return TTT_ERR_ARG;
+  }
+  ttt::MlpArgs a;
+  a.q = view(q);
+  a.k = view(k);
+  a.v = view(v);
+  a.eta = {static_cast<const float*>(eta->data), eta->stride[0], eta->stride[1], eta->stride[2]};
+  a.W1 = static_cast<const float*>(W1->data);
+  a.b1 = static_cast<const float*>(b1->data);
+  a.W2 = static_cast<const float*>(W2->data);
+  a.b2 = static_cast<const float*>(b2->data);
+  for (int m = 0; m < 4; ++m) a.p_sb[m] = per[m];
+  a.out = {out->data, out->stride[0], out->stride[1], out->stride[2]};
+  float* fin[4];
+  for (int m = 0; m < 4; ++m) fin[m] = F[m] ? static_cast<float*>(F[m]->data) : nullptr;
+  a.W1_final = fin[0];
+  a.b1_final = fin[1];
+  a.W2_final = fin[2];
+  a.b2_final = fin[3];
+  a.B = (int)B;
+  a.H = (int)H;
+  a.T = (int)T;
+  a.dk = (int)dK;
+  a.dv = (int)dV;
+  a.dh = (int)dH;
+  a.chunk = chunk;
+  a.status = device_status_ptr();
+  if (!a.status) return TTT_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t bytes = ttt::ttt_mlp_workspace(a);
+  void* ws = nullptr;
+  if (ttt::scratch_alloc(&ws, bytes, s) != cudaSuccess) return TTT_ERR_ALLOC;
+  a.ws = static_cast<float*>(ws);
+  cudaError_t e = ttt::launch_ttt_mlp(a, dt == TTT_BF16, s);
+  if (cudaFreeAsync(ws, s) != cudaSuccess && e == cudaSuccess) e = cudaErrorUnknown;
+  return e == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
+}
+
+}  // extern "C"
+
+extern "C" {
+
+ttt_status window_attention_fwd(const ttt_tensor* q, const ttt_tensor* k, const ttt_tensor* v,
+                                int32_t window, int32_t accumulate, const ttt_tensor* out,
+                                void* stream) {
+  if (!q || !k || !v || !out) return TTT_ERR_NULL;
+  if (window < 1 || (accumulate != 0 && accumulate != 1)) return TTT_ERR_ARG;
+  if (q->ndim != 4 || v->ndim != 4) return TTT_ERR_SHAPE;
+  const int64_t B = q->shape[0], H = q->shape[1], T = q->shape[2], d = q->shape[3];
+  const int64_t dV = v->shape[3];
+  if (B < 1 || H < 1 || T < 0 || d < 1 || dV < 1) return TTT_ERR_SHAPE;
+  const int32_t dt = q->dtype;
+  if (dt != TTT_F32 && dt != TTT_BF16) return TTT_ERR_DTYPE;
+  ttt_status st;
+  if ((st = check_tokens(q, B, H, T, d, dt)) != TTT_OK) return st;
+  if ((st = check_tokens(k, B, H, T, d, dt)) != TTT_OK) return st;
+  if ((st = check_tokens(v, B, H, T, dV, dt)) != TTT_OK) return st;
+  if ((st = check_tokens(out, B, H, T, dV, dt)) != TTT_OK) return st;
+  if (T > kMaxT || B * H > kMaxHeads || !ttt::window_attn_supported((int)d, (int)dV, dt))
+    return TTT_ERR_UNSUPPORTED;
+  if (overlaps(out, q) || overlaps(out, k) || overlaps(out, v)) return TTT_ERR_ARG;
+  cudaError_t e = ttt::launch_window_attn(view(q), view(k), view(v),
+                                          {out->data, out->stride[0], out->stride[1], out->stride[2]},
+                                          (int)B, (int)H, (int)T, (int)d, window, accumulate,
+                                          static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
+}
+
+ttt_status lact_swiglu_window_fwd(const ttt_tensor* q, const ttt_tensor* k, const ttt_tensor* v,
+                                  const ttt_tensor* eta, const ttt_tensor* W1,
+                                  const ttt_tensor* W2, const ttt_tensor* W3, int32_t chunk,
+                                  int32_t update_rule, int32_t window, const ttt_tensor* out,
+                                  void* stream) {
+  if (!q || !v || !out) return TTT_ERR_NULL;
+  if (window < 1) return TTT_ERR_ARG;
+  if (q->ndim != 4 || v->ndim != 4) return TTT_ERR_SHAPE;
+  if (!ttt::window_attn_supported((int)q->shape[3], (int)v->shape[3], q->dtype))
+    return TTT_ERR_UNSUPPORTED;
+  ttt_status st = lact_swiglu_fwd(q, k, v, eta, W1, W2, W3, chunk, update_rule, 1, out, stream);
+  if (st != TTT_OK) return st;
+  return window_attention_fwd(q, k, v, window, 1, out, stream);
+}
+
+}  // extern "C"
+
+extern "C" {
+
+ttt_status lact_swiglu_fwd_cp(const ttt_tensor* q, const ttt_tensor* k, const ttt_tensor* v,
+                              const ttt_tensor* eta, const ttt_tensor* W1, const ttt_tensor* W2,
+                              const ttt_tensor* W3, int32_t chunk, int32_t update_rule,
+                              int32_t causal, const ttt_tensor* out,
+                              const ttt_tensor* W1_final, const ttt_tensor* W2_final,
+                              const ttt_tensor* W3_final, lact_grad_reduce_fn reduce,
+                              void* reduce_user, void* stream) {
+  ttt::LactArgs a;
+  ttt_status st = ttt::lact_build_args(q, k, v, eta, W1, W2, W3, chunk, update_rule, causal, out,
+                                       W1_final, W2_final, W3_final, &a);
+  if (st != TTT_OK) return st;
+  a.reduce = reduce;
+  a.reduce_user = reduce_user;
+  if ((st = ttt::lact_attach_status(&a)) != TTT_OK) return st;
+  return ttt::lact_forward(a, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -114,4 +114,52 @@ cudaError_t launch_ttt_linear_wy(const LinearArgs& a, cudaStream_t s);
 bool la_tc_supported(const LinearArgs& a);
 cudaError_t launch_la_tc(const LinearArgs& a, cudaStream_t s);
 
+// The library's stream-ordered scratch pool on the current device (null if
+// it cannot be created; callers then use the device's default pool).
+cudaMemPool_t scratch_pool();
+// Stream-ordered scratch from that pool (the failure test hook applies).
+cudaError_t scratch_alloc(void** p, size_t bytes, cudaStream_t s);
+void set_failing_allocs(int n);
+
+bool window_attn_supported(int d, int dv, int dtype);
+cudaError_t launch_window_attn(const TokView& q, const TokView& k, const TokView& v,
+                               const TokViewMut& out, int B, int H, int T, int d, int window,
+                               int accumulate, cudaStream_t s);
+
+// Arguments of the TTT-MLP forward (ttt_mlp_fwd).
+struct MlpArgs {
+  TokView q, k, v;
+  EtaView eta;
+  const float *W1, *b1, *W2, *b2;   // [H or B*H] x ([dh][dk], [dh], [dv][dh], [dv])
+  int64_t p_sb[4];                  // non-zero: one copy per (batch, head)
+  TokViewMut out;
+  float *W1_final, *b1_final, *W2_final, *b2_final;  // [B*H] x ..., each may be null
+  float* ws;                        // ttt_mlp_workspace() bytes
+  int B, H, T, dk, dv, dh, chunk;
+  int* status;
+};
+bool ttt_mlp_supported(int dk, int dv, int dh);
+size_t ttt_mlp_workspace(const MlpArgs& a);
+cudaError_t launch_ttt_mlp(const MlpArgs& a, bool bf16, cudaStream_t s);
+
+// Arguments of the TTT-Linear / inner-product backward (ttt_linear_bwd).
+struct LinearBwdArgs {
+  TokView q, k, v, dy;
+  EtaView eta;
+  const float* W0;
+  int64_t w0_sb;        // 0 when W0 is shared over the batch
+  const float* dWf;     // [B,H,dk,dv] or null
+  TokViewMut gq, gk, gv;     // dL/dq, dL/dk, dL/dv (same element type as q)
+  float* deta;          // [B,H,T] contiguous
+  float* dW;            // [B*H][dk][dv]: dL/dW0 per (batch, head)
+  float* ckpt;          // [B*H][nchunks][dk][dv] chunk-start weights (MSE)
+  int B, H, T, dk, dv, chunk, loss, nchunks;
+  int* status;
+};
+
+bool ttt_linear_bwd_supported(int dk, int dv);
+size_t ttt_linear_bwd_workspace(const LinearBwdArgs& a, bool w0_shared);
+cudaError_t launch_ttt_linear_bwd(LinearBwdArgs a, bool bf16, bool w0_shared, float* dW0, void* ws,
+                                  cudaStream_t s);
+
 }  // namespace ttt

@@ -26,6 +26,7 @@
 // weights keep hi / lo and Aq is plain bf16.
 #include <cooperative_groups.h>
 
+#include <atomic>
 #include <cstdint>
 #include <mutex>
 #include <vector>
@@ -56,6 +57,12 @@ struct RowArgs {
   int Z, H, dk, dv, dh;
   int prep;                // 1: copy inputs and record norms; 0: W -= G then renorm
   int split;
+  // momentum (same row order): M <- beta M + G, then W -= M instead of W -= G
+  int momentum;
+  float beta;
+  float* M[3];             // momentum masters [Z][rows][cols]
+  const float* Min[3];     // initial momentum (prep only; null: zero)
+  int64_t min_sz[3];       // non-zero when Min holds one matrix per (batch, head)
 };
 
 // One warp per (z, row of W1 | W3 | W2).
@@ -84,6 +91,12 @@ __global__ void __launch_bounds__(256) lact_rows_kernel(RowArgs a) {
     src = a.Win[m] + ((int64_t)zin * nrows + r) * len;
   }
   float* rho = a.rho[m] + (int64_t)z * nrows + r;
+  float* M = a.momentum ? a.M[m] + ((int64_t)z * nrows + r) * len : nullptr;
+  const float* msrc = nullptr;
+  if (a.prep && a.momentum && a.Min[m]) {
+    const int zin = a.min_sz[m] ? z : z % a.H;
+    msrc = a.Min[m] + ((int64_t)zin * nrows + r) * len;
+  }
   __nv_bfloat16 *hi, *lo;
   int64_t orow;
   if (m == 2) {
@@ -125,9 +138,18 @@ __global__ void __launch_bounds__(256) lact_rows_kernel(RowArgs a) {
       const int c = 4 * (lane + 32 * i);
       if (a.prep) {
         v[i] = *reinterpret_cast<const float4*>(src + c);
+        if (M)
+          *reinterpret_cast<float4*>(M + c) =
+              msrc ? *reinterpret_cast<const float4*>(msrc + c) : make_float4(0.f, 0.f, 0.f, 0.f);
       } else {
         const float4 w = *reinterpret_cast<const float4*>(W + c);
-        const float4 g = *reinterpret_cast<const float4*>(G + c);
+        float4 g = *reinterpret_cast<const float4*>(G + c);
+        if (M) {  // heavy-ball momentum: the step is beta * M + G
+          const float4 mo = *reinterpret_cast<const float4*>(M + c);
+          g = make_float4(fmaf(a.beta, mo.x, g.x), fmaf(a.beta, mo.y, g.y), fmaf(a.beta, mo.z, g.z),
+                          fmaf(a.beta, mo.w, g.w));
+          *reinterpret_cast<float4*>(M + c) = g;
+        }
         v[i] = make_float4(w.x - g.x, w.y - g.y, w.z - g.z, w.w - g.w);
       }
       ss += v[i].x * v[i].x + v[i].y * v[i].y + v[i].z * v[i].z + v[i].w * v[i].w;
@@ -163,7 +185,17 @@ __global__ void __launch_bounds__(256) lact_rows_kernel(RowArgs a) {
   if (per > 2) return;
   for (int i = 0; i < per; ++i) {
     const int c = lane + 32 * i;
-    v[i] = a.prep ? src[c] : W[c] - G[c];
+    if (a.prep) {
+      v[i] = src[c];
+      if (M) M[c] = msrc ? msrc[c] : 0.f;
+    } else {
+      float g = G[c];
+      if (M) {
+        g = fmaf(a.beta, M[c], g);
+        M[c] = g;
+      }
+      v[i] = W[c] - g;
+    }
     ss += v[i] * v[i];
   }
   float s;
@@ -706,7 +738,7 @@ bool grad_map(CUtensorMap* m, const float* base, int Z, int rows, int cols) {
 }
 
 struct Scratch {
-  float *Wm[3], *rho[3], *G[3], *ns;
+  float *Wm[3], *rho[3], *G[3], *ns, *M[3];
   __nv_bfloat16 *w13[2], *w2[2];          // hi, lo
   __nv_bfloat16 *aq[2], *ak[2], *dh1[2], *dh3[2];
   int64_t ns_stride;
@@ -862,6 +894,7 @@ Sizes lact_sizes(const LactArgs& a) {
   // Newton-Schulz scratch: only the general-shape kernel needs it (the
   // tensor-core kernel for 128 x 512 gradients keeps everything on chip)
   if (z.split && !ns_on_chip(a)) z.f32n += (size_t)z.Z * 3 * z.ns_stride;
+  if (a.momentum) z.f32n += (size_t)z.Z * (z.nW[0] + z.nW[1] + z.nW[2]);
   z.bfn = (size_t)z.Z * (2 * dh * dk + dv * dh) * (z.split ? 2 : 1);
   z.bfn += (size_t)z.Z * z.chunk * dh * 4 * (z.split ? 2 : 1);
   z.bytes = z.f32n * 4 + z.bfn * 2 + 4096;
@@ -905,17 +938,30 @@ cudaMemPool_t scratch_pool() {
   return pools[dev];
 }
 
+namespace {
+std::atomic<int> g_fail_allocs{0};
+}  // namespace
+
+void set_failing_allocs(int n) { g_fail_allocs.store(n < 0 ? 0 : n); }
+
+cudaError_t scratch_alloc(void** p, size_t bytes, cudaStream_t s) {
+  *p = nullptr;
+  // test hook: the next n allocations fail as if the device were out of memory
+  int n = g_fail_allocs.load();
+  while (n > 0 && !g_fail_allocs.compare_exchange_weak(n, n - 1)) {
+  }
+  if (n > 0) return cudaErrorMemoryAllocation;
+  cudaMemPool_t pool = scratch_pool();
+  const cudaError_t e = pool ? cudaMallocFromPoolAsync(p, bytes, pool, s) : cudaMallocAsync(p, bytes, s);
+  if (e != cudaSuccess) cudaGetLastError();
+  return e;
+}
+
 ttt_status lact_forward(const LactArgs& a, cudaStream_t s) {
   const Sizes z = lact_sizes(a);
   if (!z.ok) return TTT_ERR_UNSUPPORTED;
   void* base = nullptr;
-  cudaMemPool_t pool = scratch_pool();
-  const cudaError_t ae = pool ? cudaMallocFromPoolAsync(&base, z.bytes, pool, s)
-                              : cudaMallocAsync(&base, z.bytes, s);
-  if (ae != cudaSuccess) {
-    cudaGetLastError();
-    return TTT_ERR_ALLOC;
-  }
+  if (scratch_alloc(&base, z.bytes, s) != cudaSuccess) return TTT_ERR_ALLOC;
   ttt_status r = lact_run(a, s, base, z.bytes);
   if (cudaFreeAsync(base, s) != cudaSuccess && r == TTT_OK) r = TTT_ERR_CUDA;
   return r;
@@ -933,18 +979,28 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
   const int64_t ns_stride = zz.ns_stride;
   Scratch sc;
   {
+    // masters, then the three gradients back to back (one buffer for the
+    // context-parallel exchange), then the row norms
     float* f = static_cast<float*>(base);
     for (int m = 0; m < 3; ++m) {
       sc.Wm[m] = f;
       f += Z * nW[m];
+    }
+    for (int m = 0; m < 3; ++m) {
       sc.G[m] = f;
       f += Z * nW[m];
+    }
+    for (int m = 0; m < 3; ++m) {
       sc.rho[m] = f;
       f += Z * nrows[m];
     }
     const bool ns_scratch = split && !ns_on_chip(a);
     sc.ns = ns_scratch ? f : nullptr;
     if (ns_scratch) f += (size_t)Z * 3 * ns_stride;
+    for (int m = 0; m < 3; ++m) {
+      sc.M[m] = a.momentum ? f : nullptr;
+      if (a.momentum) f += Z * nW[m];
+    }
     uintptr_t up = (reinterpret_cast<uintptr_t>(f) + 255) & ~uintptr_t(255);
     __nv_bfloat16* b = reinterpret_cast<__nv_bfloat16*>(up);
     auto take = [&](size_t n) {
@@ -995,6 +1051,17 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
   ra.dv = dv;
   ra.dh = dh;
   ra.split = split;
+  // momentum: LactArgs order (W1, W2, W3) -> row order (W1, W3, W2)
+  ra.momentum = a.momentum;
+  ra.beta = a.beta;
+  {
+    const int order[3] = {0, 2, 1};
+    for (int m = 0; m < 3; ++m) {
+      ra.M[m] = sc.M[m];
+      ra.Min[m] = a.momentum ? a.M0[order[m]] : nullptr;
+      ra.min_sz[m] = a.momentum ? a.m0_sb[order[m]] : 0;
+    }
+  }
   const int row_warps = Z * (2 * dh + dv);
   const int row_blocks = (row_warps * 32 + 255) / 256;
   ra.prep = 1;
@@ -1198,6 +1265,13 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
       add_grads(P);
       run(P);
     }
+    // context parallelism: sum the gradients over the ranks that hold the
+    // other token shards of this chunk
+    if (a.reduce && result == TTT_OK) {
+      if (a.reduce(sc.G[0], (size_t)Z * (nW[0] + nW[1] + nW[2]), s, a.reduce_user) != 0)
+        result = TTT_ERR_CUDA;
+      if (result != TTT_OK) break;
+    }
     // L3 / L4: Muon orthogonalisation, update and row renormalisation
     if (split) {
       if (ns_tc) {
@@ -1227,6 +1301,12 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
   for (int m = 0; m < 3 && result == TTT_OK; ++m) {
     if (!finals[m]) continue;
     copy_kernel<<<148, 256, 0, s>>>(finals[m], sc.Wm[m], Z * nW[m]);
+    check(cudaGetLastError());
+  }
+  float* mfinals[3] = {a.M_final[0], a.M_final[2], a.M_final[1]};
+  for (int m = 0; m < 3 && result == TTT_OK && a.momentum; ++m) {
+    if (!mfinals[m]) continue;
+    copy_kernel<<<148, 256, 0, s>>>(mfinals[m], sc.M[m], Z * nW[m]);
     check(cudaGetLastError());
   }
   return result;

@@ -14,6 +14,17 @@ struct LactArgs {
   float *W1_final, *W2_final, *W3_final;  // each may be null
   int B, H, T, dk, dv, dh, chunk, update_rule, causal, dtype;
   int* status;
+  // Momentum update (lact_swiglu_fwd_momentum): M <- beta M + G, W <- W - M.
+  int momentum;                // 0: GD / Muon as update_rule says
+  float beta;
+  const float* M0[3];          // initial momentum of W1, W2, W3 (null: zero)
+  int64_t m0_sb[3];            // batch stride of M0 (0: shared over batch)
+  float* M_final[3];           // each may be null
+  // Context parallelism (lact_swiglu_fwd_cp): called once per chunk, after
+  // the chunk's gradients are complete and before they are used, with the
+  // contiguous fp32 gradient buffer (G1 | G3 | G2 of every (batch, head)).
+  lact_grad_reduce_fn reduce;  // null: no exchange
+  void* reduce_user;
 };
 
 // Enqueues the whole layer forward on `s`, taking its scratch from the

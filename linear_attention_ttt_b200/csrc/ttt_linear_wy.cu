@@ -22,14 +22,20 @@
 // the chunk open at each group start starts there or earlier: chunk 16, 32 or
 // a multiple of 64.
 //
-// Layout on the chip: one CTA per (batch, head). Consumer warp w owns dv rows
-// [16w, 16w+16) of W^T as m16n8k16 accumulator fragments (transposed form:
-// E^T, Y^T and W^T have dv as their row dimension). The 16 token-block
-// products of the group (10 blocks of Q K^T, 6 of K K^T) are split over the
-// four warps and exchanged through shared memory already in the B-fragment
-// order every lane reads. The output tile of the group is assembled in shared
-// memory and written as 128-byte rows. A producer warp streams 64-token Q, K, V
-// tiles with TMA into a 4-stage ring (bounded waits).
+// Layout on the chip: one CTA per (batch, head) with eight consumer warps in
+// two roles. Chain warp w (0-3) owns dv rows [16w, 16w+16) of W^T as
+// m16n8k16 accumulator fragments (transposed form: E^T, Y^T and W^T have dv
+// as their row dimension) and runs the W-dependent chain of a group: E0, the
+// forward substitution and the W update. Output warp w + 4 owns the same dv
+// rows and forms Y^T from the group-start weights and the chain warp's errors,
+// which it receives through shared memory at two pairwise named barriers.
+// Two warps per sub-partition let the MMA chains of one hide the latencies of
+// the other. The 16 token-block products of the group (10 blocks of Q K^T, 6
+// of K K^T) are split over all eight warps and exchanged through shared
+// memory already in the B-fragment order every lane reads. The output tile of
+// the group is assembled in shared memory and written as 128-byte rows. A
+// producer warp streams 64-token Q, K, V tiles with TMA into a 4-stage ring
+// (bounded waits).
 #include "common.cuh"
 #include "tma.cuh"
 
@@ -40,8 +46,14 @@ constexpr int D = 64;
 constexpr int kG = 64;        // tokens per group
 constexpr int kSub = 4;       // 16-token sub-blocks per group
 constexpr int kStages = 4;
-constexpr int kWarps = 4;     // consumer warps, 16 dv rows each
+constexpr int kRowBlocks = 4;  // 16 dv rows each
+constexpr int kWarps = 2 * kRowBlocks;  // consumer warps: 4 chain + 4 output
 constexpr int kThreads = (kWarps + 1) * 32;
+// Named barriers (0 is __syncthreads): all consumers; per row block, the
+// chain warp's errors and its next group-start weights for the output warp.
+constexpr int kBarConsumers = 1;
+constexpr int kBarErr = 2;     // + row block
+constexpr int kBarW = 6;       // + row block
 constexpr int kTile = kG * D * 2;  // one [64 x 64] bf16 tile, 8 KB
 constexpr int kProducts = 16;      // 10 Q K^T blocks + 6 K K^T blocks
 
@@ -77,6 +89,8 @@ struct Smem {
   alignas(1024) uint8_t v[kStages][kTile];
   alignas(1024) uint8_t ostage[2][kTile];            // output tile [64 t][64 dv]
   uint32_t frag[2][kProducts][2][2][32];             // [buf][product][n-tile][b0|b1][lane]
+  uint32_t wy[kRowBlocks][4][4][32];                 // group-start W^T (bf16 A fragments)
+  uint32_t ae[2][kRowBlocks][kSub][4][32];           // errors E^T (bf16 A fragments)
   float eta[kStages][kG];
   uint64_t full[kStages], empty[kStages];
   int abort;
@@ -189,19 +203,17 @@ __global__ void __launch_bounds__(kThreads, 1) ttt_linear_wy_kernel(const __grid
 
   // ---------------- consumers ----------------
   const int g = lane >> 2, c4 = lane & 3, mi = lane >> 3, rr = lane & 7;
-  const int r0 = warp * 16;  // this warp's dv rows
-  const float* W0 = p.W0 + b * p.w0_sb + (int64_t)h * D * D;
+  const bool chain = warp < kRowBlocks;
+  const int rb = warp & (kRowBlocks - 1);
+  const int r0 = rb * 16;  // this warp's dv rows
+  const int tid = threadIdx.x;
+  auto bar_consumers = [] { asm volatile("bar.sync %0, %1;" ::"n"(kBarConsumers), "n"(kWarps * 32) : "memory"); };
+  auto pair_arrive = [](int id) { asm volatile("bar.arrive %0, 64;" ::"r"(id) : "memory"); };
+  auto pair_sync = [](int id) { asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory"); };
 
-  // W_cur^T fragments: Wc[j] covers dv rows r0+{g, g+8}, dk columns 8j+2c4+{0,1}.
+  // W_cur^T fragments (chain warps): Wc[j] covers dv rows r0+{g, g+8}, dk
+  // columns 8j+2c4+{0,1}.
   float Wc[8][4];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int c = 8 * j + 2 * c4;
-    Wc[j][0] = W0[(int64_t)c * D + r0 + g];
-    Wc[j][1] = W0[(int64_t)(c + 1) * D + r0 + g];
-    Wc[j][2] = W0[(int64_t)c * D + r0 + g + 8];
-    Wc[j][3] = W0[(int64_t)(c + 1) * D + r0 + g + 8];
-  }
   // Wy: W_g^T as bf16 A fragments per dk block; Ws: start weights of the open chunk.
   uint32_t Wy[4][4], Ws[4][4];
   auto pack_cur = [&]() {
@@ -219,18 +231,37 @@ __global__ void __launch_bounds__(kThreads, 1) ttt_linear_wy_kernel(const __grid
 #pragma unroll
       for (int u = 0; u < 4; ++u) Ws[kb][u] = Wy[kb][u];
   };
-  pack_cur();
-  start_chunk();
+  auto publish_w = [&]() {  // chain warp -> output warp: the next group-start weights
+#pragma unroll
+    for (int kb = 0; kb < 4; ++kb)
+#pragma unroll
+      for (int u = 0; u < 4; ++u) sm.wy[rb][kb][u][lane] = Wy[kb][u];
+    pair_arrive(kBarW + rb);
+  };
+  if (chain) {
+    const float* W0 = p.W0 + b * p.w0_sb + (int64_t)h * D * D;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int c = 8 * j + 2 * c4;
+      Wc[j][0] = W0[(int64_t)c * D + r0 + g];
+      Wc[j][1] = W0[(int64_t)(c + 1) * D + r0 + g];
+      Wc[j][2] = W0[(int64_t)c * D + r0 + g + 8];
+      Wc[j][3] = W0[(int64_t)(c + 1) * D + r0 + g + 8];
+    }
+    pack_cur();
+    start_chunk();
+    if (ngroups > 0) publish_w();
+  }
 
   __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(p.out.p) + b * p.out.sb + h * p.out.sh;
   // rows of the previous group's staged output: every consumer thread stores 16 bytes
-  // of 4 rows after the next barrier
+  // of 2 rows after the next barrier
   auto store_rows = [&](int gi) {
     const uint8_t* os = sm.ostage[gi & 1];
-    const int tid = threadIdx.x, cch = tid & 7;
+    const int cch = tid & 7;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int t = (tid >> 3) + 16 * i;
+    for (int i = 0; i < 2; ++i) {
+      const int t = (tid >> 3) + 32 * i;
       if (gi * kG + t < p.T)
         *reinterpret_cast<uint4*>(outp + (int64_t)(gi * kG + t) * p.out.st + cch * 8) =
             *reinterpret_cast<const uint4*>(os + t * 128 + ((cch ^ (t & 7)) << 4));
@@ -241,15 +272,18 @@ __global__ void __launch_bounds__(kThreads, 1) ttt_linear_wy_kernel(const __grid
     const int st = gi % kStages, fb = gi & 1;
     const int g0 = gi * kG;
     const bool ok = mbar_wait(&sm.full[st], (gi / kStages) & 1, p.status);
-    if (!ok) *reinterpret_cast<volatile int*>(&sm.abort) = 1;
+    // A timed-out wait ends every consumer warp at the barrier of this group:
+    // the first failing group is recorded, and a warp still reading the flag
+    // of an earlier group does not see a later group's failure.
+    if (!ok) atomicCAS(&sm.abort, 0, gi + 1);
     const uint32_t qa = smem_u32(sm.q[st]), ka = smem_u32(sm.k[st]);
     const uint8_t* vb = sm.v[st];
     const float* et = sm.eta[st];
 
-    // 1) this warp's four token-block products, packed in consumer B order
+    // 1) this warp's two token-block products, packed in consumer B order
 #pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
-      const int pi = 4 * warp + jj;
+    for (int jj = 0; jj < 2; ++jj) {
+      const int pi = 2 * warp + jj;
       const int code = prod_of(pi);
       const int kind = code >> 4, c = (code >> 2) & 3, cp = code & 3;
       float X[2][4] = {};
@@ -282,112 +316,152 @@ __global__ void __launch_bounds__(kThreads, 1) ttt_linear_wy_kernel(const __grid
           sm.frag[fb][pi][nn][bb][lane] = pack_bf16(X[bb][2 * nn], X[bb][2 * nn + 1]);
     }
 
-    // 2) E0^T = W_s^T K^T - V^T and Y0^T = W_g^T Q^T for the four sub-blocks
-    float E[kSub][2][4], Y[kSub][2][4];
+    if (chain) {
+      // 2c) E0^T = W_s^T K^T - V^T for the four sub-blocks
+      float E[kSub][2][4];
 #pragma unroll
-    for (int c = 0; c < kSub; ++c) {
+      for (int c = 0; c < kSub; ++c) {
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        const int t = 16 * c + 8 * nt + 2 * c4;
-        auto vv = [&](int tt, int r) {
-          return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(vb + sw(tt, r)));
-        };
-        E[c][nt][0] = -vv(t, r0 + g);
-        E[c][nt][1] = -vv(t + 1, r0 + g);
-        E[c][nt][2] = -vv(t, r0 + g + 8);
-        E[c][nt][3] = -vv(t + 1, r0 + g + 8);
+        for (int nt = 0; nt < 2; ++nt) {
+          const int t = 16 * c + 8 * nt + 2 * c4;
+          auto vv = [&](int tt, int r) {
+            return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(vb + sw(tt, r)));
+          };
+          E[c][nt][0] = -vv(t, r0 + g);
+          E[c][nt][1] = -vv(t + 1, r0 + g);
+          E[c][nt][2] = -vv(t, r0 + g + 8);
+          E[c][nt][3] = -vv(t + 1, r0 + g + 8);
+        }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) Y[c][nt][u] = 0.f;
+        for (int kb = 0; kb < 4; ++kb) {
+          uint32_t bk[4];
+          ldsm_x4(bk, ka + sw(16 * c + 8 * (mi >> 1) + rr, 16 * kb + 8 * (mi & 1)));
+          mma16816(E[c][0], Ws[kb], bk[0], bk[1]);
+          mma16816(E[c][1], Ws[kb], bk[2], bk[3]);
+        }
       }
-#pragma unroll
-      for (int kb = 0; kb < 4; ++kb) {
-        uint32_t bk[4], bq[4];
-        ldsm_x4(bk, ka + sw(16 * c + 8 * (mi >> 1) + rr, 16 * kb + 8 * (mi & 1)));
-        ldsm_x4(bq, qa + sw(16 * c + 8 * (mi >> 1) + rr, 16 * kb + 8 * (mi & 1)));
-        mma16816(E[c][0], Ws[kb], bk[0], bk[1]);
-        mma16816(E[c][1], Ws[kb], bk[2], bk[3]);
-        mma16816(Y[c][0], Wy[kb], bq[0], bq[1]);
-        mma16816(Y[c][1], Wy[kb], bq[2], bq[3]);
+
+      // 3c) the products of all warps are visible; the previous group's
+      //     output tile is complete (it is stored now)
+      bar_consumers();
+      {
+        const int ab = *reinterpret_cast<volatile int*>(&sm.abort);
+        if (ab != 0 && ab <= gi + 1) return;
       }
+      if (gi > 0) store_rows(gi - 1);
+
+      // 4c) forward substitution: E_c -= sum over earlier sub-blocks of other
+      //     chunks of (-N E_c')^T (K_c' K_c^T); As[c] = (-N_c E_c)^T as A fragments
+      int chunk_id[kSub];
+#pragma unroll
+      for (int c = 0; c < kSub; ++c) chunk_id[c] = (g0 + 16 * c) / p.chunk;
+      uint32_t As[kSub][4];
+#pragma unroll
+      for (int c = 0; c < kSub; ++c) {
+#pragma unroll
+        for (int cp = 0; cp < c; ++cp) {
+          if (chunk_id[cp] == chunk_id[c]) continue;
+          const uint32_t* f = &sm.frag[fb][m_index(c, cp)][0][0][0];
+          mma16816(E[c][0], As[cp], f[0 * 64 + 0 * 32 + lane], f[0 * 64 + 1 * 32 + lane]);
+          mma16816(E[c][1], As[cp], f[1 * 64 + 0 * 32 + lane], f[1 * 64 + 1 * 32 + lane]);
+        }
+        const float e0 = -et[16 * c + 2 * c4], e1 = -et[16 * c + 2 * c4 + 1];
+        const float e8 = -et[16 * c + 8 + 2 * c4], e9 = -et[16 * c + 9 + 2 * c4];
+        As[c][0] = pack_bf16(e0 * E[c][0][0], e1 * E[c][0][1]);
+        As[c][1] = pack_bf16(e0 * E[c][0][2], e1 * E[c][0][3]);
+        As[c][2] = pack_bf16(e8 * E[c][1][0], e9 * E[c][1][1]);
+        As[c][3] = pack_bf16(e8 * E[c][1][2], e9 * E[c][1][3]);
+        uint32_t* ae = &sm.ae[fb][rb][c][0][0];
+        ae[0 * 32 + lane] = pack_bf16(E[c][0][0], E[c][0][1]);
+        ae[1 * 32 + lane] = pack_bf16(E[c][0][2], E[c][0][3]);
+        ae[2 * 32 + lane] = pack_bf16(E[c][1][0], E[c][1][1]);
+        ae[3 * 32 + lane] = pack_bf16(E[c][1][2], E[c][1][3]);
+      }
+      pair_arrive(kBarErr + rb);  // errors of this group -> output warp
+
+      // 5c) W_g^T += sum_c (-N_c E_c)^T K_c
+#pragma unroll
+      for (int c = 0; c < kSub; ++c)
+#pragma unroll
+        for (int jn = 0; jn < 8; jn += 2) {
+          uint32_t r[4];
+          ldsm_x4_t(r, ka + sw(16 * c + rr + 8 * (mi & 1), 8 * (jn + (mi >> 1))));
+          mma16816(Wc[jn], As[c], r[0], r[1]);
+          mma16816(Wc[jn + 1], As[c], r[2], r[3]);
+        }
+      __syncwarp();
+      if (ok && lane == 0) mbar_arrive(&sm.empty[st]);  // this warp is done with the stage
+      pack_cur();
+      if ((g0 + kG) % p.chunk == 0) start_chunk();
+      if (gi + 1 < ngroups) publish_w();
+    } else {
+      // 2y) Y0^T = W_g^T Q^T with the group-start weights from the chain warp
+      pair_sync(kBarW + rb);
+#pragma unroll
+      for (int kb = 0; kb < 4; ++kb)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) Wy[kb][u] = sm.wy[rb][kb][u][lane];
+      float Y[kSub][2][4];
+#pragma unroll
+      for (int c = 0; c < kSub; ++c) {
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int u = 0; u < 4; ++u) Y[c][nt][u] = 0.f;
+#pragma unroll
+        for (int kb = 0; kb < 4; ++kb) {
+          uint32_t bq[4];
+          ldsm_x4(bq, qa + sw(16 * c + 8 * (mi >> 1) + rr, 16 * kb + 8 * (mi & 1)));
+          mma16816(Y[c][0], Wy[kb], bq[0], bq[1]);
+          mma16816(Y[c][1], Wy[kb], bq[2], bq[3]);
+        }
+      }
+      __syncwarp();
+      if (ok && lane == 0) mbar_arrive(&sm.empty[st]);  // Q of this stage is consumed
+
+      // 3y) see 3c
+      bar_consumers();
+      {
+        const int ab = *reinterpret_cast<volatile int*>(&sm.abort);
+        if (ab != 0 && ab <= gi + 1) return;
+      }
+      if (gi > 0) store_rows(gi - 1);
+
+      // 4y) Y^T_c += sum_{c' <= c} E_c'^T P_{c,c'}^T with the chain warp's errors
+      pair_sync(kBarErr + rb);
+      uint32_t Ae[kSub][4];
+#pragma unroll
+      for (int c = 0; c < kSub; ++c)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) Ae[c][u] = sm.ae[fb][rb][c][u][lane];
+#pragma unroll
+      for (int c = 0; c < kSub; ++c)
+#pragma unroll
+        for (int cp = 0; cp <= c; ++cp) {
+          const uint32_t* f = &sm.frag[fb][s_index(c, cp)][0][0][0];
+          mma16816(Y[c][0], Ae[cp], f[0 * 64 + 0 * 32 + lane], f[0 * 64 + 1 * 32 + lane]);
+          mma16816(Y[c][1], Ae[cp], f[1 * 64 + 0 * 32 + lane], f[1 * 64 + 1 * 32 + lane]);
+        }
+
+      // 5y) Y^T -> staged [t][dv] bf16 tile
+      uint8_t* os = sm.ostage[fb];
+#pragma unroll
+      for (int c = 0; c < kSub; ++c)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          const int t = 16 * c + 8 * nt + 2 * c4;
+          *reinterpret_cast<__nv_bfloat16*>(os + sw(t, r0 + g)) = __float2bfloat16_rn(Y[c][nt][0]);
+          *reinterpret_cast<__nv_bfloat16*>(os + sw(t + 1, r0 + g)) = __float2bfloat16_rn(Y[c][nt][1]);
+          *reinterpret_cast<__nv_bfloat16*>(os + sw(t, r0 + g + 8)) = __float2bfloat16_rn(Y[c][nt][2]);
+          *reinterpret_cast<__nv_bfloat16*>(os + sw(t + 1, r0 + g + 8)) =
+              __float2bfloat16_rn(Y[c][nt][3]);
+        }
     }
-
-    // 3) the products of all warps are visible; the previous group's output
-    //    tile is complete (it is stored now)
-    asm volatile("bar.sync 1, %0;" ::"n"(kWarps * 32) : "memory");
-    if (*reinterpret_cast<volatile int*>(&sm.abort)) return;
-    if (gi > 0) store_rows(gi - 1);
-
-    // 4) forward substitution: E_c -= sum over earlier sub-blocks of other chunks
-    //    of (-N E_c')^T (K_c' K_c^T); As[c] = (-N_c E_c)^T as A fragments
-    int chunk_id[kSub];
-#pragma unroll
-    for (int c = 0; c < kSub; ++c) chunk_id[c] = (g0 + 16 * c) / p.chunk;
-    uint32_t As[kSub][4], Ae[kSub][4];
-#pragma unroll
-    for (int c = 0; c < kSub; ++c) {
-#pragma unroll
-      for (int cp = 0; cp < c; ++cp) {
-        if (chunk_id[cp] == chunk_id[c]) continue;
-        const uint32_t* f = &sm.frag[fb][m_index(c, cp)][0][0][0];
-        mma16816(E[c][0], As[cp], f[0 * 64 + 0 * 32 + lane], f[0 * 64 + 1 * 32 + lane]);
-        mma16816(E[c][1], As[cp], f[1 * 64 + 0 * 32 + lane], f[1 * 64 + 1 * 32 + lane]);
-      }
-      const float e0 = -et[16 * c + 2 * c4], e1 = -et[16 * c + 2 * c4 + 1];
-      const float e8 = -et[16 * c + 8 + 2 * c4], e9 = -et[16 * c + 9 + 2 * c4];
-      As[c][0] = pack_bf16(e0 * E[c][0][0], e1 * E[c][0][1]);
-      As[c][1] = pack_bf16(e0 * E[c][0][2], e1 * E[c][0][3]);
-      As[c][2] = pack_bf16(e8 * E[c][1][0], e9 * E[c][1][1]);
-      As[c][3] = pack_bf16(e8 * E[c][1][2], e9 * E[c][1][3]);
-      Ae[c][0] = pack_bf16(E[c][0][0], E[c][0][1]);
-      Ae[c][1] = pack_bf16(E[c][0][2], E[c][0][3]);
-      Ae[c][2] = pack_bf16(E[c][1][0], E[c][1][1]);
-      Ae[c][3] = pack_bf16(E[c][1][2], E[c][1][3]);
-    }
-
-    // 5) Y^T_c += sum_{c' <= c} E_c'^T P_{c,c'}^T
-#pragma unroll
-    for (int c = 0; c < kSub; ++c)
-#pragma unroll
-      for (int cp = 0; cp <= c; ++cp) {
-        const uint32_t* f = &sm.frag[fb][s_index(c, cp)][0][0][0];
-        mma16816(Y[c][0], Ae[cp], f[0 * 64 + 0 * 32 + lane], f[0 * 64 + 1 * 32 + lane]);
-        mma16816(Y[c][1], Ae[cp], f[1 * 64 + 0 * 32 + lane], f[1 * 64 + 1 * 32 + lane]);
-      }
-
-    // 6) W_g^T += sum_c (-N_c E_c)^T K_c
-#pragma unroll
-    for (int c = 0; c < kSub; ++c)
-#pragma unroll
-      for (int jn = 0; jn < 8; jn += 2) {
-        uint32_t r[4];
-        ldsm_x4_t(r, ka + sw(16 * c + rr + 8 * (mi & 1), 8 * (jn + (mi >> 1))));
-        mma16816(Wc[jn], As[c], r[0], r[1]);
-        mma16816(Wc[jn + 1], As[c], r[2], r[3]);
-      }
-    __syncwarp();
-    if (ok && lane == 0) mbar_arrive(&sm.empty[st]);  // this warp is done with the stage
-
-    // 7) Y^T -> staged [t][dv] bf16 tile
-    uint8_t* os = sm.ostage[fb];
-#pragma unroll
-    for (int c = 0; c < kSub; ++c)
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        const int t = 16 * c + 8 * nt + 2 * c4;
-        *reinterpret_cast<__nv_bfloat16*>(os + sw(t, r0 + g)) = __float2bfloat16_rn(Y[c][nt][0]);
-        *reinterpret_cast<__nv_bfloat16*>(os + sw(t + 1, r0 + g)) = __float2bfloat16_rn(Y[c][nt][1]);
-        *reinterpret_cast<__nv_bfloat16*>(os + sw(t, r0 + g + 8)) = __float2bfloat16_rn(Y[c][nt][2]);
-        *reinterpret_cast<__nv_bfloat16*>(os + sw(t + 1, r0 + g + 8)) =
-            __float2bfloat16_rn(Y[c][nt][3]);
-      }
-
-    pack_cur();
-    if ((g0 + kG) % p.chunk == 0) start_chunk();
   }
-  asm volatile("bar.sync 1, %0;" ::"n"(kWarps * 32) : "memory");
+  bar_consumers();
   if (ngroups > 0) store_rows(ngroups - 1);
 
-  if (p.W_final) {
+  if (chain && p.W_final) {
     float* Wf = p.W_final + (int64_t)bh * D * D;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {

@@ -1,0 +1,234 @@
+// TTT-MLP forward: a two-layer ReLU MLP fast weight under the mini-batch GD
+// rule ("Test-Time Training (TTT)" summary, sections "TTT-MLP" and "병렬화:
+// Mini-batch Gradient Descent").
+//
+// f(x) = W2 ReLU(W1 x + b1) + b2 with W1 [dh][dk], b1 [dh], W2 [dv][dh],
+// b2 [dv]; per-token loss 1/2 ||f(k) - v||^2. In a chunk with start
+// parameters P_s every gradient is taken at P_s, and token t sees
+// P_t = P_s - sum_{i<=t} eta_i grad_i(P_s). For key token i, with
+// h_i = W1 k_i + b1, a_i = ReLU(h_i), r_i = W2 a_i + b2 - v_i and
+// g_i = (W2^T r_i) [h_i > 0] (ReLU derivative 0 at 0), the gradient is
+// (g_i k_i^T, g_i, r_i a_i^T, r_i). So for a query token t:
+//   z_t = W1_t q_t + b1_t = W1_s q_t + b1_s - sum_{i<=t} eta_i (q_t . k_i + 1) g_i
+//   y_t = W2_t a'_t + b2_t = W2_s a'_t + b2_s - sum_{i<=t} eta_i (a'_t . a_i + 1) r_i,
+// with a'_t = ReLU(z_t): the dual (attention-like) form of the chunk.
+//
+// Layout: one CTA of 256 threads per (batch, head), fp32 arithmetic on the
+// CUDA cores. A chunk is walked in blocks of 16 tokens; the parameters live in
+// an fp32 workspace (L2-resident) as the chunk-start copy P_s, used for the
+// keys' h, a, r, g, and the running copy, which already holds the updates of
+// the chunk's earlier blocks and serves the queries.
+#include "common.cuh"
+
+namespace ttt {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kTB = 16;
+
+template <typename T>
+__device__ __forceinline__ float ldt(const TokView& v, int b, int h, int64_t t, int c) {
+  return to_f32((static_cast<const T*>(v.p) + b * v.sb + h * v.sh + t * v.st)[c]);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) ttt_mlp_kernel(MlpArgs a) {
+  extern __shared__ float smem[];
+  const int dk = a.dk, dv = a.dv, dh = a.dh;
+  const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
+  const int tid = threadIdx.x;
+  const int64_t nP = (int64_t)dh * dk + dh + (int64_t)dv * dh + dv;
+
+  // workspace: start and running copies of (W1, b1, W2, b2)
+  float* ps = a.ws + (int64_t)bh * 2 * nP;
+  float* sW1 = ps;
+  float* sb1 = sW1 + (int64_t)dh * dk;
+  float* sW2 = sb1 + dh;
+  float* sb2 = sW2 + (int64_t)dv * dh;
+  float* rW1 = ps + nP;
+  float* rb1 = rW1 + (int64_t)dh * dk;
+  float* rW2 = rb1 + dh;
+  float* rb2 = rW2 + (int64_t)dv * dh;
+
+  float* Qs = smem;              // [16][dk]
+  float* Ks = Qs + kTB * dk;     // [16][dk]
+  float* Vs = Ks + kTB * dk;     // [16][dv]  v, then r
+  float* Hs = Vs + kTB * dv;     // [16][dh]  h, then a = ReLU(h)
+  float* Gs = Hs + kTB * dh;     // [16][dh]  g
+  float* Zs = Gs + kTB * dh;     // [16][dh]  z, then a' = ReLU(z)
+  float* Hm = Zs + kTB * dh;     // [16][dh]  1 where h > 0
+  float* S1 = Hm + kTB * dh;     // [16][16]
+  float* S2 = S1 + kTB * kTB;    // [16][16]
+  float* et = S2 + kTB * kTB;    // [16]
+
+  // initial parameters into both copies
+  {
+    const float* src[4] = {a.W1 + (int64_t)(a.p_sb[0] ? bh : h) * dh * dk,
+                           a.b1 + (int64_t)(a.p_sb[1] ? bh : h) * dh,
+                           a.W2 + (int64_t)(a.p_sb[2] ? bh : h) * dv * dh,
+                           a.b2 + (int64_t)(a.p_sb[3] ? bh : h) * dv};
+    const int64_t len[4] = {(int64_t)dh * dk, dh, (int64_t)dv * dh, dv};
+    float* dst[4] = {sW1, sb1, sW2, sb2};
+    float* dst2[4] = {rW1, rb1, rW2, rb2};
+    for (int m = 0; m < 4; ++m)
+      for (int64_t x = tid; x < len[m]; x += kThreads) dst[m][x] = dst2[m][x] = src[m][x];
+  }
+  __syncthreads();
+
+  const float* eta = a.eta.p + b * a.eta.sb + h * a.eta.sh;
+  for (int cs = 0; cs < a.T; cs += a.chunk) {
+    const int ce = min(cs + a.chunk, a.T);
+    for (int t0 = cs; t0 < ce; t0 += kTB) {
+      const int nt = min(kTB, ce - t0);
+      for (int x = tid; x < kTB * dk; x += kThreads) {
+        const int i = x / dk, c = x % dk;
+        Qs[x] = i < nt ? ldt<T>(a.q, b, h, t0 + i, c) : 0.f;
+        Ks[x] = i < nt ? ldt<T>(a.k, b, h, t0 + i, c) : 0.f;
+      }
+      for (int x = tid; x < kTB * dv; x += kThreads) {
+        const int i = x / dv, c = x % dv;
+        Vs[x] = i < nt ? ldt<T>(a.v, b, h, t0 + i, c) : 0.f;
+      }
+      if (tid < kTB) et[tid] = tid < nt ? eta[(int64_t)(t0 + tid) * a.eta.st] : 0.f;
+      __syncthreads();
+      // h = W1_s k + b1_s, and z0 = W1_run q + b1_run (running: earlier blocks applied)
+      for (int x = tid; x < kTB * dh; x += kThreads) {
+        const int j = x / kTB, i = x % kTB;
+        float hk = sb1[j], zq = rb1[j];
+        const float* w = sW1 + (int64_t)j * dk;
+        const float* wr = rW1 + (int64_t)j * dk;
+        for (int r = 0; r < dk; ++r) {
+          hk = fmaf(w[r], Ks[i * dk + r], hk);
+          zq = fmaf(wr[r], Qs[i * dk + r], zq);
+        }
+        Hs[i * dh + j] = fmaxf(hk, 0.f);
+        Hm[i * dh + j] = hk > 0.f ? 1.f : 0.f;
+        Zs[i * dh + j] = zq;
+      }
+      // S1[t][i] = q_t . k_i + 1 (i <= t)
+      {
+        const int t = tid / kTB, i = tid % kTB;
+        float s = 0.f;
+        if (i <= t) {
+          s = 1.f;
+          for (int r = 0; r < dk; ++r) s = fmaf(Qs[t * dk + r], Ks[i * dk + r], s);
+        }
+        S1[tid] = s;
+      }
+      __syncthreads();
+      // r = W2_s a + b2_s - v
+      for (int x = tid; x < kTB * dv; x += kThreads) {
+        const int c = x / kTB, i = x % kTB;
+        float s = sb2[c];
+        const float* w = sW2 + (int64_t)c * dh;
+        for (int j = 0; j < dh; ++j) s = fmaf(w[j], Hs[i * dh + j], s);
+        Vs[i * dv + c] = s - Vs[i * dv + c];
+      }
+      __syncthreads();
+      // g = (W2_s^T r) [h > 0]
+      for (int x = tid; x < kTB * dh; x += kThreads) {
+        const int j = x / kTB, i = x % kTB;
+        float s = 0.f;
+        for (int c = 0; c < dv; ++c) s = fmaf(sW2[(int64_t)c * dh + j], Vs[i * dv + c], s);
+        Gs[i * dh + j] = s * Hm[i * dh + j];
+      }
+      __syncthreads();
+      // z = z0 - sum_{i<=t} eta_i S1[t][i] g_i ; a' = ReLU(z)
+      for (int x = tid; x < kTB * dh; x += kThreads) {
+        const int t = x / dh, j = x % dh;
+        float z = Zs[x];
+        for (int i = 0; i <= t; ++i) z = fmaf(-et[i] * S1[t * kTB + i], Gs[i * dh + j], z);
+        Zs[x] = fmaxf(z, 0.f);
+      }
+      __syncthreads();
+      // S2[t][i] = a'_t . a_i + 1 (i <= t)
+      {
+        const int t = tid / kTB, i = tid % kTB;
+        float s = 0.f;
+        if (i <= t) {
+          s = 1.f;
+          for (int j = 0; j < dh; ++j) s = fmaf(Zs[t * dh + j], Hs[i * dh + j], s);
+        }
+        S2[tid] = s;
+      }
+      __syncthreads();
+      // y = W2_run a' + b2_run - sum_{i<=t} eta_i S2[t][i] r_i
+      for (int x = tid; x < kTB * dv; x += kThreads) {
+        const int c = x / kTB, t = x % kTB;
+        if (t < nt) {
+          float y = rb2[c];
+          const float* w = rW2 + (int64_t)c * dh;
+          for (int j = 0; j < dh; ++j) y = fmaf(w[j], Zs[t * dh + j], y);
+          for (int i = 0; i <= t; ++i) y = fmaf(-et[i] * S2[t * kTB + i], Vs[i * dv + c], y);
+          T* o = static_cast<T*>(a.out.p) + b * a.out.sb + h * a.out.sh + (int64_t)(t0 + t) * a.out.st;
+          o[c] = T(y);
+        }
+      }
+      __syncthreads();
+      // running parameters: subtract this block's eta-weighted gradients
+      for (int64_t x = tid; x < (int64_t)dh * dk; x += kThreads) {
+        const int j = (int)(x / dk), r = (int)(x % dk);
+        float s = 0.f;
+        for (int i = 0; i < nt; ++i) s = fmaf(et[i] * Gs[i * dh + j], Ks[i * dk + r], s);
+        rW1[x] -= s;
+      }
+      for (int j = tid; j < dh; j += kThreads) {
+        float s = 0.f;
+        for (int i = 0; i < nt; ++i) s = fmaf(et[i], Gs[i * dh + j], s);
+        rb1[j] -= s;
+      }
+      for (int64_t x = tid; x < (int64_t)dv * dh; x += kThreads) {
+        const int c = (int)(x / dh), j = (int)(x % dh);
+        float s = 0.f;
+        for (int i = 0; i < nt; ++i) s = fmaf(et[i] * Vs[i * dv + c], Hs[i * dh + j], s);
+        rW2[x] -= s;
+      }
+      for (int c = tid; c < dv; c += kThreads) {
+        float s = 0.f;
+        for (int i = 0; i < nt; ++i) s = fmaf(et[i], Vs[i * dv + c], s);
+        rb2[c] -= s;
+      }
+      __syncthreads();
+    }
+    // chunk end: the running parameters start the next chunk
+    for (int64_t x = tid; x < nP; x += kThreads) ps[x] = ps[nP + x];
+    __syncthreads();
+  }
+
+  float* fin[4] = {a.W1_final, a.b1_final, a.W2_final, a.b2_final};
+  const int64_t len[4] = {(int64_t)dh * dk, dh, (int64_t)dv * dh, dv};
+  const float* run[4] = {rW1, rb1, rW2, rb2};
+  for (int m = 0; m < 4; ++m)
+    if (fin[m])
+      for (int64_t x = tid; x < len[m]; x += kThreads) fin[m][(int64_t)bh * len[m] + x] = run[m][x];
+}
+
+}  // namespace
+
+bool ttt_mlp_supported(int dk, int dv, int dh) { return dk <= 256 && dv <= 256 && dh <= 512; }
+
+size_t ttt_mlp_workspace(const MlpArgs& a) {
+  const int64_t nP = (int64_t)a.dh * a.dk + a.dh + (int64_t)a.dv * a.dh + a.dv;
+  return (size_t)a.B * a.H * 2 * nP * sizeof(float);
+}
+
+cudaError_t launch_ttt_mlp(const MlpArgs& a, bool bf16, cudaStream_t s) {
+  const size_t smem = sizeof(float) * (2 * kTB * a.dk + kTB * a.dv + 4 * kTB * a.dh +
+                                       2 * kTB * kTB + kTB);
+  cudaError_t e;
+  if (bf16) {
+    e = cudaFuncSetAttribute(ttt_mlp_kernel<__nv_bfloat16>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    ttt_mlp_kernel<__nv_bfloat16><<<a.B * a.H, kThreads, smem, s>>>(a);
+  } else {
+    e = cudaFuncSetAttribute(ttt_mlp_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+    ttt_mlp_kernel<float><<<a.B * a.H, kThreads, smem, s>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace ttt

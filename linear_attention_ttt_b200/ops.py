@@ -46,6 +46,9 @@ class TTTTensor(ctypes.Structure):
 
 _LIB = None
 P = ctypes.POINTER(TTTTensor)
+# lact_grad_reduce_fn of include/ttt.h
+REDUCE_FN = ctypes.CFUNCTYPE(ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
+                             ctypes.c_void_p)
 
 SIGNATURES = {
     "ttt_linear_fwd": ([P, P, P, P, P, ctypes.c_int32, ctypes.c_int32, P, P, ctypes.c_void_p],
@@ -56,9 +59,24 @@ SIGNATURES = {
                             P, P, P, P, ctypes.c_void_p], ctypes.c_int32),
     "lact_swiglu_fwd_noalloc": ([P, P, P, P, P, P, P, ctypes.c_int32, ctypes.c_int32,
                                  ctypes.c_int32, P, P, P, P, ctypes.c_void_p], ctypes.c_int32),
+    "lact_swiglu_fwd_momentum": ([P, P, P, P, P, P, P, ctypes.c_int32, ctypes.c_float,
+                                  ctypes.c_int32, P, P, P, P, P, P, P, P, P, P,
+                                  ctypes.c_void_p], ctypes.c_int32),
+    "ttt_linear_bwd": ([P, P, P, P, P, ctypes.c_int32, ctypes.c_int32, P, P, P, P, P, P, P,
+                        ctypes.c_void_p], ctypes.c_int32),
+    "ttt_mlp_fwd": ([P, P, P, P, P, P, P, P, ctypes.c_int32, P, P, P, P, P, ctypes.c_void_p],
+                    ctypes.c_int32),
+    "window_attention_fwd": ([P, P, P, ctypes.c_int32, ctypes.c_int32, P, ctypes.c_void_p],
+                             ctypes.c_int32),
+    "lact_swiglu_window_fwd": ([P, P, P, P, P, P, P, ctypes.c_int32, ctypes.c_int32,
+                               ctypes.c_int32, P, ctypes.c_void_p], ctypes.c_int32),
+    "lact_swiglu_fwd_cp": ([P, P, P, P, P, P, P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                            P, P, P, P, REDUCE_FN, ctypes.c_void_p, ctypes.c_void_p],
+                           ctypes.c_int32),
     "ttt_status_string": ([ctypes.c_int32], ctypes.c_char_p),
     "ttt_get_device_status": ([ctypes.c_void_p], ctypes.c_int32),
     "ttt_version": ([], ctypes.c_int32),
+    "ttt_test_fail_allocations": ([ctypes.c_int32], None),
     "ttt_selftest_wait_timeout": ([ctypes.c_void_p], ctypes.c_int32),
 }
 
@@ -132,6 +150,38 @@ def ttt_linear_fwd(q, k, v, eta, W0, chunk: int, loss: int, out=None, W_final=No
     return out, W_final
 
 
+def ttt_linear_bwd(q, k, v, eta, W0, chunk: int, loss: int, dy, dW_final=None, stream=None):
+    """Backward of ttt_linear_fwd: given dL/dy (and optionally dL/dW_final),
+    returns (dq, dk, dv, deta, dW0); dW0 has W0's shape (summed over the
+    batch when W0 is shared by it)."""
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    deta = torch.empty(eta.shape, dtype=torch.float32, device=q.device)
+    dW0 = torch.empty(W0.shape, dtype=torch.float32, device=q.device)
+    ds = [describe(x) for x in (q, k, v, eta, W0, dy, dW_final, dq, dk, dv, deta, dW0)]
+    r = [_ref(d) for d in ds]
+    code = load().ttt_linear_bwd(*r[:5], int(chunk), int(loss), *r[5:], _stream(stream))
+    _check(code, "ttt_linear_bwd")
+    return dq, dk, dv, deta, dW0
+
+
+def ttt_mlp_fwd(q, k, v, eta, W1, b1, W2, b2, chunk: int, out=None, finals=False, stream=None):
+    """TTT-MLP forward (two-layer ReLU MLP fast weight, mini-batch rule). With
+    finals=True also returns the final (W1, b1, W2, b2) as [B,H,...] tensors."""
+    B, H, T, dk = q.shape
+    dv, dh = v.shape[-1], W1.shape[-2]
+    if out is None:
+        out = torch.empty((B, H, T, dv), dtype=q.dtype, device=q.device)
+    F = [None] * 4
+    if finals:
+        F = [torch.empty(s, dtype=torch.float32, device=q.device)
+             for s in ((B, H, dh, dk), (B, H, dh), (B, H, dv, dh), (B, H, dv))]
+    ds = [describe(x) for x in (q, k, v, eta, W1, b1, W2, b2, out, *F)]
+    r = [_ref(d) for d in ds]
+    code = load().ttt_mlp_fwd(*r[:8], int(chunk), *r[8:], _stream(stream))
+    _check(code, "ttt_mlp_fwd")
+    return (out, *F) if finals else out
+
+
 def lact_swiglu_fwd(q, k, v, eta, W1, W2, W3, chunk: int, update_rule: int = LACT_UPDATE_GD,
                     causal: int = 1, out=None, finals=False, stream=None):
     """LaCT SwiGLU fast-weight layer forward. With finals=True also returns
@@ -178,6 +228,56 @@ def lact_swiglu_fwd_noalloc(q, k, v, eta, W1, W2, W3, chunk: int,
                                           r[8], r[9], r[10], _stream(stream))
     _check(code, "lact_swiglu_fwd_noalloc")
     return (out, *F) if finals else out
+
+
+def lact_swiglu_fwd_momentum(q, k, v, eta, W1, W2, W3, chunk: int, beta: float,
+                             causal: int = 1, M0=(None, None, None), out=None, finals=False,
+                             stream=None):
+    """LaCT forward with heavy-ball momentum on the chunk gradients
+    (M <- beta M + G, W <- W - M, then the row renorm). M0 = (M1, M2, M3)
+    initial momentum (None: zero). With finals=True also returns the final
+    (W1, W2, W3) and (M1, M2, M3) as [B,H,...] fp32 tensors."""
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    dh = W1.shape[-2]
+    if out is None:
+        out = torch.empty((B, H, T, dv), dtype=q.dtype, device=q.device)
+    F = [None] * 6
+    if finals:
+        shapes = [(B, H, dh, dk), (B, H, dv, dh), (B, H, dh, dk)] * 2
+        F = [torch.empty(s, dtype=torch.float32, device=q.device) for s in shapes]
+    ds = [describe(x) for x in (q, k, v, eta, W1, W2, W3, *M0, out, *F)]
+    r = [_ref(d) for d in ds]
+    code = load().lact_swiglu_fwd_momentum(*r[:7], int(chunk), float(beta), int(causal),
+                                           r[7], r[8], r[9], r[10], *r[11:17], _stream(stream))
+    _check(code, "lact_swiglu_fwd_momentum")
+    return (out, tuple(F[:3]), tuple(F[3:])) if finals else out
+
+
+def window_attention_fwd(q, k, v, window: int, out=None, accumulate: bool = False, stream=None):
+    """Sliding-window causal softmax attention (scale 1/sqrt(d)); with
+    accumulate=True the result is added into `out`."""
+    if out is None:
+        out = torch.zeros_like(v) if accumulate else torch.empty_like(v)
+    ds = [describe(x) for x in (q, k, v, out)]
+    r = [_ref(d) for d in ds]
+    code = load().window_attention_fwd(r[0], r[1], r[2], int(window), int(bool(accumulate)), r[3],
+                                       _stream(stream))
+    _check(code, "window_attention_fwd")
+    return out
+
+
+def lact_swiglu_window_fwd(q, k, v, eta, W1, W2, W3, chunk: int, update_rule: int, window: int,
+                           out=None, stream=None):
+    """LaCT layer (causal) plus window attention on the same q, k, v, summed."""
+    if out is None:
+        out = torch.empty_like(v)
+    ds = [describe(x) for x in (q, k, v, eta, W1, W2, W3, out)]
+    r = [_ref(d) for d in ds]
+    code = load().lact_swiglu_window_fwd(*r[:7], int(chunk), int(update_rule), int(window), r[7],
+                                         _stream(stream))
+    _check(code, "lact_swiglu_window_fwd")
+    return out
 
 
 def selftest_wait_timeout(stream=None) -> None:

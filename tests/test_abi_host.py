@@ -23,6 +23,7 @@ def lib():
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"^\s*typedef[^;]*;", "", text, flags=re.M | re.S)
     names = re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\*?(\w+)\s*\(", text, flags=re.M)
     return sorted(set(n for n in names if n not in ("if", "return")))
 
@@ -30,7 +31,9 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("ttt_linear_fwd", "lact_swiglu_fwd", "lact_swiglu_fwd_ex", "ttt_status_string",
-              "ttt_get_device_status", "ttt_version"):
+              "ttt_get_device_status", "ttt_version", "ttt_linear_bwd", "lact_swiglu_fwd_momentum",
+              "ttt_mlp_fwd", "window_attention_fwd", "lact_swiglu_window_fwd",
+              "lact_swiglu_fwd_cp", "lact_swiglu_fwd_noalloc", "ttt_test_fail_allocations"):
         assert n in names
 
 
@@ -250,3 +253,43 @@ def test_noalloc_scratch_limit_is_the_documented_formula(lib, d, dh, chunk, T, r
     assert n_max >= 1
     assert noalloc_call(lib, n_max, T, d, dh, chunk, rule) == ERR["TTT_ERR_CUDA"]
     assert noalloc_call(lib, n_max + 1, T, d, dh, chunk, rule) == ERR["TTT_ERR_SCRATCH"]
+
+
+def momentum_call(lib, beta=0.9, mutate=None):
+    gap = 1 << 28
+    Bs, H, T, d, dh = 1, 2, 64, 128, 256
+    ts = dict(q=tok(Bs, H, T, d, base=FAKE), k=tok(Bs, H, T, d, base=FAKE + gap),
+              v=tok(Bs, H, T, d, base=FAKE + 2 * gap), eta=dense((Bs, H, T), FAKE + 3 * gap),
+              W1=dense((H, dh, d), FAKE + 4 * gap), W2=dense((H, d, dh), FAKE + 5 * gap),
+              W3=dense((H, dh, d), FAKE + 6 * gap), M1=dense((H, dh, d), FAKE + 7 * gap),
+              M2=None, M3=None, out=tok(Bs, H, T, d, base=FAKE + 8 * gap),
+              M1f=dense((Bs, H, dh, d), FAKE + 9 * gap))
+    if mutate:
+        mutate(ts)
+    r = lambda x: ctypes.byref(x) if x is not None else None
+    return lib.lact_swiglu_fwd_momentum(*(r(ts[n]) for n in ("q", "k", "v", "eta", "W1", "W2", "W3")),
+                                        32, beta, 1, r(ts["M1"]), r(ts["M2"]), r(ts["M3"]),
+                                        r(ts["out"]), None, None, None, r(ts["M1f"]), None, None,
+                                        None)
+
+
+def test_momentum_entry_rejects_bad_arguments(lib):
+    beta = float
+    assert momentum_call(lib, beta(float("nan"))) == ERR["TTT_ERR_ARG"]
+    assert momentum_call(lib, beta(float("inf"))) == ERR["TTT_ERR_ARG"]
+
+    def bad_m1(ts):
+        ts["M1"] = dense((2, 128, 256), ts["M1"].data)
+    assert momentum_call(lib, beta(0.9), bad_m1) == ERR["TTT_ERR_SHAPE"]
+
+    def m1_bf16(ts):
+        ts["M1"].dtype = ops.TTT_BF16
+    assert momentum_call(lib, beta(0.9), m1_bf16) == ERR["TTT_ERR_DTYPE"]
+
+    def final_on_input(ts):
+        ts["M1f"].data = ts["M1"].data
+    assert momentum_call(lib, beta(0.9), final_on_input) == ERR["TTT_ERR_ARG"]
+
+    def final_on_out(ts):
+        ts["M1f"].data = ts["out"].data
+    assert momentum_call(lib, beta(0.9), final_on_out) == ERR["TTT_ERR_ARG"]

@@ -23,3 +23,42 @@ def test_bounded_wait_reports_timeout_and_the_context_survives():
     yo, Wo = O.ttt_linear_minibatch(w.q, w.k, w.v, w.eta, w.W0, w.chunk, w.loss)
     check(y, yo, w.dtype, "y")
     check(Wf, Wo, w.dtype, "W_final")
+
+
+def test_failed_scratch_allocation_is_reported_and_recovers():
+    """Host-side injection (no GPU fault): the next scratch allocation fails as
+    if the device were out of memory. The call returns TTT_ERR_ALLOC, writes
+    nothing, and the next call runs normally."""
+    import torch
+    from linear_attention_ttt_b200 import synth
+    from tests.gpu_util import upload_lact
+    w = synth.make_lact(1, 2, 256, 128, 256, 64, synth.UPDATE_GD, seed=8)
+    t = upload_lact(w)
+    args = (t["q"], t["k"], t["v"], t["eta"], t["W1"], t["W2"], t["W3"], w.chunk)
+    sentinel = torch.full((1, 2, 256, 128), 7.0, dtype=torch.bfloat16, device="cuda")
+    out = sentinel.clone()
+    lib = ops.load()
+    lib.ttt_test_fail_allocations(1)
+    try:
+        with pytest.raises(ops.TTTError) as e:
+            ops.lact_swiglu_fwd(*args, out=out)
+        assert e.value.code == -8   # TTT_ERR_ALLOC
+    finally:
+        lib.ttt_test_fail_allocations(0)
+    torch.cuda.synchronize()
+    assert torch.equal(out, sentinel)
+    assert ops.device_status() == 0
+    ref = ops.lact_swiglu_fwd(*args)
+    again = ops.lact_swiglu_fwd(*args, out=out)
+    torch.cuda.synchronize()
+    assert torch.equal(ref, again)
+    # the same hook reaches the other allocating entry points
+    lib.ttt_test_fail_allocations(1)
+    try:
+        with pytest.raises(ops.TTTError) as e:
+            ops.ttt_mlp_fwd(t["q"], t["k"], t["v"], t["eta"], t["W1"][:, :, :128],
+                            torch.zeros(2, 256, device="cuda"), t["W2"][:, :, :256].contiguous(),
+                            torch.zeros(2, 128, device="cuda"), 16)
+        assert e.value.code == -8
+    finally:
+        lib.ttt_test_fail_allocations(0)
