@@ -60,11 +60,13 @@
  *    same process is not supported.
  *  - Supported sizes: B, H, T >= 1 (T = 0 is accepted and does nothing
  *    except copying W0 to W_final); chunk >= 1 (a shorter last chunk is
- *    allowed); dk, dv in [1, 256] for fp32 tensors. bf16 kernels take
- *    dk = dv in {64, 128} for TTT-Linear and d in {64, 128, 256},
- *    dh a multiple of 128 up to 1024 for LaCT; other sizes return
- *    TTT_ERR_UNSUPPORTED, and so do T > 2^30 tokens and B*H > 2^24
- *    (the kernels index tokens and (batch, head) pairs with 32-bit integers).
+ *    allowed). TTT-Linear: dk, dv in [1, 256] (bf16: multiples of 8, from
+ *    the stride rule); dk = dv = 64 or 128 run the tensor-core kernels, every
+ *    other size (dk != dv included) a CUDA-core kernel with fp32
+ *    arithmetic. LaCT: d = dk = dv in {64, 128, 256} and dh a multiple of
+ *    128 up to 1024, bf16 tokens. Other sizes return TTT_ERR_UNSUPPORTED, and
+ *    so do T > 2^30 tokens and B*H > 2^24 (the kernels index tokens and
+ *    (batch, head) pairs with 32-bit integers).
  */
 #ifndef TTT_B200_H
 #define TTT_B200_H

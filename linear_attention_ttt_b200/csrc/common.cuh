@@ -108,6 +108,7 @@ struct LinearArgs {
 };
 
 cudaError_t launch_ttt_linear_f32(const LinearArgs& a, cudaStream_t s);
+cudaError_t launch_ttt_linear_cc_bf16(const LinearArgs& a, cudaStream_t s);
 cudaError_t launch_ttt_linear_bf16(const LinearArgs& a, cudaStream_t s, bool* supported);
 bool ttt_linear_wy_supported(const LinearArgs& a);
 cudaError_t launch_ttt_linear_wy(const LinearArgs& a, cudaStream_t s);

@@ -393,8 +393,9 @@ cudaError_t launch(const LinearArgs& a, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_ttt_linear_bf16(const LinearArgs& a, cudaStream_t s, bool* supported) {
-  *supported = (a.dk == a.dv) && (a.dk == 64 || a.dk == 128);
-  if (!*supported) return cudaSuccess;
+  *supported = true;
+  // head sizes without a tensor-core kernel: fp32 arithmetic on the CUDA cores
+  if (!((a.dk == a.dv) && (a.dk == 64 || a.dk == 128))) return launch_ttt_linear_cc_bf16(a, s);
   if (la_tc_supported(a)) return launch_la_tc(a, s);
   if (ttt_linear_wy_supported(a)) return launch_ttt_linear_wy(a, s);
   return a.dk == 64 ? launch<64>(a, s) : launch<128>(a, s);

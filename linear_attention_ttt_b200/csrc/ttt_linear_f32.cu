@@ -1,5 +1,6 @@
-// TTT-Linear / inner-product layer forward for fp32 tokens (CUDA cores, fp32
-// throughout).
+// TTT-Linear / inner-product layer forward on the CUDA cores with fp32
+// arithmetic throughout: every fp32 shape, and the bf16 head sizes the
+// tensor-core kernels do not cover (dk or dv other than 64 / 128, dk != dv).
 //
 // Computes, per (batch, head), the mini-batch GD rule of the "Test-Time
 // Training (TTT)" summary ("병렬화: Mini-batch Gradient Descent"): with t' the
@@ -28,6 +29,7 @@ __device__ __forceinline__ const T* tok_row(const TokView& v, int b, int h, int6
   return static_cast<const T*>(v.p) + b * v.sb + h * v.sh + t * v.st;
 }
 
+template <typename TT>
 __global__ void __launch_bounds__(kThreads)
 ttt_linear_f32_kernel(LinearArgs a) {
   extern __shared__ float smem[];
@@ -63,12 +65,12 @@ ttt_linear_f32_kernel(LinearArgs a) {
       for (int x = tid; x < kTB * dk; x += kThreads) {
         int i = x / dk, c = x % dk;
         bool ok = i < nt;
-        Qs[x] = ok ? tok_row<float>(a.q, b, h, t0 + i)[c] : 0.f;
-        Ks[x] = ok ? tok_row<float>(a.k, b, h, t0 + i)[c] : 0.f;
+        Qs[x] = ok ? to_f32(tok_row<TT>(a.q, b, h, t0 + i)[c]) : 0.f;
+        Ks[x] = ok ? to_f32(tok_row<TT>(a.k, b, h, t0 + i)[c]) : 0.f;
       }
       for (int x = tid; x < kTB * kCols; x += kThreads) {
         int i = x / kCols, c = x % kCols;
-        Vs[x] = (i < nt && c < ncol) ? tok_row<float>(a.v, b, h, t0 + i)[j0 + c] : 0.f;
+        Vs[x] = (i < nt && c < ncol) ? to_f32(tok_row<TT>(a.v, b, h, t0 + i)[j0 + c]) : 0.f;
       }
       if (tid < kTB) etas[tid] = tid < nt ? eta[(int64_t)(t0 + tid) * a.eta.st] : 0.f;
       __syncthreads();
@@ -98,9 +100,9 @@ ttt_linear_f32_kernel(LinearArgs a) {
           for (int r = 0; r < dk; ++r)
             acc = fmaf(Qs[t * dk + r], Wst[r * kCols + c] - dW[r * kCols + c], acc);
           for (int i = 0; i <= t; ++i) acc = fmaf(-etas[i] * Ss[t * kTB + i], Es[i * kCols + c], acc);
-          float* o = static_cast<float*>(a.out.p) + b * a.out.sb + h * a.out.sh +
-                     (int64_t)(t0 + t) * a.out.st;
-          o[j0 + c] = acc;
+          TT* o = static_cast<TT*>(a.out.p) + b * a.out.sb + h * a.out.sh +
+                  (int64_t)(t0 + t) * a.out.st;
+          o[j0 + c] = TT(acc);
         }
       }
       __syncthreads();
@@ -130,17 +132,26 @@ ttt_linear_f32_kernel(LinearArgs a) {
   }
 }
 
-}  // namespace
-
-cudaError_t launch_ttt_linear_f32(const LinearArgs& a, cudaStream_t s) {
+template <typename TT>
+cudaError_t launch_cc(const LinearArgs& a, cudaStream_t s) {
   const size_t smem =
       sizeof(float) * (2 * a.dk * kCols + 2 * kTB * a.dk + 2 * kTB * kCols + kTB * kTB + kTB);
-  cudaError_t e = cudaFuncSetAttribute(ttt_linear_f32_kernel,
+  cudaError_t e = cudaFuncSetAttribute(ttt_linear_f32_kernel<TT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.B * a.H, (a.dv + kCols - 1) / kCols);
-  ttt_linear_f32_kernel<<<grid, kThreads, smem, s>>>(a);
+  ttt_linear_f32_kernel<TT><<<grid, kThreads, smem, s>>>(a);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_ttt_linear_f32(const LinearArgs& a, cudaStream_t s) {
+  return launch_cc<float>(a, s);
+}
+
+cudaError_t launch_ttt_linear_cc_bf16(const LinearArgs& a, cudaStream_t s) {
+  return launch_cc<__nv_bfloat16>(a, s);
 }
 
 }  // namespace ttt

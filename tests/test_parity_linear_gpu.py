@@ -169,9 +169,25 @@ def test_bf16_resume_from_w_final(loss, split):
         check(Wb.float().cpu().numpy(), Wo, synth.BF16, "resumed W_final")
 
 
-def test_bf16_unsupported_head_size_is_rejected():
+@pytest.mark.parametrize("dk,dv", [(16, 16), (32, 32), (48, 48), (80, 80), (256, 256),
+                                   (64, 32), (32, 128), (128, 48)])
+@pytest.mark.parametrize("loss", [ops.TTT_LOSS_MSE, ops.TTT_LOSS_NEG_DOT])
+def test_bf16_other_head_sizes(dk, dv, loss):
+    """bf16 head sizes without a tensor-core kernel (any multiple of 16 up to
+    256, dk != dv) run the CUDA-core kernel; ragged last chunk."""
+    w = synth.make_ttt_linear(2, 2, 70, dk, dv, 16, synth.BF16, loss, seed=dk + 3 * dv,
+                              eta_kind="softplus", eta_scale=0.05)
+    y, Wf = run_linear(w)
+    yo, Wo = oracle_linear(w, definition=True)
+    check(y, yo, w.dtype, f"y dk{dk} dv{dv}")
+    check(Wf, Wo, w.dtype, f"W_final dk{dk} dv{dv}")
+
+
+def test_oversized_head_is_rejected():
     w = synth.make_ttt_linear(1, 1, 16, 32, 32, 16, synth.BF16, 0, seed=1)
     t = upload_linear(w)
+    q = torch.zeros((1, 1, 16, 272), dtype=torch.bfloat16, device="cuda")
+    W0 = torch.zeros((1, 272, 32), device="cuda")
     with pytest.raises(ops.TTTError) as e:
-        ops.ttt_linear_fwd(t["q"], t["k"], t["v"], t["eta"], t["W0"], 16, 0)
+        ops.ttt_linear_fwd(q, q, t["v"], t["eta"], W0, 16, 0)
     assert e.value.code == -5
