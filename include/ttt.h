@@ -267,6 +267,38 @@ ttt_status lact_swiglu_fwd_cp(const ttt_tensor* q, const ttt_tensor* k, const tt
                               void* reduce_user, void* stream);
 
 /*
+ * LaCT SwiGLU layer backward (training): the gradients of a scalar objective
+ * through lact_swiglu_fwd_ex, given dL/dy and optionally dL/d(final weights).
+ * Same review and sections as lact_swiglu_fwd. The chunks are walked in
+ * reverse; each one differentiates, in this order, the row renorm to the
+ * initial norms (whose target norms pass gradient back to the initial
+ * weights), the step, Newton-Schulz under Muon (through its five polynomial
+ * iterations and the Frobenius normalisation), the gradient formulas
+ * themselves (second order: through silu, silu' and silu'' of K W1^T), and
+ * the SwiGLU apply of the chunk's queries.
+ *  q, k, v, eta, W1, W2, W3, chunk, update_rule, causal   as lact_swiglu_fwd
+ *           (bf16 or fp32 tokens; d, dh <= 256, 1024; B*H <= 65535)
+ *  dy       [B,H,T,dv], same type as q
+ *  dW?_final NULL (zero) or [B,H,...] fp32 contiguous
+ *  dq, dk   [B,H,T,dk], dv [B,H,T,dv]: same type as q
+ *  deta     [B,H,T] fp32 contiguous
+ *  dW1, dW2, dW3  the shapes of W1, W2, W3, fp32 contiguous; per-head
+ *           weights ([H,...], shared over the batch) get the batch sum
+ * Arithmetic: fp32 throughout (batched fp32 GEMMs on the CUDA cores), from a
+ * forward recomputed in fp32, so the result is the derivative of the fp32
+ * forward. Workspace is stream-ordered from the library's pool (failure ->
+ * TTT_ERR_ALLOC).
+ */
+ttt_status lact_swiglu_bwd(const ttt_tensor* q, const ttt_tensor* k, const ttt_tensor* v,
+                           const ttt_tensor* eta, const ttt_tensor* W1, const ttt_tensor* W2,
+                           const ttt_tensor* W3, int32_t chunk, int32_t update_rule,
+                           int32_t causal, const ttt_tensor* dy, const ttt_tensor* dW1_final,
+                           const ttt_tensor* dW2_final, const ttt_tensor* dW3_final,
+                           const ttt_tensor* dq, const ttt_tensor* dk, const ttt_tensor* dv,
+                           const ttt_tensor* deta, const ttt_tensor* dW1, const ttt_tensor* dW2,
+                           const ttt_tensor* dW3, void* stream);
+
+/*
  * lact_swiglu_fwd_ex without any device memory allocation. (The pages have
  * no counterpart to this call: it exists for callers that cannot allocate.)
  *

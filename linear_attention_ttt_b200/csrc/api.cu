@@ -732,3 +732,65 @@ ttt_status lact_swiglu_fwd_cp(const ttt_tensor* q, const ttt_tensor* k, const tt
 }
 
 }  // extern "C"
+
+extern "C" {
+
+ttt_status lact_swiglu_bwd(const ttt_tensor* q, const ttt_tensor* k, const ttt_tensor* v,
+                           const ttt_tensor* eta, const ttt_tensor* W1, const ttt_tensor* W2,
+                           const ttt_tensor* W3, int32_t chunk, int32_t update_rule,
+                           int32_t causal, const ttt_tensor* dy, const ttt_tensor* dW1_final,
+                           const ttt_tensor* dW2_final, const ttt_tensor* dW3_final,
+                           const ttt_tensor* dq, const ttt_tensor* dk, const ttt_tensor* dv,
+                           const ttt_tensor* deta, const ttt_tensor* dW1, const ttt_tensor* dW2,
+                           const ttt_tensor* dW3, void* stream) {
+  if (!dy || !dq || !dk || !dv || !deta || !dW1 || !dW2 || !dW3) return TTT_ERR_NULL;
+  ttt::LactArgs a;
+  // the forward's arguments, with dy in the place of the output (same shape)
+  ttt_status st = ttt::lact_build_args(q, k, v, eta, W1, W2, W3, chunk, update_rule, causal, dy,
+                                       nullptr, nullptr, nullptr, &a);
+  if (st != TTT_OK) return st;
+  if (!ttt::lact_bwd_supported(a)) return TTT_ERR_UNSUPPORTED;
+  const int64_t B = a.B, H = a.H, T = a.T, dK = a.dk, dV = a.dv, dH = a.dh;
+  if ((st = check_tokens(dq, B, H, T, dK, a.dtype)) != TTT_OK) return st;
+  if ((st = check_tokens(dk, B, H, T, dK, a.dtype)) != TTT_OK) return st;
+  if ((st = check_tokens(dv, B, H, T, dV, a.dtype)) != TTT_OK) return st;
+  if (deta->ndim != 3 || deta->shape[0] != B || deta->shape[1] != H || deta->shape[2] != T)
+    return TTT_ERR_SHAPE;
+  if (deta->dtype != TTT_F32) return TTT_ERR_DTYPE;
+  if (!deta->data && T > 0) return TTT_ERR_NULL;
+  if (T > 0 && (!contiguous(deta) || !aligned16(deta->data))) return TTT_ERR_LAYOUT;
+  const ttt_tensor* Wt[3] = {W1, W2, W3};
+  const ttt_tensor* dWt[3] = {dW1, dW2, dW3};
+  const ttt_tensor* dWf[3] = {dW1_final, dW2_final, dW3_final};
+  const int64_t rows[3] = {dH, dV, dH}, cols[3] = {dK, dH, dK};
+  for (int m = 0; m < 3; ++m) {
+    int64_t sb = 0;
+    if ((st = lact_check_weight(dWt[m], B, H, rows[m], cols[m], &sb)) != TTT_OK) return st;
+    if (dWt[m]->ndim != Wt[m]->ndim) return TTT_ERR_SHAPE;
+    if ((st = lact_check_final(dWf[m], B, H, rows[m], cols[m])) != TTT_OK) return st;
+  }
+  const ttt_tensor* ins[] = {q, k, v, eta, W1, W2, W3, dy, dW1_final, dW2_final, dW3_final};
+  const ttt_tensor* outs[] = {dq, dk, dv, deta, dW1, dW2, dW3};
+  for (const ttt_tensor* o : outs) {
+    for (const ttt_tensor* in : ins)
+      if (overlaps(o, in)) return TTT_ERR_ARG;
+    for (const ttt_tensor* o2 : outs)
+      if (o != o2 && overlaps(o, o2)) return TTT_ERR_ARG;
+  }
+  ttt::LactBwdArgs g;
+  g.dy = view(dy);
+  g.dW1_final = dW1_final ? static_cast<const float*>(dW1_final->data) : nullptr;
+  g.dW2_final = dW2_final ? static_cast<const float*>(dW2_final->data) : nullptr;
+  g.dW3_final = dW3_final ? static_cast<const float*>(dW3_final->data) : nullptr;
+  g.dq = {dq->data, dq->stride[0], dq->stride[1], dq->stride[2]};
+  g.dk = {dk->data, dk->stride[0], dk->stride[1], dk->stride[2]};
+  g.dv = {dv->data, dv->stride[0], dv->stride[1], dv->stride[2]};
+  g.deta = static_cast<float*>(deta->data);
+  g.dW1 = static_cast<float*>(dW1->data);
+  g.dW2 = static_cast<float*>(dW2->data);
+  g.dW3 = static_cast<float*>(dW3->data);
+  if ((st = ttt::lact_attach_status(&a)) != TTT_OK) return st;
+  return ttt::lact_backward(a, g, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -38,6 +38,19 @@ size_t lact_scratch_bytes(const LactArgs& a);
 // 256-byte aligned. Allocates nothing.
 ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* scratch, size_t bytes);
 
+// Backward (lact_swiglu_bwd): upstream gradients in, gradients out.
+struct LactBwdArgs {
+  TokView dy;                         // [B,H,T,dv]
+  const float *dW1_final, *dW2_final, *dW3_final;  // [B*H] x weight, each may be null
+  TokViewMut dq, dk, dv;              // same element type as q
+  float* deta;                        // [B,H,T] contiguous
+  float *dW1, *dW2, *dW3;             // shape of W1, W2, W3 (batch-summed when shared)
+};
+bool lact_bwd_supported(const LactArgs& a);
+// Enqueues the backward on `s` (fp32 arithmetic; allocates its workspace
+// stream-ordered from the library's pool).
+ttt_status lact_backward(const LactArgs& a, const LactBwdArgs& g, cudaStream_t s);
+
 // Validates the C-ABI arguments of lact_swiglu_fwd_ex and fills `a`, except
 // its status pointer. Makes no CUDA call.
 ttt_status lact_build_args(const ttt_tensor* q, const ttt_tensor* k, const ttt_tensor* v,

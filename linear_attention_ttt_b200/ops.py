@@ -73,6 +73,8 @@ SIGNATURES = {
     "lact_swiglu_fwd_cp": ([P, P, P, P, P, P, P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                             P, P, P, P, REDUCE_FN, ctypes.c_void_p, ctypes.c_void_p],
                            ctypes.c_int32),
+    "lact_swiglu_bwd": ([P, P, P, P, P, P, P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                         P, P, P, P, P, P, P, P, P, P, P, ctypes.c_void_p], ctypes.c_int32),
     "ttt_status_string": ([ctypes.c_int32], ctypes.c_char_p),
     "ttt_get_device_status": ([ctypes.c_void_p], ctypes.c_int32),
     "ttt_version": ([], ctypes.c_int32),
@@ -202,6 +204,21 @@ def lact_swiglu_fwd(q, k, v, eta, W1, W2, W3, chunk: int, update_rule: int = LAC
                                      r[8], r[9], r[10], _stream(stream))
     _check(code, "lact_swiglu_fwd")
     return (out, *F) if finals else out
+
+
+def lact_swiglu_bwd(q, k, v, eta, W1, W2, W3, chunk: int, update_rule: int, causal: int, dy,
+                    dW_final=(None, None, None), stream=None):
+    """Backward of lact_swiglu_fwd: returns (dq, dk, dv, deta, dW1, dW2, dW3),
+    the weight gradients in the shapes of W1, W2, W3."""
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    deta = torch.empty(eta.shape, dtype=torch.float32, device=q.device)
+    dW = [torch.empty(W.shape, dtype=torch.float32, device=q.device) for W in (W1, W2, W3)]
+    ds = [describe(x) for x in (q, k, v, eta, W1, W2, W3, dy, *dW_final, dq, dk, dv, deta, *dW)]
+    r = [_ref(d) for d in ds]
+    code = load().lact_swiglu_bwd(*r[:7], int(chunk), int(update_rule), int(causal), *r[7:],
+                                  _stream(stream))
+    _check(code, "lact_swiglu_bwd")
+    return (dq, dk, dv, deta, *dW)
 
 
 def lact_swiglu_fwd_noalloc(q, k, v, eta, W1, W2, W3, chunk: int,
