@@ -446,6 +446,102 @@ class Runner:
         return res
 
 
+def window_flops(B, H, T, d, window):
+    """QK^T and PV over the causal window: 4 d flops per (query, key) pair."""
+    pairs = sum(min(t + 1, window) for t in range(T)) if T <= 1 << 16 else (
+        window * (window + 1) // 2 + (T - window) * window if T > window else T * (T + 1) // 2)
+    return 4 * d * B * H * pairs
+
+
+def measure_next_rows(runner, device):
+    """The scope table's next rows, each timed like the hot path (device
+    events over K steps after W warm-ups, L2 flushed by a read before every
+    step) on synthetic inputs of the pages' shapes. Returns a list of dicts."""
+    from linear_attention_ttt_b200 import cp  # noqa: F401  (binding of the context-parallel call)
+    pk = peaks()
+    out = []
+
+    def dev(x, dtype):
+        a = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(device)
+        return a.to(torch.bfloat16) if dtype == synth.BF16 else a
+
+    def run(row, cfg, step, tokens, roof=None, launches=None):
+        ms, clocks, _ = runner.device_timing(step)
+        item = {"row": row, "config": cfg, "ms_per_step": ms, "value": tokens / (ms / 1e3),
+                "unit": "tokens/s", "clocks": clocks}
+        if roof is not None:
+            kind, work, peak, unit, kernel = roof
+            ach = work / (ms / 1e3) / (1e12 if unit == "TFLOP/s" else 1e9)
+            item["roofline"] = {"bound": kind, "achieved": ach, "peak": peak, "unit": unit,
+                                "frac": ach / peak, "kernel": kernel,
+                                "peak_source": pk["_source"]}
+        out.append(item)
+        torch.cuda.empty_cache()
+
+    # f1: TTT-Linear MSE / inner-product backward
+    for idx, T in ((3, 2048), (2, 1024)):
+        w = synth.config(idx, T=T)
+        t = {n: dev(getattr(w, n), w.dtype if n in "qkv" else synth.F32)
+             for n in ("q", "k", "v", "eta", "W0")}
+        dy = torch.randn_like(t["v"])
+        run(f"f1 backward {'mse' if w.loss == 0 else 'inner product'}",
+            {"workload": w.name, "batch": w.B, "heads": w.H, "seq_len": T, "d": w.dk,
+             "chunk": w.chunk},
+            lambda: ops.ttt_linear_bwd(t["q"], t["k"], t["v"], t["eta"], t["W0"], w.chunk,
+                                       w.loss, dy), w.B * T)
+        del t, dy
+    # f1: LaCT backward (GD), one shortened head pair of the d = 128 shape
+    w = synth.make_lact(1, 2, 4096, 128, 512, 1024, synth.UPDATE_GD, seed=1090)
+    t = {n: dev(getattr(w, n), w.dtype if n in "qkv" else synth.F32)
+         for n in ("q", "k", "v", "eta", "W1", "W2", "W3")}
+    dy = torch.randn_like(t["v"])
+    run("f1 backward lact gd", {"workload": "lact_bwd_B1_H2_T4096_d128_dh512_b1024"},
+        lambda: ops.lact_swiglu_bwd(t["q"], t["k"], t["v"], t["eta"], t["W1"], t["W2"], t["W3"],
+                                    w.chunk, 0, 1, dy), w.B * w.T)
+    del t, dy
+    # f2: LaCT momentum at the GD workload's size
+    w = synth.config(4)
+    t = {n: dev(getattr(w, n), w.dtype if n in "qkv" else synth.F32)
+         for n in ("q", "k", "v", "eta", "W1", "W2", "W3")}
+    o = torch.empty_like(t["v"])
+    run("f2 momentum (beta 0.9)", {"workload": w.name + "_momentum"},
+        lambda: ops.lact_swiglu_fwd_momentum(t["q"], t["k"], t["v"], t["eta"], t["W1"], t["W2"],
+                                             t["W3"], w.chunk, 0.9, out=o), w.B * w.T,
+        ("tensor", lact_flops(w), pk["bf16_tflops"], "TFLOP/s", "lact step (all launches)"))
+    # f4b: context-parallel call with no exchange (one rank) at the same size
+    run("f4b context parallel (1 rank)", {"workload": w.name + "_cp1"},
+        lambda: cp.lact_swiglu_fwd_cp(t["q"], t["k"], t["v"], t["eta"], t["W1"], t["W2"],
+                                      t["W3"], w.chunk, 0, None, out=o), w.B * w.T,
+        ("tensor", lact_flops(w), pk["bf16_tflops"], "TFLOP/s", "lact step (all launches)"))
+    del t, o
+    # f3: TTT-MLP, head 64, hidden 256, chunk 16
+    w = synth.config(3, B=4, T=2048)
+    rng = np.random.default_rng(7)
+    P = [rng.standard_normal((w.H, 256, 64)) / 8, np.zeros((w.H, 256)),
+         rng.standard_normal((w.H, 64, 256)) / 16, np.zeros((w.H, 64))]
+    t = [dev(getattr(w, n), w.dtype) for n in ("q", "k", "v")] + [dev(w.eta, synth.F32)]
+    Pd = [dev(p, synth.F32) for p in P]
+    run("f3 ttt-mlp", {"workload": "ttt_mlp_bf16_B4_H16_T2048_d64_dh256_b16"},
+        lambda: ops.ttt_mlp_fwd(*t, *Pd, 16), w.B * w.T)
+    del t, Pd
+    # f4a: window attention (window 4096) and the LaCT + window block, Muon workload
+    w = synth.config(5)
+    t = {n: dev(getattr(w, n), w.dtype if n in "qkv" else synth.F32)
+         for n in ("q", "k", "v", "eta", "W1", "W2", "W3")}
+    o = torch.empty_like(t["v"])
+    wf = window_flops(w.B, w.H, w.T, w.dk, 4096)
+    run("f4a window attention (w 4096)", {"workload": w.name + "_window4096"},
+        lambda: ops.window_attention_fwd(t["q"], t["k"], t["v"], 4096, out=o), w.B * w.T,
+        ("tensor", wf, pk["bf16_tflops"], "TFLOP/s", "window_attn_kernel"))
+    run("f4a lact + window attention", {"workload": w.name + "_lact_window4096"},
+        lambda: ops.lact_swiglu_window_fwd(t["q"], t["k"], t["v"], t["eta"], t["W1"], t["W2"],
+                                           t["W3"], w.chunk, w.update_rule, 4096, out=o),
+        w.B * w.T,
+        ("tensor", wf + lact_flops(w), pk["bf16_tflops"], "TFLOP/s", "lact step + window"))
+    del t, o
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -462,6 +558,9 @@ def main():
                          "line uses the workload's own length")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-next-rows", action="store_true",
+                    help="skip timing the next rows (backward, momentum, TTT-MLP, window "
+                         "attention, context parallelism), reported under 'next_rows'")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -535,6 +634,8 @@ def main():
     if extras:
         line["workloads"] = extras
         line["gpu_launches"] += sum(x["gpu_launches"] for x in extras)
+    if not args.no_next_rows:
+        line["next_rows"] = measure_next_rows(runner, device)
 
     if rank == 0:
         print(json.dumps(line), flush=True)
