@@ -537,6 +537,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
   __syncthreads();
   umma::fence_after();
   const uint32_t tmem = sm.tmem_base;
+  // launched as a programmatic dependent of the previous kernel of the
+  // stream: the prologue above overlaps its tail; wait for its results here
+  pdl_wait();
+  pdl_trigger();
 
   if (warp == 0) {
     // ---------------- TMA producer: one continuous ring over all tiles ----------------

@@ -67,6 +67,8 @@ struct RowArgs {
 
 // One warp per (z, row of W1 | W3 | W2).
 __global__ void __launch_bounds__(256) lact_rows_kernel(RowArgs a) {
+  pdl_wait();
+  pdl_trigger();
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   const int rows_z = 2 * a.dh + a.dv;
   if (gw >= a.Z * rows_z) return;
@@ -368,6 +370,8 @@ __device__ float block_sum(float v) {
 // the cluster owns rows (tall) or columns (wide) [c L, c L + L) of X.
 __global__ void __cluster_dims__(kNsCluster, 1, 1) __launch_bounds__(kNsThreads)
     ns_kernel(NsArgs a) {
+  pdl_wait();
+  pdl_trigger();
   const int mat = blockIdx.x / kNsCluster, c = blockIdx.x % kNsCluster;
   const int z = mat / 3, m = mat % 3;
   const int R = a.rows[m], C = a.cols[m];
@@ -430,9 +434,14 @@ constexpr int kN5 = 128;          // slab side of the 128 x 512 Newton-Schulz ke
 // ---------------------------------------------------------------------------
 // Newton-Schulz for 128 x 512 (or 512 x 128) gradients on the 5th-generation
 // tensor cores: a cluster of kNsCluster CTAs per matrix, CTA c owning the
-// 128 x 128 slab c of the long side; Gram partials are summed through
-// distributed shared memory (CTA c reduces rows [32c, 32c + 32) of G and writes
-// them into every CTA's copy). X, G and P stay in shared memory as bf16 hi / lo
+// 128 x 128 slab c of the long side. The Gram matrix M = X^T X of the
+// normalised gradient is formed once: partials over the slabs are summed
+// through distributed shared memory (CTA c reduces rows [32c, 32c + 32) and
+// writes them into every CTA's copy). The five iterations then run on the
+// Gram side with no further exchange: a X + b (X X^T) X + c (X X^T)^2 X equals
+// X P with P = a I + b M + c M^2, which commutes with M, so the next Gram
+// matrix is P M P; each CTA updates its own slab and its own copy of M (four
+// 128 x 128 products per iteration). X, M and P stay in shared memory as bf16 hi / lo
 // (x = hi + lo to about 16 bits) in the 128-byte-swizzled layout of two
 // 64-column boxes [128 rows][128 B]; one storage serves as a K-major operand
 // (rows = M or N) and as an MN-major operand (rows = K). Each split product
@@ -485,6 +494,8 @@ __global__ void __cluster_dims__(kNsCluster, 1, 1) __launch_bounds__(kT5Threads,
   __syncthreads();
   umma::fence_after();
   const uint32_t tmem = sm.tmem_base;
+  pdl_wait();
+  pdl_trigger();
 
   // Frobenius norm of the whole matrix (four slabs), then the scaled slab as hi / lo
   // the slab as 8-column pieces (two float4 each), 4 per thread, kept in registers
@@ -602,86 +613,105 @@ __global__ void __cluster_dims__(kNsCluster, 1, 1) __launch_bounds__(kT5Threads,
   uint8_t* const P2[2] = {sm.p[0], sm.p[1]};
   uint8_t* const part = sm.p[0];  // 64 KB: p[0] and p[1] are contiguous
   bool ok = true;
-  for (int it = 0; it < a.steps; ++it) {
-    // Gram partial: tall X^T X (both operands MN-major), wide X X^T (both K-major)
-    ok = product(X2, tall, X2, tall) && ok;
-    {
-      float v[32];
-      acc_load(v);
+  // The Gram matrix of the whole (normalised) X, once: partial over this
+  // CTA's slab (tall X^T X, both operands MN-major; wide X X^T, both
+  // K-major), then CTA c sums rows [32c, 32c + 32) of the four partials and
+  // writes them into every CTA's M (sm.g) as hi / lo.
+  ok = product(X2, tall, X2, tall) && ok;
+  {
+    float v[32];
+    acc_load(v);
 #pragma unroll
-      for (int q = 0; q < 8; ++q)
-        *reinterpret_cast<float4*>(part + t5_part(er, ec / 4 + q)) =
-            make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    for (int q = 0; q < 8; ++q)
+      *reinterpret_cast<float4*>(part + t5_part(er, ec / 4 + q)) =
+          make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+  }
+  umma::fence_before();
+  cluster.sync();
+  {
+    const int r = 32 * c + (tid >> 4), c0 = (tid & 15) * 8;
+    float gsum[8] = {};
+    for (int rk = 0; rk < kNsCluster; ++rk) {
+      const uint8_t* rp = cluster.map_shared_rank(part, rk);
+      const float4 u0 = *reinterpret_cast<const float4*>(rp + t5_part(r, c0 / 4));
+      const float4 u1 = *reinterpret_cast<const float4*>(rp + t5_part(r, c0 / 4 + 1));
+      gsum[0] += u0.x, gsum[1] += u0.y, gsum[2] += u0.z, gsum[3] += u0.w;
+      gsum[4] += u1.x, gsum[5] += u1.y, gsum[6] += u1.z, gsum[7] += u1.w;
     }
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float v0 = gsum[2 * u], v1 = gsum[2 * u + 1];
+      const __nv_bfloat16 h0 = __float2bfloat16_rn(v0), h1 = __float2bfloat16_rn(v1);
+      hi[u] = gemm::pack_bf16x2(__bfloat162float(h0), __bfloat162float(h1));
+      lo[u] = gemm::pack_bf16x2(v0 - __bfloat162float(h0), v1 - __bfloat162float(h1));
+    }
+    for (int rk = 0; rk < kNsCluster; ++rk) {
+      *reinterpret_cast<uint4*>(cluster.map_shared_rank(sm.g[0], rk) + t5_off(r, c0)) =
+          make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      *reinterpret_cast<uint4*>(cluster.map_shared_rank(sm.g[1], rk) + t5_off(r, c0)) =
+          make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    }
+  }
+  cluster.sync();
+  umma::fence_proxy_async_smem();
+  __syncthreads();
+  // The iteration on the Gram side, with no further exchange: with
+  // P = a I + b M + c M^2 (a polynomial in M = X^T X, so symmetric and
+  // commuting with M), a X + b (X X^T) X + c (X X^T)^2 X = X P, and the next
+  // Gram matrix is (X P)^T (X P) = P M P. Each CTA updates its own slab
+  // (X <- X P tall, P X wide) and its own copy of M.
+  auto sync_operands = [&]() {
     umma::fence_before();
-    cluster.sync();
-    // rows [32c, 32c + 32) of G: sum of the four partials, into every CTA's G
-    {
-      const int r = 32 * c + (tid >> 4), c0 = (tid & 15) * 8;
-      float gsum[8] = {};
-      for (int rk = 0; rk < kNsCluster; ++rk) {
-        const uint8_t* rp = cluster.map_shared_rank(part, rk);
-        const float4 u0 = *reinterpret_cast<const float4*>(rp + t5_part(r, c0 / 4));
-        const float4 u1 = *reinterpret_cast<const float4*>(rp + t5_part(r, c0 / 4 + 1));
-        gsum[0] += u0.x, gsum[1] += u0.y, gsum[2] += u0.z, gsum[3] += u0.w;
-        gsum[4] += u1.x, gsum[5] += u1.y, gsum[6] += u1.z, gsum[7] += u1.w;
-      }
-      uint32_t hi[4], lo[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float v0 = gsum[2 * u], v1 = gsum[2 * u + 1];
-        const __nv_bfloat16 h0 = __float2bfloat16_rn(v0), h1 = __float2bfloat16_rn(v1);
-        hi[u] = gemm::pack_bf16x2(__bfloat162float(h0), __bfloat162float(h1));
-        lo[u] = gemm::pack_bf16x2(v0 - __bfloat162float(h0), v1 - __bfloat162float(h1));
-      }
-      for (int rk = 0; rk < kNsCluster; ++rk) {
-        *reinterpret_cast<uint4*>(cluster.map_shared_rank(sm.g[0], rk) + t5_off(r, c0)) =
-            make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4*>(cluster.map_shared_rank(sm.g[1], rk) + t5_off(r, c0)) =
-            make_uint4(lo[0], lo[1], lo[2], lo[3]);
-      }
-    }
-    cluster.sync();
     umma::fence_proxy_async_smem();
     __syncthreads();
-    // P = c G^2 + b G   (A = G K-major, B = G MN-major)
+  };
+  for (int it = 0; it < a.steps; ++it) {
+    // P = a I + b M + c M^2
     ok = product(G2, false, G2, true) && ok;
     {
       float v[32], gv[32];
       acc_load(v);
       val32(G2, er, ec, gv);
 #pragma unroll
-      for (int u = 0; u < 32; ++u) v[u] = a.c * v[u] + a.b * gv[u];
+      for (int u = 0; u < 32; ++u) v[u] = a.c * v[u] + a.b * gv[u] + (ec + u == er ? a.a : 0.f);
       put32(P2, er, ec, v);
     }
-    umma::fence_before();
-    umma::fence_proxy_async_smem();
-    __syncthreads();
-    // X <- a X + X P (tall) or a X + P X (wide)   (B MN-major)
+    sync_operands();
+    // X <- X P (tall) or P X (wide)   (B MN-major)
     if (tall)
       ok = product(X2, false, P2, true) && ok;
     else
       ok = product(P2, false, X2, true) && ok;
     {
-      float v[32], xv[32];
+      float v[32];
       acc_load(v);
-      val32(X2, er, ec, xv);
-#pragma unroll
-      for (int u = 0; u < 32; ++u) v[u] += a.a * xv[u];
       if (it + 1 == a.steps) {
         float4* dst = reinterpret_cast<float4*>(Xc + (int64_t)er * C + ec);
 #pragma unroll
         for (int q = 0; q < 8; ++q)
           dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
       } else {
-        umma::fence_before();
-        __syncthreads();  // every thread has read its old X values
         put32(X2, er, ec, v);
       }
     }
-    umma::fence_before();
-    umma::fence_proxy_async_smem();
-    __syncthreads();
+    if (it + 1 == a.steps) break;
+    sync_operands();
+    // M <- P (M P): T = M P into M's storage, then P T
+    ok = product(G2, false, P2, true) && ok;
+    {
+      float v[32];
+      acc_load(v);
+      put32(G2, er, ec, v);
+    }
+    sync_operands();
+    ok = product(P2, false, G2, true) && ok;
+    {
+      float v[32];
+      acc_load(v);
+      put32(G2, er, ec, v);
+    }
+    sync_operands();
     // A timed-out wait is recorded in the status word; the loop still runs to
     // its end so that every CTA of the cluster meets the same cluster barriers.
   }
@@ -691,6 +721,8 @@ __global__ void __cluster_dims__(kNsCluster, 1, 1) __launch_bounds__(kT5Threads,
 }
 
 __global__ void copy_kernel(float* dst, const float* src, int64_t n) {
+  pdl_wait();
+  pdl_trigger();
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x)
     dst[i] = src[i];
@@ -789,8 +821,7 @@ cudaError_t launch_gemm(Params& P, cudaStream_t s) {
   cudaError_t e = gemm_attr_once();
   if (e != cudaSuccess) return e;
   const int grid = P.total_tiles < num_sms() ? P.total_tiles : num_sms();
-  gemm::gemm_kernel<BN><<<grid, gemm::kThreads, smem, s>>>(P);
-  return cudaGetLastError();
+  return launch_pdl(gemm::gemm_kernel<BN>, dim3(grid), dim3(gemm::kThreads), smem, s, P);
 }
 
 // Operand helpers -----------------------------------------------------------
@@ -1108,7 +1139,8 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
     ok &= buf_op(W13, sc.w13, Z, 2 * dh, 2 * dh, dk, 0, BN, split);
     ok &= buf_op(W13h, sc.w13, Z, 2 * dh, 2 * dh, dk, 0, 2 * gemm::kHid, split);
     ok &= buf_op(W2mn, sc.w2, Z, dv, dv, dh, 1, 64, split);
-    ok &= buf_op(W2k, sc.w2, Z, dv, dv, dh, 0, BN, split);
+    // the Y tiles are only as wide as dv when dv <= 128 (no columns of zeros)
+    ok &= buf_op(W2k, sc.w2, Z, dv, dv, dh, 0, dv <= 128 ? 128 : BN, split);
     ok &= tok_kmajor(Qk0, a.q, a, dk, 0, gemm::BM);
     ok &= tok_kmajor(Kk0, a.k, a, dk, 0, gemm::BM);
     ok &= tok_kmajor(Vk0, a.v, a, dv, 0, gemm::BM);
@@ -1175,6 +1207,7 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
       else
         segs(p, 1, kSegExact);
       p.epi = gemm::EPI_Y;
+      p.tn = dv <= 128 ? 128 : BN;
       p.e = epi_base(a, s0, bc);
       p.e.orow0 = s0;
     };
@@ -1220,6 +1253,7 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
           p.b = Kmn;
           p.M = dh;
           p.N = dk;
+          p.tn = dk <= 128 ? 128 : BN;  // (MN-major B: loaded in 64-column boxes)
           if (split)
             segs(p, 2, kSegAsplit);
           else
@@ -1275,14 +1309,13 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
     // L3 / L4: Muon orthogonalisation, update and row renormalisation
     if (split) {
       if (ns_tc) {
-        ns5_kernel<<<Z * 3 * kNsCluster, kT5Threads, sizeof(Ns5Smem) + 1024, s>>>(na);
+        check(launch_pdl(ns5_kernel, dim3(Z * 3 * kNsCluster), dim3(kT5Threads),
+                         sizeof(Ns5Smem) + 1024, s, na));
       } else {
-        ns_kernel<<<Z * 3 * kNsCluster, kNsThreads, 0, s>>>(na);
+        check(launch_pdl(ns_kernel, dim3(Z * 3 * kNsCluster), dim3(kNsThreads), 0, s, na));
       }
-      check(cudaGetLastError());
     }
-    lact_rows_kernel<<<row_blocks, 256, 0, s>>>(ra);
-    check(cudaGetLastError());
+    check(launch_pdl(lact_rows_kernel, dim3(row_blocks), dim3(256), 0, s, ra));
     if (!a.causal) {
       Params P;
       memset(&P, 0, sizeof(P));
@@ -1300,14 +1333,14 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
   float* finals[3] = {a.W1_final, a.W3_final, a.W2_final};
   for (int m = 0; m < 3 && result == TTT_OK; ++m) {
     if (!finals[m]) continue;
-    copy_kernel<<<148, 256, 0, s>>>(finals[m], sc.Wm[m], Z * nW[m]);
-    check(cudaGetLastError());
+    check(launch_pdl(copy_kernel, dim3(148), dim3(256), 0, s, finals[m], (const float*)sc.Wm[m],
+                     (int64_t)Z * nW[m]));
   }
   float* mfinals[3] = {a.M_final[0], a.M_final[2], a.M_final[1]};
   for (int m = 0; m < 3 && result == TTT_OK && a.momentum; ++m) {
     if (!mfinals[m]) continue;
-    copy_kernel<<<148, 256, 0, s>>>(mfinals[m], sc.M[m], Z * nW[m]);
-    check(cudaGetLastError());
+    check(launch_pdl(copy_kernel, dim3(148), dim3(256), 0, s, mfinals[m], (const float*)sc.M[m],
+                     (int64_t)Z * nW[m]));
   }
   return result;
 }
