@@ -26,6 +26,7 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kTB = 16;
+constexpr int kP = kTB + 1;   // padded token stride of the block buffers
 
 template <typename T>
 __device__ __forceinline__ float ldt(const TokView& v, int b, int h, int64_t t, int c) {
@@ -51,16 +52,19 @@ __global__ void __launch_bounds__(kThreads) ttt_mlp_kernel(MlpArgs a) {
   float* rW2 = rb1 + dh;
   float* rb2 = rW2 + (int64_t)dv * dh;
 
-  float* Qs = smem;              // [16][dk]
-  float* Ks = Qs + kTB * dk;     // [16][dk]
-  float* Vs = Ks + kTB * dk;     // [16][dv]  v, then r
-  float* Hs = Vs + kTB * dv;     // [16][dh]  h, then a = ReLU(h)
-  float* Gs = Hs + kTB * dh;     // [16][dh]  g
-  float* Zs = Gs + kTB * dh;     // [16][dh]  z, then a' = ReLU(z)
-  float* Hm = Zs + kTB * dh;     // [16][dh]  1 where h > 0
-  float* S1 = Hm + kTB * dh;     // [16][16]
-  float* S2 = S1 + kTB * kTB;    // [16][16]
-  float* et = S2 + kTB * kTB;    // [16]
+  // Block buffers, stored transposed with a padded token stride kP, so that
+  // the threads of a warp (which differ in the token or in the feature
+  // index) touch distinct banks: X(i, c) = X[c * kP + i] for token i.
+  float* Qs = smem;                    // [dk][kP]
+  float* Ks = Qs + dk * kP;            // [dk][kP]
+  float* Vs = Ks + dk * kP;            // [dv][kP]  v, then r
+  float* Hs = Vs + dv * kP;            // [dh][kP]  h, then a = ReLU(h)
+  float* Gs = Hs + dh * kP;            // [dh][kP]  g
+  float* Zs = Gs + dh * kP;            // [dh][kP]  z, then a' = ReLU(z)
+  float* Hm = Zs + dh * kP;            // [dh][kP]  1 where h > 0
+  float* S1 = Hm + dh * kP;            // [16][kP]  S1[t][i]
+  float* S2 = S1 + kTB * kP;           // [16][kP]
+  float* et = S2 + kTB * kP;           // [16]
 
   // initial parameters into both copies
   {
@@ -83,12 +87,12 @@ __global__ void __launch_bounds__(kThreads) ttt_mlp_kernel(MlpArgs a) {
       const int nt = min(kTB, ce - t0);
       for (int x = tid; x < kTB * dk; x += kThreads) {
         const int i = x / dk, c = x % dk;
-        Qs[x] = i < nt ? ldt<T>(a.q, b, h, t0 + i, c) : 0.f;
-        Ks[x] = i < nt ? ldt<T>(a.k, b, h, t0 + i, c) : 0.f;
+        Qs[c * kP + i] = i < nt ? ldt<T>(a.q, b, h, t0 + i, c) : 0.f;
+        Ks[c * kP + i] = i < nt ? ldt<T>(a.k, b, h, t0 + i, c) : 0.f;
       }
       for (int x = tid; x < kTB * dv; x += kThreads) {
         const int i = x / dv, c = x % dv;
-        Vs[x] = i < nt ? ldt<T>(a.v, b, h, t0 + i, c) : 0.f;
+        Vs[c * kP + i] = i < nt ? ldt<T>(a.v, b, h, t0 + i, c) : 0.f;
       }
       if (tid < kTB) et[tid] = tid < nt ? eta[(int64_t)(t0 + tid) * a.eta.st] : 0.f;
       __syncthreads();
@@ -99,58 +103,58 @@ __global__ void __launch_bounds__(kThreads) ttt_mlp_kernel(MlpArgs a) {
         const float* w = sW1 + (int64_t)j * dk;
         const float* wr = rW1 + (int64_t)j * dk;
         for (int r = 0; r < dk; ++r) {
-          hk = fmaf(w[r], Ks[i * dk + r], hk);
-          zq = fmaf(wr[r], Qs[i * dk + r], zq);
+          hk = fmaf(w[r], Ks[r * kP + i], hk);
+          zq = fmaf(wr[r], Qs[r * kP + i], zq);
         }
-        Hs[i * dh + j] = fmaxf(hk, 0.f);
-        Hm[i * dh + j] = hk > 0.f ? 1.f : 0.f;
-        Zs[i * dh + j] = zq;
+        Hs[j * kP + i] = fmaxf(hk, 0.f);
+        Hm[j * kP + i] = hk > 0.f ? 1.f : 0.f;
+        Zs[j * kP + i] = zq;
       }
       // S1[t][i] = q_t . k_i + 1 (i <= t)
       {
         const int t = tid / kTB, i = tid % kTB;
-        float s = 0.f;
+        float sv = 0.f;
         if (i <= t) {
-          s = 1.f;
-          for (int r = 0; r < dk; ++r) s = fmaf(Qs[t * dk + r], Ks[i * dk + r], s);
+          sv = 1.f;
+          for (int r = 0; r < dk; ++r) sv = fmaf(Qs[r * kP + t], Ks[r * kP + i], sv);
         }
-        S1[tid] = s;
+        S1[t * kP + i] = sv;
       }
       __syncthreads();
       // r = W2_s a + b2_s - v
       for (int x = tid; x < kTB * dv; x += kThreads) {
         const int c = x / kTB, i = x % kTB;
-        float s = sb2[c];
+        float sv = sb2[c];
         const float* w = sW2 + (int64_t)c * dh;
-        for (int j = 0; j < dh; ++j) s = fmaf(w[j], Hs[i * dh + j], s);
-        Vs[i * dv + c] = s - Vs[i * dv + c];
+        for (int j = 0; j < dh; ++j) sv = fmaf(w[j], Hs[j * kP + i], sv);
+        Vs[c * kP + i] = sv - Vs[c * kP + i];
       }
       __syncthreads();
       // g = (W2_s^T r) [h > 0]
       for (int x = tid; x < kTB * dh; x += kThreads) {
         const int j = x / kTB, i = x % kTB;
-        float s = 0.f;
-        for (int c = 0; c < dv; ++c) s = fmaf(sW2[(int64_t)c * dh + j], Vs[i * dv + c], s);
-        Gs[i * dh + j] = s * Hm[i * dh + j];
+        float sv = 0.f;
+        for (int c = 0; c < dv; ++c) sv = fmaf(sW2[(int64_t)c * dh + j], Vs[c * kP + i], sv);
+        Gs[j * kP + i] = sv * Hm[j * kP + i];
       }
       __syncthreads();
       // z = z0 - sum_{i<=t} eta_i S1[t][i] g_i ; a' = ReLU(z)
       for (int x = tid; x < kTB * dh; x += kThreads) {
         const int t = x / dh, j = x % dh;
-        float z = Zs[x];
-        for (int i = 0; i <= t; ++i) z = fmaf(-et[i] * S1[t * kTB + i], Gs[i * dh + j], z);
-        Zs[x] = fmaxf(z, 0.f);
+        float z = Zs[j * kP + t];
+        for (int i = 0; i <= t; ++i) z = fmaf(-et[i] * S1[t * kP + i], Gs[j * kP + i], z);
+        Zs[j * kP + t] = fmaxf(z, 0.f);
       }
       __syncthreads();
       // S2[t][i] = a'_t . a_i + 1 (i <= t)
       {
         const int t = tid / kTB, i = tid % kTB;
-        float s = 0.f;
+        float sv = 0.f;
         if (i <= t) {
-          s = 1.f;
-          for (int j = 0; j < dh; ++j) s = fmaf(Zs[t * dh + j], Hs[i * dh + j], s);
+          sv = 1.f;
+          for (int j = 0; j < dh; ++j) sv = fmaf(Zs[j * kP + t], Hs[j * kP + i], sv);
         }
-        S2[tid] = s;
+        S2[t * kP + i] = sv;
       }
       __syncthreads();
       // y = W2_run a' + b2_run - sum_{i<=t} eta_i S2[t][i] r_i
@@ -159,8 +163,8 @@ __global__ void __launch_bounds__(kThreads) ttt_mlp_kernel(MlpArgs a) {
         if (t < nt) {
           float y = rb2[c];
           const float* w = rW2 + (int64_t)c * dh;
-          for (int j = 0; j < dh; ++j) y = fmaf(w[j], Zs[t * dh + j], y);
-          for (int i = 0; i <= t; ++i) y = fmaf(-et[i] * S2[t * kTB + i], Vs[i * dv + c], y);
+          for (int j = 0; j < dh; ++j) y = fmaf(w[j], Zs[j * kP + t], y);
+          for (int i = 0; i <= t; ++i) y = fmaf(-et[i] * S2[t * kP + i], Vs[c * kP + i], y);
           T* o = static_cast<T*>(a.out.p) + b * a.out.sb + h * a.out.sh + (int64_t)(t0 + t) * a.out.st;
           o[c] = T(y);
         }
@@ -169,25 +173,25 @@ __global__ void __launch_bounds__(kThreads) ttt_mlp_kernel(MlpArgs a) {
       // running parameters: subtract this block's eta-weighted gradients
       for (int64_t x = tid; x < (int64_t)dh * dk; x += kThreads) {
         const int j = (int)(x / dk), r = (int)(x % dk);
-        float s = 0.f;
-        for (int i = 0; i < nt; ++i) s = fmaf(et[i] * Gs[i * dh + j], Ks[i * dk + r], s);
-        rW1[x] -= s;
+        float sv = 0.f;
+        for (int i = 0; i < nt; ++i) sv = fmaf(et[i] * Gs[j * kP + i], Ks[r * kP + i], sv);
+        rW1[x] -= sv;
       }
       for (int j = tid; j < dh; j += kThreads) {
-        float s = 0.f;
-        for (int i = 0; i < nt; ++i) s = fmaf(et[i], Gs[i * dh + j], s);
-        rb1[j] -= s;
+        float sv = 0.f;
+        for (int i = 0; i < nt; ++i) sv = fmaf(et[i], Gs[j * kP + i], sv);
+        rb1[j] -= sv;
       }
       for (int64_t x = tid; x < (int64_t)dv * dh; x += kThreads) {
         const int c = (int)(x / dh), j = (int)(x % dh);
-        float s = 0.f;
-        for (int i = 0; i < nt; ++i) s = fmaf(et[i] * Vs[i * dv + c], Hs[i * dh + j], s);
-        rW2[x] -= s;
+        float sv = 0.f;
+        for (int i = 0; i < nt; ++i) sv = fmaf(et[i] * Vs[c * kP + i], Hs[j * kP + i], sv);
+        rW2[x] -= sv;
       }
       for (int c = tid; c < dv; c += kThreads) {
-        float s = 0.f;
-        for (int i = 0; i < nt; ++i) s = fmaf(et[i], Vs[i * dv + c], s);
-        rb2[c] -= s;
+        float sv = 0.f;
+        for (int i = 0; i < nt; ++i) sv = fmaf(et[i], Vs[c * kP + i], sv);
+        rb2[c] -= sv;
       }
       __syncthreads();
     }
@@ -214,8 +218,7 @@ size_t ttt_mlp_workspace(const MlpArgs& a) {
 }
 
 cudaError_t launch_ttt_mlp(const MlpArgs& a, bool bf16, cudaStream_t s) {
-  const size_t smem = sizeof(float) * (2 * kTB * a.dk + kTB * a.dv + 4 * kTB * a.dh +
-                                       2 * kTB * kTB + kTB);
+  const size_t smem = sizeof(float) * ((2 * a.dk + a.dv + 4 * a.dh) * kP + 2 * kTB * kP + kTB);
   cudaError_t e;
   if (bf16) {
     e = cudaFuncSetAttribute(ttt_mlp_kernel<__nv_bfloat16>,
