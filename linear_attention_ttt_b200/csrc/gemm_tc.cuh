@@ -122,6 +122,16 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// bf16 hi / lo parts of (a, b) as two packed words: hi = bf16(x) (round to
+// nearest even), lo = bf16(x - hi). One paired conversion per part: a bf16 is
+// the upper half of the float with the same value, so the float value of each
+// hi half is recovered from the packed word by a shift or a mask. Equal to
+// converting hi and lo element by element, with half the conversions.
+__device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  hi = pack_bf16x2(a, b);
+  lo = pack_bf16x2(a - __uint_as_float(hi << 16), b - __uint_as_float(hi & 0xffff0000u));
+}
+
 // Row `lane` of the buffer, columns [16p, 16p + 16) as bf16 (chunks 2p, 2p+1):
 // bf16(v), or the residual v - bf16(v) for LO.
 template <bool LO>
@@ -204,6 +214,17 @@ __device__ __forceinline__ void put_bf16_64(uint8_t* s, int lane, int p, const f
   }
   *reinterpret_cast<uint4*>(s + sw64(lane, 2 * p)) = make_uint4(w[0], w[1], w[2], w[3]);
   *reinterpret_cast<uint4*>(s + sw64(lane, 2 * p + 1)) = make_uint4(w[4], w[5], w[6], w[7]);
+}
+// put_bf16_64<false> into sh and put_bf16_64<true> into sl, one conversion per part.
+__device__ __forceinline__ void put_split_64(uint8_t* sh, uint8_t* sl, int lane, int p,
+                                             const float (&v)[16]) {
+  uint32_t h[8], l[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) split_bf16x2(v[2 * u], v[2 * u + 1], h[u], l[u]);
+  *reinterpret_cast<uint4*>(sh + sw64(lane, 2 * p)) = make_uint4(h[0], h[1], h[2], h[3]);
+  *reinterpret_cast<uint4*>(sh + sw64(lane, 2 * p + 1)) = make_uint4(h[4], h[5], h[6], h[7]);
+  *reinterpret_cast<uint4*>(sl + sw64(lane, 2 * p)) = make_uint4(l[0], l[1], l[2], l[3]);
+  *reinterpret_cast<uint4*>(sl + sw64(lane, 2 * p + 1)) = make_uint4(l[4], l[5], l[6], l[7]);
 }
 // Staged rows r < nrows (64 bytes each) -> dst + r * ld: eight rows per store.
 __device__ __forceinline__ void flush_rows64(const uint8_t* s, int lane, uint8_t* dst, int64_t ld,
@@ -398,11 +419,12 @@ __device__ __forceinline__ void epilogue_body(const Problem& pr, const TileCoord
         a[u] = eta_i * s1 * h3[u];
         d[u] = gz[u] * s1;
       }
-      put_bf16_64<false>(bA, lane, p, a);
-      if constexpr (SPLIT)
-        put_bf16_64<true>(bB, lane, p, a);
-      else
+      if constexpr (SPLIT) {
+        put_split_64(bA, bB, lane, p, a);
+      } else {
+        put_bf16_64<false>(bA, lane, p, a);
         put_bf16_64<false>(bB, lane, p, d);
+      }
     }
     flush_rows64(bA, lane, dst(0), ld, nrows);
     flush_rows64(bB, lane, dst(SPLIT ? 3 : 2), ld, nrows);
@@ -414,8 +436,7 @@ __device__ __forceinline__ void epilogue_body(const Problem& pr, const TileCoord
         load3(p, h1, h3, gz);
 #pragma unroll
         for (int u = 0; u < 16; ++u) d[u] = gz[u] * h1[u] * sgm[p][u];
-        put_bf16_64<false>(bA, lane, p, d);
-        put_bf16_64<true>(bB, lane, p, d);
+        put_split_64(bA, bB, lane, p, d);
       }
       flush_rows64(bA, lane, dst(2), ld, nrows);
       flush_rows64(bB, lane, dst(5), ld, nrows);
@@ -430,8 +451,10 @@ __device__ __forceinline__ void epilogue_body(const Problem& pr, const TileCoord
         const float sg1 = sgm[p][u];
         d[u] = gz[u] * h3[u] * sg1 * (1.f + h1[u] * (1.f - sg1));
       }
-      put_bf16_64<false>(bA, lane, p, d);
-      if constexpr (SPLIT) put_bf16_64<true>(bB, lane, p, d);
+      if constexpr (SPLIT)
+        put_split_64(bA, bB, lane, p, d);
+      else
+        put_bf16_64<false>(bA, lane, p, d);
     }
     flush_rows64(bA, lane, dst(1), ld, nrows);
     if constexpr (SPLIT) flush_rows64(bB, lane, dst(4), ld, nrows);

@@ -165,18 +165,11 @@ __global__ void __launch_bounds__(256) lact_rows_kernel(RowArgs a) {
       const float4 x = make_float4(v[i].x * s, v[i].y * s, v[i].z * s, v[i].w * s);
       *reinterpret_cast<float4*>(W + c) = x;
       *reinterpret_cast<float4*>(G + c) = make_float4(0.f, 0.f, 0.f, 0.f);
-      const __nv_bfloat16 h0 = __float2bfloat16_rn(x.x), h1 = __float2bfloat16_rn(x.y);
-      const __nv_bfloat16 h2 = __float2bfloat16_rn(x.z), h3 = __float2bfloat16_rn(x.w);
-      __nv_bfloat162 p0, p1;
-      p0.x = h0, p0.y = h1, p1.x = h2, p1.y = h3;
-      *reinterpret_cast<uint2*>(hi + c) =
-          make_uint2(*reinterpret_cast<uint32_t*>(&p0), *reinterpret_cast<uint32_t*>(&p1));
-      if (a.split) {
-        __nv_bfloat162 q0 = __floats2bfloat162_rn(x.x - __bfloat162float(h0), x.y - __bfloat162float(h1));
-        __nv_bfloat162 q1 = __floats2bfloat162_rn(x.z - __bfloat162float(h2), x.w - __bfloat162float(h3));
-        *reinterpret_cast<uint2*>(lo + c) =
-            make_uint2(*reinterpret_cast<uint32_t*>(&q0), *reinterpret_cast<uint32_t*>(&q1));
-      }
+      uint32_t h0, h1, l0, l1;
+      gemm::split_bf16x2(x.x, x.y, h0, l0);
+      gemm::split_bf16x2(x.z, x.w, h1, l1);
+      *reinterpret_cast<uint2*>(hi + c) = make_uint2(h0, h1);
+      if (a.split) *reinterpret_cast<uint2*>(lo + c) = make_uint2(l0, l1);
     }
     return;
   }
@@ -525,11 +518,7 @@ __global__ void __cluster_dims__(kNsCluster, 1, 1) __launch_bounds__(kT5Threads,
     uint32_t hi[4], lo[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const float v0 = xv[2 * u] * inv;
-      const float v1 = xv[2 * u + 1] * inv;
-      const __nv_bfloat16 h0 = __float2bfloat16_rn(v0), h1 = __float2bfloat16_rn(v1);
-      hi[u] = gemm::pack_bf16x2(__bfloat162float(h0), __bfloat162float(h1));
-      lo[u] = gemm::pack_bf16x2(v0 - __bfloat162float(h0), v1 - __bfloat162float(h1));
+      gemm::split_bf16x2(xv[2 * u] * inv, xv[2 * u + 1] * inv, hi[u], lo[u]);
     }
     *reinterpret_cast<uint4*>(sm.x[0] + t5_off(r, c0)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
     *reinterpret_cast<uint4*>(sm.x[1] + t5_off(r, c0)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
@@ -598,10 +587,7 @@ __global__ void __cluster_dims__(kNsCluster, 1, 1) __launch_bounds__(kT5Threads,
       uint32_t hi[4], lo[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const float v0 = v[8 * q + 2 * u], v1 = v[8 * q + 2 * u + 1];
-        const __nv_bfloat16 h0 = __float2bfloat16_rn(v0), h1 = __float2bfloat16_rn(v1);
-        hi[u] = gemm::pack_bf16x2(__bfloat162float(h0), __bfloat162float(h1));
-        lo[u] = gemm::pack_bf16x2(v0 - __bfloat162float(h0), v1 - __bfloat162float(h1));
+        gemm::split_bf16x2(v[8 * q + 2 * u], v[8 * q + 2 * u + 1], hi[u], lo[u]);
       }
       *reinterpret_cast<uint4*>(S[0] + t5_off(r, cc + 8 * q)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
       *reinterpret_cast<uint4*>(S[1] + t5_off(r, cc + 8 * q)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
@@ -641,10 +627,7 @@ __global__ void __cluster_dims__(kNsCluster, 1, 1) __launch_bounds__(kT5Threads,
     uint32_t hi[4], lo[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const float v0 = gsum[2 * u], v1 = gsum[2 * u + 1];
-      const __nv_bfloat16 h0 = __float2bfloat16_rn(v0), h1 = __float2bfloat16_rn(v1);
-      hi[u] = gemm::pack_bf16x2(__bfloat162float(h0), __bfloat162float(h1));
-      lo[u] = gemm::pack_bf16x2(v0 - __bfloat162float(h0), v1 - __bfloat162float(h1));
+      gemm::split_bf16x2(gsum[2 * u], gsum[2 * u + 1], hi[u], lo[u]);
     }
     for (int rk = 0; rk < kNsCluster; ++rk) {
       *reinterpret_cast<uint4*>(cluster.map_shared_rank(sm.g[0], rk) + t5_off(r, c0)) =
