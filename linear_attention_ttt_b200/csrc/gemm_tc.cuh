@@ -87,8 +87,18 @@ struct Problem {
   int M, N, K;      // K per segment (both products)
   int tn;           // tile width in columns of the first product (<= BN)
   int nseg, nseg2;
+  // 0: one ring stage per segment and K block. 1: the two segments of each
+  // product share A (maps seg_a[0] = seg_a[1]; B maps hi, lo): one stage holds
+  // A, B0 and B1 (B1 at b + bn*BK*2). 2: they share B (A maps hi, lo): one
+  // stage holds A0, B and A1 (A1 at b + bn*BK*2). Pairs need bn <= 128.
+  int pair;
   int seg_a[3], seg_b[3], seg2_a[3], seg2_b[3];
   int nz, ksplit, mtiles, ntiles, tile_begin;
+  // filled by fill_problem_tiles on the host: K blocks in total and per split,
+  // and reciprocal multipliers ceil(2^32 / d) of ntiles, mtiles and ksplit, so
+  // that the single-thread roles decode tiles without integer division
+  int kblocks, kb_per;
+  uint64_t mag_n, mag_m, mag_k;
   int epi;
   EpiArgs e;
 };
@@ -284,21 +294,26 @@ struct TileCoord {
   int pi, z, ks, m0, n0;
 };
 
+// floor(n / d) from mag = ceil(2^32 / d); exact for n * d < 2^32 (tile
+// indices and counts here are far below 2^16).
+__device__ __forceinline__ int div_mag(int n, uint64_t mag) {
+  return (int)(((uint64_t)(uint32_t)n * mag) >> 32);
+}
+
 __device__ __forceinline__ TileCoord decode_tile(const Params& P, int t) {
   TileCoord c;
   int pi = 0;
   while (pi + 1 < P.nprob && t >= P.p[pi + 1].tile_begin) ++pi;
   const Problem& pr = P.p[pi];
-  int local = t - pr.tile_begin;
-  const int nt = local % pr.ntiles;
-  local /= pr.ntiles;
-  const int mt = local % pr.mtiles;
-  local /= pr.mtiles;
+  const int local = t - pr.tile_begin;
+  const int q1 = div_mag(local, pr.mag_n);
+  const int q2 = div_mag(q1, pr.mag_m);
+  const int z = div_mag(q2, pr.mag_k);
   c.pi = pi;
-  c.ks = local % pr.ksplit;
-  c.z = local / pr.ksplit;
-  c.m0 = mt * BM;
-  c.n0 = nt;  // n-tile index; the kernel scales it by the problem's tile width
+  c.z = z;
+  c.ks = q2 - z * pr.ksplit;
+  c.m0 = (q1 - q2 * pr.mtiles) * BM;
+  c.n0 = local - q1 * pr.ntiles;  // n-tile index; the kernel scales it by the problem's tile width
   return c;
 }
 
@@ -327,10 +342,8 @@ __device__ __forceinline__ float eta_of(const EpiArgs& e, int z, int row) {
 
 // K-block range of one tile (one K split of it).
 __device__ __forceinline__ void k_range(const Problem& pr, int ks, int& kb0, int& nk) {
-  const int kblocks = (pr.K + BK - 1) / BK;
-  const int kb_per = (kblocks + pr.ksplit - 1) / pr.ksplit;
-  kb0 = ks * kb_per;
-  nk = max(0, min(kblocks, kb0 + kb_per) - kb0);
+  kb0 = ks * pr.kb_per;
+  nk = max(0, min(pr.kblocks, kb0 + pr.kb_per) - kb0);
 }
 
 // Epilogue of one accumulator tile, run by one warp: its 32 TMEM lanes (tile
@@ -565,6 +578,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
   pdl_wait();
   pdl_trigger();
 
+  int* const status = P.status;
+
+  // The producer and the MMA issuer are single threads on the critical path:
+  // per pass (one segment, or the two segments of a pair) they copy what they
+  // need from the problem into registers, because every asm statement below
+  // clobbers memory and would make the compiler re-read parameter space.
   if (warp == 0) {
     // ---------------- TMA producer: one continuous ring over all tiles ----------------
     if (lane == 0) {
@@ -575,37 +594,56 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         const Problem& pr = P.p[tc.pi];
         int kb0, nk;
         k_range(pr, tc.ks, kb0, nk);
-        const int tn = pr.tn, n0 = tc.n0 * tn, m0 = tc.m0;
-        for (int seg = 0; seg < pr.nseg + pr.nseg2 && ok; ++seg) {
-          const bool second = seg >= pr.nseg;
+        const int tn = pr.tn, n0 = tc.n0 * tn, m0 = tc.m0, pair = pr.pair, nseg = pr.nseg;
+        // passes: one per segment, or one per product when its segments are paired
+        const int npass = pair ? (pr.nseg2 ? 2 : 1) : nseg + pr.nseg2;
+        for (int ps = 0; ps < npass && ok; ++ps) {
+          const bool second = pair ? ps == 1 : ps >= nseg;
+          const int s0 = pair ? 0 : (second ? ps - nseg : ps);
           const Operand& A = second ? pr.a2 : pr.a;
           const Operand& B = second ? pr.b2 : pr.b;
-          const CUtensorMap* am = &A.map[second ? pr.seg2_a[seg - pr.nseg] : pr.seg_a[seg]];
-          const CUtensorMap* bm = &B.map[second ? pr.seg2_b[seg - pr.nseg] : pr.seg_b[seg]];
+          const int* sa = second ? pr.seg2_a : pr.seg_a;
+          const int* sb = second ? pr.seg2_b : pr.seg_b;
+          const CUtensorMap* const am = &A.map[sa[s0]];
+          const CUtensorMap* const bm = &B.map[sb[s0]];
+          // the other part of a pair: B lo (pair 1) or A lo (pair 2)
+          const CUtensorMap* const m1 = pair == 1 ? &B.map[sb[1]] : &A.map[sa[1]];
+          const int a_mn = A.mn_major, b_mn = B.mn_major, arow = A.row0, brow = B.row0;
           const int bn = second ? tn / 2 : tn;   // B rows (columns of this product)
           const int bn0 = second ? n0 / 2 : n0;
+          const int bbytes = bn * BK * 2;
+          const int na = pair == 2 ? 2 : 1, nb = pair == 1 ? 2 : 1;
+          const uint32_t tx = (uint32_t)(na * BM * BK * 2 + nb * bbytes);
           const int az2 = tc.z % A.zdiv, az3 = tc.z / A.zdiv, bz2 = tc.z % B.zdiv,
                     bz3 = tc.z / B.zdiv;
           for (int kb = kb0; kb < kb0 + nk; ++kb, ++it) {
             const int st = it % kStages;
-            if (it >= kStages && !mbar_wait(&sm.empty[st], ((it / kStages) - 1) & 1, P.status)) {
+            if (it >= kStages && !mbar_wait(&sm.empty[st], ((it / kStages) - 1) & 1, status)) {
               ok = false;
               break;
             }
             const int k = kb * BK;
-            mbar_arrive_expect_tx(&sm.full[st], (BM + bn) * BK * 2);
-            if (!A.mn_major) {
-              tma_load_4d(sm.a[st], am, &sm.full[st], k, A.row0 + m0, az2, az3);
-            } else {
-              tma_load_4d(sm.a[st], am, &sm.full[st], m0, A.row0 + k, az2, az3);
-              tma_load_4d(sm.a[st] + 8192, am, &sm.full[st], m0 + 64, A.row0 + k, az2, az3);
+            uint64_t* const full = &sm.full[st];
+            mbar_arrive_expect_tx(full, tx);
+            for (int x = 0; x < na; ++x) {  // A, then A lo of a pair at b + bbytes
+              uint8_t* const dst = x ? sm.b[st] + bbytes : sm.a[st];
+              const CUtensorMap* const map = x ? m1 : am;
+              if (!a_mn) {
+                tma_load_4d(dst, map, full, k, arow + m0, az2, az3);
+              } else {
+                tma_load_4d(dst, map, full, m0, arow + k, az2, az3);
+                tma_load_4d(dst + 8192, map, full, m0 + 64, arow + k, az2, az3);
+              }
             }
-            if (!B.mn_major) {
-              tma_load_4d(sm.b[st], bm, &sm.full[st], k, B.row0 + bn0, bz2, bz3);
-            } else {
-              for (int x = 0; x < bn / 64; ++x)
-                tma_load_4d(sm.b[st] + x * 8192, bm, &sm.full[st], bn0 + 64 * x, B.row0 + k, bz2,
-                            bz3);
+            for (int x = 0; x < nb; ++x) {  // B, then B lo of a pair at b + bbytes
+              uint8_t* const dst = sm.b[st] + (x ? bbytes : 0);
+              const CUtensorMap* const map = x ? m1 : bm;
+              if (!b_mn) {
+                tma_load_4d(dst, map, full, k, brow + bn0, bz2, bz3);
+              } else {
+                for (int y = 0; y < bn / 64; ++y)
+                  tma_load_4d(dst + y * 8192, map, full, bn0 + 64 * y, brow + k, bz2, bz3);
+              }
             }
           }
         }
@@ -621,33 +659,47 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         const Problem& pr = P.p[tc.pi];
         int kb0, nk;
         k_range(pr, tc.ks, kb0, nk);
+        const int tn = pr.tn, pair = pr.pair, nseg = pr.nseg;
+        const int npass = pair ? (pr.nseg2 ? 2 : 1) : nseg + pr.nseg2;
         const int ab = lt & 1;
-        if (lt >= 2 && !mbar_wait(&sm.acc_empty[ab], ((lt >> 1) - 1) & 1, P.status)) break;
+        if (lt >= 2 && !mbar_wait(&sm.acc_empty[ab], ((lt >> 1) - 1) & 1, status)) break;
         umma::fence_after();
         const uint32_t dacc = tmem + ab * BN;
-        for (int seg = 0; seg < pr.nseg + pr.nseg2 && ok; ++seg) {
-          const bool second = seg >= pr.nseg;
-          const Operand& A = second ? pr.a2 : pr.a;
-          const Operand& B = second ? pr.b2 : pr.b;
-          const uint32_t d = dacc + (second ? pr.tn : 0);
-          const uint32_t idesc =
-              umma::instr_desc(1, BM, second ? pr.tn / 2 : pr.tn, A.mn_major, B.mn_major);
-          const bool first_seg = seg == 0 || seg == pr.nseg;  // accumulator starts at zero
+        for (int ps = 0; ps < npass && ok; ++ps) {
+          const bool second = pair ? ps == 1 : ps >= nseg;
+          const int a_mn = (second ? pr.a2 : pr.a).mn_major;
+          const int b_mn = (second ? pr.b2 : pr.b).mn_major;
+          const int bn = second ? tn / 2 : tn;
+          const uint32_t bpart = (uint32_t)(bn * BK * 2) >> 4;  // offset of a pair's second part, 16 B units
+          const uint32_t d = dacc + (second ? tn : 0);
+          const uint32_t idesc = umma::instr_desc(1, BM, bn, a_mn, b_mn);
+          // descriptors: fixed fields | start address, K steps of 16 as address
+          // increments (2 KB for an MN-major operand, 32 B for a K-major one)
+          const uint64_t abase = a_mn ? umma::smem_desc_base(8192, 1024) : umma::smem_desc_base(16, 1024);
+          const uint64_t bbase = b_mn ? umma::smem_desc_base(8192, 1024) : umma::smem_desc_base(16, 1024);
+          const uint32_t astep = a_mn ? 128u : 2u, bstep = b_mn ? 128u : 2u;
+          // the accumulator (region) starts at zero with the product's first MMA
+          const bool first = pair || ps == 0 || ps == nseg;
           for (int i = 0; i < nk; ++i, ++it) {
             const int st = it % kStages;
-            if (!mbar_wait(&sm.full[st], (it / kStages) & 1, P.status)) {
+            if (!mbar_wait(&sm.full[st], (it / kStages) & 1, status)) {
               ok = false;
               break;
             }
             umma::fence_after();
-            const uint32_t sa = smem_u32(sm.a[st]), sb = smem_u32(sm.b[st]);
+            const uint32_t sa = (smem_u32(sm.a[st]) >> 4) & 0x3FFF;
+            const uint32_t sb = (smem_u32(sm.b[st]) >> 4) & 0x3FFF;
+            const uint64_t ad = abase | sa, bd = bbase | sb;
 #pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk) {
-              const uint64_t ad = A.mn_major ? umma::smem_desc(sa + kk * 2048, 8192, 1024)
-                                             : umma::smem_desc(sa + kk * 32, 16, 1024);
-              const uint64_t bd = B.mn_major ? umma::smem_desc(sb + kk * 2048, 8192, 1024)
-                                             : umma::smem_desc(sb + kk * 32, 16, 1024);
-              umma::mma_bf16(d, ad, bd, idesc, (!first_seg || i > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < BK / 16; ++kk)
+              umma::mma_bf16(d, ad + kk * astep, bd + kk * bstep, idesc,
+                             (!first || i > 0 || kk > 0) ? 1u : 0u);
+            if (pair) {  // the second part: A with B lo (pair 1) or A lo with B (pair 2)
+              const uint64_t ad1 = pair == 2 ? abase | (sb + bpart) : ad;
+              const uint64_t bd1 = pair == 1 ? bbase | (sb + bpart) : bd;
+#pragma unroll
+              for (int kk = 0; kk < BK / 16; ++kk)
+                umma::mma_bf16(d, ad1 + kk * astep, bd1 + kk * bstep, idesc, 1u);
             }
             umma::commit(&sm.empty[st]);
           }
@@ -668,7 +720,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
       int kb0, nk;
       k_range(pr, tc.ks, kb0, nk);
       const int ab = lt & 1;
-      const bool waited = mbar_wait(&sm.acc_full[ab], (lt >> 1) & 1, P.status);
+      const bool waited = mbar_wait(&sm.acc_full[ab], (lt >> 1) & 1, status);
       umma::fence_after();
       const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + ab * BN;
       epilogue_tile<BN>(pr, tc, quarter, tbase, waited && nk > 0, ch, sgr);

@@ -766,6 +766,12 @@ void fill_problem_tiles(Params& P) {
     p.mtiles = (p.M + gemm::BM - 1) / gemm::BM;
     p.ntiles = (p.N + p.tn - 1) / p.tn;
     p.tile_begin = t;
+    p.kblocks = (p.K + gemm::BK - 1) / gemm::BK;
+    p.kb_per = (p.kblocks + p.ksplit - 1) / p.ksplit;
+    auto mag = [](int d) { return ((uint64_t(1) << 32) + (uint64_t)d - 1) / (uint64_t)d; };
+    p.mag_n = mag(p.ntiles);
+    p.mag_m = mag(p.mtiles);
+    p.mag_k = mag(p.ksplit);
     t += p.nz * p.ksplit * p.mtiles * p.ntiles;
   }
   P.total_tiles = t;
@@ -1191,6 +1197,7 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
         segs(p, 1, kSegExact);
       p.epi = gemm::EPI_Y;
       p.tn = dv <= 128 ? 128 : BN;
+      p.pair = split && p.tn <= 128 ? 1 : 0;  // Aq loaded once for both W2 parts
       p.e = epi_base(a, s0, bc);
       p.e.orow0 = s0;
     };
@@ -1211,6 +1218,7 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
         p.seg2_b[i] = segW[2 * i + 1];
       }
       p.epi = gemm::EPI_HKG;
+      p.pair = split ? 1 : 0;  // K (and V) loaded once for the hi and lo weight parts
       p.e = epi_base(a, s0, bc);
       p.e.nsplit = split ? 2 : 1;
       for (int x = 0; x < (split ? 2 : 1); ++x) {
@@ -1241,6 +1249,7 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
             segs(p, 2, kSegAsplit);
           else
             segs(p, 1, kSegExact);
+          p.pair = split && p.tn <= 128 ? 2 : 0;  // K loaded once for the dH hi and lo parts
           p.e = epi_base(a, s0, dh);
           p.e.ozdiv = Z;
           p.e.gmap = gmaps[g];

@@ -26,6 +26,13 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
   return d;
 }
 
+// smem_desc without the start address: smem_desc(a, l, s) == smem_desc_base(l, s) | ((a >> 4) & 0x3FFF).
+// Adding n to such a descriptor advances its start address by 16 n bytes.
+__host__ __device__ constexpr uint64_t smem_desc_base(uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  return ((uint64_t)((lbo_bytes >> 4) & 0x3FFF) << 16) |
+         ((uint64_t)((sbo_bytes >> 4) & 0x3FFF) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
 // Instruction descriptor: fp32 accumulate, bf16 x bf16 (fmt 1) or tf32 (fmt 2).
 __host__ __device__ constexpr uint32_t instr_desc(int fmt, int M, int N, int a_mn_major,
                                                   int b_mn_major) {
