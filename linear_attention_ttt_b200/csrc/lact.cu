@@ -449,7 +449,7 @@ struct Ns5Smem {
   alignas(1024) uint8_t x[2][2 * kT5Box];  // [hi|lo]
   alignas(1024) uint8_t g[2][2 * kT5Box];
   alignas(1024) uint8_t p[2][2 * kT5Box];  // also the fp32 Gram partial [128][128]
-  uint64_t mma_done;
+  uint64_t mma_done[2];  // one per TMEM accumulator
   uint32_t tmem_base;
   float nrm;
 };
@@ -479,10 +479,11 @@ __global__ void __cluster_dims__(kNsCluster, 1, 1) __launch_bounds__(kT5Threads,
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (tid == 0) {
-    mbar_init(&sm.mma_done, 1);
+    mbar_init(&sm.mma_done[0], 1);
+    mbar_init(&sm.mma_done[1], 1);
     fence_mbar_init();
   }
-  if (warp == 0) umma::tmem_alloc(&sm.tmem_base, 128);
+  if (warp == 0) umma::tmem_alloc(&sm.tmem_base, 256);  // two 128-column accumulators
   umma::fence_before();
   __syncthreads();
   umma::fence_after();
@@ -526,10 +527,12 @@ __global__ void __cluster_dims__(kNsCluster, 1, 1) __launch_bounds__(kT5Threads,
   umma::fence_proxy_async_smem();
   __syncthreads();
 
-  // One split product into the accumulator: A, B given as [hi, lo] storages and
-  // whether each is read MN-major (rows = K) or K-major (rows = M or N).
-  int phase = 0;
-  auto product = [&](uint8_t* const (&A)[2], bool a_mn, uint8_t* const (&B)[2], bool b_mn) {
+  // One split product into accumulator `acc` (0 or 1): A, B given as [hi, lo]
+  // storages and whether each is read MN-major (rows = K) or K-major (rows =
+  // M or N). issue() enqueues the 24 MMAs from one thread and commits them to
+  // the accumulator's barrier; wait() blocks every thread until they are done.
+  int phase[2] = {0, 0};
+  auto issue = [&](uint8_t* const (&A)[2], bool a_mn, uint8_t* const (&B)[2], bool b_mn, int acc) {
     if (tid == 0) {
       umma::fence_after();
       const uint32_t idesc = umma::instr_desc(1, kN5, kN5, a_mn, b_mn);
@@ -542,23 +545,29 @@ __global__ void __cluster_dims__(kNsCluster, 1, 1) __launch_bounds__(kT5Threads,
                                    : umma::smem_desc(sa + (kk >> 2) * kT5Box + (kk & 3) * 32, 16, 1024);
           const uint64_t bd = b_mn ? umma::smem_desc(sb + kk * 2048, kT5Box, 1024)
                                    : umma::smem_desc(sb + (kk >> 2) * kT5Box + (kk & 3) * 32, 16, 1024);
-          umma::mma_bf16(tmem, ad, bd, idesc, (pr > 0 || kk > 0) ? 1u : 0u);
+          umma::mma_bf16(tmem + 128 * acc, ad, bd, idesc, (pr > 0 || kk > 0) ? 1u : 0u);
         }
       }
-      umma::commit(&sm.mma_done);
+      umma::commit(&sm.mma_done[acc]);
     }
-    const bool ok = mbar_wait(&sm.mma_done, phase, a.status);
-    phase ^= 1;
+  };
+  auto wait = [&](int acc) {
+    const bool ok = mbar_wait(&sm.mma_done[acc], phase[acc], a.status);
+    phase[acc] ^= 1;
     umma::fence_after();
     return ok;
+  };
+  auto product = [&](uint8_t* const (&A)[2], bool a_mn, uint8_t* const (&B)[2], bool b_mn) {
+    issue(A, a_mn, B, b_mn, 0);
+    return wait(0);
   };
   // This thread's 32 accumulator values: row 32 (warp & 3) + lane, columns 32 (warp >> 2) ..
   const int er = 32 * (warp & 3) + lane, ec = 32 * (warp >> 2);
   const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + ec;
-  auto acc_load = [&](float (&v)[32]) {
+  auto acc_load = [&](float (&v)[32], int acc = 0) {
     uint32_t r0[16], r1[16];
-    umma::tmem_ld16_async(tl, r0);
-    umma::tmem_ld16_async(tl + 16, r1);
+    umma::tmem_ld16_async(tl + 128 * acc, r0);
+    umma::tmem_ld16_async(tl + 128 * acc + 16, r1);
     umma::tmem_wait_ld(r0);
     umma::tmem_wait_ld(r1);
 #pragma unroll
@@ -661,15 +670,20 @@ __global__ void __cluster_dims__(kNsCluster, 1, 1) __launch_bounds__(kT5Threads,
       put32(P2, er, ec, v);
     }
     sync_operands();
-    // X <- X P (tall) or P X (wide)   (B MN-major)
+    // X <- X P (tall) or P X (wide)   (B MN-major) into accumulator 0, and,
+    // unless this is the last step, T = M P into accumulator 1 right behind it:
+    // the X epilogue then overlaps the M P products.
+    const bool last = it + 1 == a.steps;
     if (tall)
-      ok = product(X2, false, P2, true) && ok;
+      issue(X2, false, P2, true, 0);
     else
-      ok = product(P2, false, X2, true) && ok;
+      issue(P2, false, X2, true, 0);
+    if (!last) issue(G2, false, P2, true, 1);
+    ok = wait(0) && ok;
     {
       float v[32];
-      acc_load(v);
-      if (it + 1 == a.steps) {
+      acc_load(v, 0);
+      if (last) {
         float4* dst = reinterpret_cast<float4*>(Xc + (int64_t)er * C + ec);
 #pragma unroll
         for (int q = 0; q < 8; ++q)
@@ -678,13 +692,12 @@ __global__ void __cluster_dims__(kNsCluster, 1, 1) __launch_bounds__(kT5Threads,
         put32(X2, er, ec, v);
       }
     }
-    if (it + 1 == a.steps) break;
-    sync_operands();
-    // M <- P (M P): T = M P into M's storage, then P T
-    ok = product(G2, false, P2, true) && ok;
+    if (last) break;
+    // M <- P (M P): T = M P (accumulator 1) into M's storage, then P T
+    ok = wait(1) && ok;
     {
       float v[32];
-      acc_load(v);
+      acc_load(v, 1);
       put32(G2, er, ec, v);
     }
     sync_operands();
@@ -700,7 +713,7 @@ __global__ void __cluster_dims__(kNsCluster, 1, 1) __launch_bounds__(kT5Threads,
   }
   (void)ok;
   cluster.sync();  // no CTA leaves while another may still read its shared memory
-  if (warp == 0) umma::tmem_dealloc(tmem, 128);
+  if (warp == 0) umma::tmem_dealloc(tmem, 256);
 }
 
 __global__ void copy_kernel(float* dst, const float* src, int64_t n) {
