@@ -89,7 +89,9 @@ typedef enum {
   TTT_ERR_TIMEOUT = -7,     /* a device-side bounded wait gave up */
   TTT_ERR_ALLOC = -8,       /* stream-ordered scratch allocation failed */
   TTT_ERR_ARG = -9,         /* scalar argument out of range (chunk, enums) */
-  TTT_ERR_SCRATCH = -10     /* scratch need exceeds lact_swiglu_fwd_noalloc's fixed pool */
+  TTT_ERR_SCRATCH = -10,    /* scratch need exceeds lact_swiglu_fwd_noalloc's fixed pool */
+  TTT_ERR_BOUNDS = -11      /* debug-bounds build only: a kernel index check failed (the
+                               access was skipped); reported by ttt_get_device_status */
 } ttt_status;
 
 typedef enum { TTT_F32 = 0, TTT_BF16 = 1 } ttt_dtype;
@@ -390,6 +392,17 @@ int32_t ttt_version(void);
  * returns TTT_ERR_TIMEOUT (and clears it). Returns TTT_OK once launched.
  */
 ttt_status ttt_selftest_wait_timeout(void* stream);
+
+/*
+ * Self-test of the debug-bounds build (the library compiled with
+ * -DTTT_DEBUG_BOUNDS, libttt_b200_dbg.so): enqueues one CTA whose index check
+ * fails by construction, without touching memory; ttt_get_device_status()
+ * then returns TTT_ERR_BOUNDS (and clears it). In that build every kernel
+ * index check that fails records TTT_ERR_BOUNDS the same way and skips the
+ * access instead of trapping. Returns TTT_OK once launched, or
+ * TTT_ERR_UNSUPPORTED from the normal build, whose checks are compiled out.
+ */
+ttt_status ttt_selftest_bounds(void* stream);
 
 #ifdef __cplusplus
 }

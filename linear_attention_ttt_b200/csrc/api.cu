@@ -129,11 +129,29 @@ __global__ void selftest_wait_kernel(int* status) {
   if (threadIdx.x == 0) ttt::mbar_wait(&bar, 0, status);
 }
 
+// Debug-bounds self-test: one index check that fails by construction (no
+// memory is accessed); the debug-bounds build records TTT_ERR_BOUNDS.
+__global__ void selftest_bounds_kernel(int* status) {
+  if (!TTT_BOUNDS(threadIdx.x > 1024u, status)) return;
+}
+
 }  // namespace
 
 extern "C" {
 
 int32_t ttt_version(void) { return 200; }
+
+ttt_status ttt_selftest_bounds(void* stream) {
+#ifdef TTT_DEBUG_BOUNDS
+  int* p = device_status_ptr();
+  if (!p) return TTT_ERR_CUDA;
+  selftest_bounds_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  return cudaGetLastError() == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
+#else
+  (void)stream;
+  return TTT_ERR_UNSUPPORTED;  // the checks are compiled out of this build
+#endif
+}
 
 void ttt_test_fail_allocations(int32_t n) { ttt::set_failing_allocs(n); }
 
@@ -157,6 +175,7 @@ const char* ttt_status_string(int32_t s) {
     case TTT_ERR_ALLOC: return "stream-ordered scratch allocation failed";
     case TTT_ERR_ARG: return "scalar argument out of range";
     case TTT_ERR_SCRATCH: return "scratch need exceeds the fixed pool of lact_swiglu_fwd_noalloc";
+    case TTT_ERR_BOUNDS: return "a kernel index check of the debug-bounds build failed";
     default: return "unknown status";
   }
 }
@@ -170,6 +189,7 @@ ttt_status ttt_get_device_status(void* stream) {
   if (cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return TTT_ERR_CUDA;
   if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return TTT_ERR_CUDA;
   if (v == ttt::DEV_TIMEOUT) return TTT_ERR_TIMEOUT;
+  if (v == ttt::DEV_BOUNDS) return TTT_ERR_BOUNDS;
   if (v != ttt::DEV_OK) return TTT_ERR_CUDA;
   return TTT_OK;
 }

@@ -10,7 +10,7 @@
 namespace ttt {
 
 // Error codes a kernel can record in the device status word.
-enum : int { DEV_OK = 0, DEV_TIMEOUT = 1, DEV_BAD_ARGS = 2 };
+enum : int { DEV_OK = 0, DEV_TIMEOUT = 1, DEV_BAD_ARGS = 2, DEV_BOUNDS = 3 };
 
 // A wait on one barrier gives up after this many nanoseconds of %globaltimer
 // (legitimate waits in these kernels last microseconds).
@@ -25,6 +25,20 @@ __device__ __forceinline__ uint64_t global_ns() {
 __device__ __forceinline__ void record_error(int* status, int code) {
   if (status) atomicCAS(status, DEV_OK, code);
 }
+
+// Index checks of the debug-bounds build (compiled with -DTTT_DEBUG_BOUNDS):
+// TTT_BOUNDS(cond, status) is `cond`, and a false `cond` also records
+// DEV_BOUNDS in the status word; the caller skips the access (no trap). In the
+// normal build it is the constant `true`, so the checks compile away.
+__device__ __forceinline__ bool bounds_check(bool ok, int* status) {
+  if (!ok) record_error(status, DEV_BOUNDS);
+  return ok;
+}
+#ifdef TTT_DEBUG_BOUNDS
+#define TTT_BOUNDS(cond, status) (::ttt::bounds_check(static_cast<bool>(cond), (status)))
+#else
+#define TTT_BOUNDS(cond, status) true
+#endif
 
 // Strided view of a [B,H,T,d] token tensor (element strides, last stride 1).
 struct TokView {

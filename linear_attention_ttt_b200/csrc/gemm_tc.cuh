@@ -258,6 +258,7 @@ struct Stage {
   uint8_t* buf;
   int lane;
   bool pending;  // a TMA read may still be in flight (warp-uniform)
+  int* status;   // device status word (index checks of the debug-bounds build)
 
   __device__ __forceinline__ void drain() {
     if (pending) {
@@ -360,6 +361,8 @@ __device__ __forceinline__ void epilogue_body(const Problem& pr, const TileCoord
   const bool lane_ok = lane < nrows;       // this lane's row exists
   uint8_t* const buf = sg.buf;
   sg.drain();
+  if (!TTT_BOUNDS(z >= 0 && z < pr.nz && row0 >= 0 && row0 < pr.M && nrows <= 32, sg.status))
+    return;
   // 64 bf16 columns of this warp's rows: values of columns [16p, 16p + 16)
   // from val(p, v), staged as bf16 (or as residuals for LO), then written.
   auto emit = [&](uint8_t* d, int64_t ld, auto lo_c, auto&& val) {
@@ -380,6 +383,9 @@ __device__ __forceinline__ void epilogue_body(const Problem& pr, const TileCoord
     const int64_t ld = (int64_t)e.ocols * 2;
     const int c0 = ch * 2 * kHid;
     const int hid = n0 / 2 + ch * kHid;
+    if (!TTT_BOUNDS(hid + kHid <= e.ocols && row0 + nrows <= e.orows && c0 + 2 * kHid <= BN,
+                    sg.status))
+      return;
     auto aq = [&](int p, float (&a)[16]) {
       float h1[16], h3[16];
       tmem_ld2x16(tbase + c0 + 16 * p, tbase + c0 + kHid + 16 * p, h1, h3);
@@ -398,6 +404,9 @@ __device__ __forceinline__ void epilogue_body(const Problem& pr, const TileCoord
     const int64_t ld = (int64_t)e.ocols * 2;
     const int cw = ch * 32;
     const int hid = tc.n0 * kHid + cw;
+    if (!TTT_BOUNDS(hid + 32 <= e.ocols && row0 + nrows <= e.orows && 2 * kHid + cw + 32 <= BN,
+                    sg.status))
+      return;
     const float eta_i = lane_ok ? eta_of(e, z, row0 + lane) : 0.f;
     auto dst = [&](int o) {
       return static_cast<uint8_t*>(e.optr[o]) + (((int64_t)z * e.orows + row0) * e.ocols + hid) * 2;
@@ -476,6 +485,7 @@ __device__ __forceinline__ void epilogue_body(const Problem& pr, const TileCoord
     for (int gi = 0; gi < pr.tn / 64; ++gi) {   // 32 fp32 columns per group
       const int gc = n0 + ch * (pr.tn / 2) + 32 * gi;
       if (gc >= pr.N) break;
+      if (!TTT_BOUNDS((gc & 3) == 0 && gc - n0 + 32 <= BN, sg.status)) break;
       float v[16], w[16];
       tmem_ld2x16(tbase + gc - n0, tbase + gc - n0 + 16, v, w);
       const float sc = e.scale;
@@ -498,6 +508,7 @@ __device__ __forceinline__ void epilogue_body(const Problem& pr, const TileCoord
       for (int gi = 0; gi < pr.tn / 64; ++gi) {
         const int gc = n0 + ch * (pr.tn / 2) + 32 * gi;
         if (gc >= pr.N) break;
+        if (!TTT_BOUNDS(gc + 32 <= pr.N && gc - n0 + 32 <= BN, sg.status)) break;
         float v[16], w[16];
         tmem_ld2x16(tbase + gc - n0, tbase + gc - n0 + 16, v, w);
         put_f32(buf, lane, 0, v);
@@ -509,6 +520,7 @@ __device__ __forceinline__ void epilogue_body(const Problem& pr, const TileCoord
       for (int gi = 0; gi < pr.tn / 128; ++gi) {
         const int gc = n0 + ch * (pr.tn / 2) + 64 * gi;
         if (gc >= pr.N) break;
+        if (!TTT_BOUNDS(gc + 64 <= pr.N && gc - n0 + 64 <= BN, sg.status)) break;
         auto y = [&](int p, float (&v)[16]) {
           uint32_t r[16];
           umma::tmem_ld16_async(tbase + gc - n0 + 16 * p, r);
@@ -616,6 +628,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
           const uint32_t tx = (uint32_t)(na * BM * BK * 2 + nb * bbytes);
           const int az2 = tc.z % A.zdiv, az3 = tc.z / A.zdiv, bz2 = tc.z % B.zdiv,
                     bz3 = tc.z / B.zdiv;
+          // TMA x coordinates are multiples of 8 bf16 (16 bytes) and the pass's
+          // boxes fit the stage's A and B slots
+          if (!TTT_BOUNDS((m0 & 7) == 0 && (bn0 & 7) == 0 && (kb0 * BK & 7) == 0 &&
+                              nb * bbytes + (na - 1) * BM * BK * 2 <= BN * BK * 2 && bn <= BN &&
+                              tc.z < pr.nz,
+                          status)) {
+            ok = false;
+            break;
+          }
           for (int kb = kb0; kb < kb0 + nk; ++kb, ++it) {
             const int st = it % kStages;
             if (it >= kStages && !mbar_wait(&sm.empty[st], ((it / kStages) - 1) & 1, status)) {
@@ -712,7 +733,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     // ---------------- epilogue: warps 2..9 ----------------
     const int quarter = warp & 3;
     const int ch = (warp - 2) >> 2;       // column half
-    Stage sgr{sm.ostage[warp - 2], lane, false};
+    Stage sgr{sm.ostage[warp - 2], lane, false, status};
     int lt = 0;
     for (int t = blockIdx.x; t < P.total_tiles; t += gridDim.x, ++lt) {
       const TileCoord tc = decode_tile(P, t);

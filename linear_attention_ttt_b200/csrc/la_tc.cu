@@ -129,6 +129,7 @@ __global__ void __launch_bounds__(kThreads, 1) la_tc_kernel(const __grid_constan
                                       ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.x >> 1, seg = blockIdx.x & 1, b = bh / p.H, h = bh % p.H;
+  if (!TTT_BOUNDS(bh < p.B * p.H, p.status)) return;  // uniform over both CTAs of the head
   const int ntot = (p.T + TT - 1) / TT, mid = (ntot + 1) / 2;
   // tiles [0, p1) build the state only; tiles [p1, tend) run the full loop
   const int p1 = seg ? mid : 0, tend = seg ? ntot : mid, n2 = tend - p1;
@@ -447,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1) la_tc_kernel(const __grid_constan
       __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out.p) + b * p.out.sb + h * p.out.sh;
       for (int it = ti; it < TT * 16 && ok; it += 128) {
         const int tt = it >> 4, c = it & 15;
-        if (t0 + tt < p.T)
+        if (t0 + tt < p.T && TTT_BOUNDS(tt < TT && c * 8 + 8 <= D, p.status))
           *reinterpret_cast<uint4*>(o + (int64_t)(t0 + tt) * p.out.st + c * 8) =
               *reinterpret_cast<const uint4*>(st + tt * D + c * 8);
       }

@@ -63,6 +63,7 @@ struct RowArgs {
   float* M[3];             // momentum masters [Z][rows][cols]
   const float* Min[3];     // initial momentum (prep only; null: zero)
   int64_t min_sz[3];       // non-zero when Min holds one matrix per (batch, head)
+  int* status;             // device status word (index checks of the debug-bounds build)
 };
 
 // One warp per (z, row of W1 | W3 | W2).
@@ -111,6 +112,10 @@ __global__ void __launch_bounds__(256) lact_rows_kernel(RowArgs a) {
     orow = (int64_t)z * 2 * a.dh + (r / gemm::kHid) * 2 * gemm::kHid + (m == 1 ? gemm::kHid : 0) +
            (r % gemm::kHid);
   }
+  if (!TTT_BOUNDS(orow >= 0 && orow < (int64_t)a.Z * (m == 2 ? a.dv : 2 * a.dh) && r < nrows &&
+                      (len % 128 != 0 || len <= 1024),
+                  a.status))
+    return;
   hi += orow * len;
   if (a.split) lo += orow * len;
 
@@ -477,6 +482,11 @@ __global__ void __cluster_dims__(kNsCluster, 1, 1) __launch_bounds__(kT5Threads,
   const bool tall = R >= C;
   float* Xc = a.G[m] + (int64_t)z * R * C + (tall ? (int64_t)c * kN5 * C : (int64_t)c * kN5);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // this CTA's 128 x 128 slab lies inside the matrix (a failed check skips the
+  // slab's global loads and stores but keeps every cluster barrier)
+  const bool slab_ok = TTT_BOUNDS(tall ? (C == kN5 && (c + 1) * kN5 <= R)
+                                       : (R == kN5 && (c + 1) * kN5 <= C),
+                                  a.status);
 
   if (tid == 0) {
     mbar_init(&sm.mma_done[0], 1);
@@ -499,8 +509,8 @@ __global__ void __cluster_dims__(kNsCluster, 1, 1) __launch_bounds__(kT5Threads,
   for (int i = 0; i < 4; ++i) {
     const int e = tid + i * kT5Threads, r = e >> 4, c0 = (e & 15) * 8;
     const float4* src = reinterpret_cast<const float4*>(Xc + (int64_t)r * C + c0);
-    xs[i][0] = src[0];
-    xs[i][1] = src[1];
+    xs[i][0] = slab_ok ? src[0] : make_float4(0.f, 0.f, 0.f, 0.f);
+    xs[i][1] = slab_ok ? src[1] : make_float4(0.f, 0.f, 0.f, 0.f);
     ss += xs[i][0].x * xs[i][0].x + xs[i][0].y * xs[i][0].y + xs[i][0].z * xs[i][0].z +
           xs[i][0].w * xs[i][0].w + xs[i][1].x * xs[i][1].x + xs[i][1].y * xs[i][1].y +
           xs[i][1].z * xs[i][1].z + xs[i][1].w * xs[i][1].w;
@@ -687,7 +697,7 @@ __global__ void __cluster_dims__(kNsCluster, 1, 1) __launch_bounds__(kT5Threads,
         float4* dst = reinterpret_cast<float4*>(Xc + (int64_t)er * C + ec);
 #pragma unroll
         for (int q = 0; q < 8; ++q)
-          dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+          if (slab_ok) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
       } else {
         put32(X2, er, ec, v);
       }
@@ -1084,6 +1094,7 @@ ttt_status lact_run(const LactArgs& a, cudaStream_t s, void* base, size_t bytes)
   ra.dv = dv;
   ra.dh = dh;
   ra.split = split;
+  ra.status = a.status;
   // momentum: LactArgs order (W1, W2, W3) -> row order (W1, W3, W2)
   ra.momentum = a.momentum;
   ra.beta = a.beta;

@@ -145,6 +145,7 @@ __global__ void __launch_bounds__(kThreads, 1) ttt_linear_wy_kernel(const __grid
                                       ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.x, b = bh / p.H, h = bh % p.H;
+  if (!TTT_BOUNDS(bh < p.B * p.H, p.status)) return;  // uniform over the CTA
   const int ngroups = (p.T + kG - 1) / kG;
 
   if (threadIdx.x == 0) {
@@ -262,7 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1) ttt_linear_wy_kernel(const __grid
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       const int t = (tid >> 3) + 32 * i;
-      if (gi * kG + t < p.T)
+      if (gi * kG + t < p.T && TTT_BOUNDS(t < kG && cch * 8 + 8 <= D, p.status))
         *reinterpret_cast<uint4*>(outp + (int64_t)(gi * kG + t) * p.out.st + cch * 8) =
             *reinterpret_cast<const uint4*>(os + t * 128 + ((cch ^ (t & 7)) << 4));
     }

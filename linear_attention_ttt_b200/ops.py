@@ -13,7 +13,11 @@ from typing import Optional
 
 import torch
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libttt_b200.so")
+_PKG = os.path.dirname(os.path.abspath(__file__))
+# TTT_B200_LIB selects another build of the library, e.g. the debug-bounds one
+# (libttt_b200_dbg.so, from `python -m linear_attention_ttt_b200.build --debug-bounds`).
+LIB_PATH = os.environ.get("TTT_B200_LIB") or os.path.join(_PKG, "libttt_b200.so")
+DEBUG_LIB_PATH = os.path.join(_PKG, "libttt_b200_dbg.so")
 
 TTT_F32, TTT_BF16 = 0, 1
 TTT_LOSS_MSE, TTT_LOSS_NEG_DOT = 0, 1
@@ -23,7 +27,9 @@ STATUS = {
     0: "TTT_OK", -1: "TTT_ERR_NULL", -2: "TTT_ERR_SHAPE", -3: "TTT_ERR_DTYPE",
     -4: "TTT_ERR_LAYOUT", -5: "TTT_ERR_UNSUPPORTED", -6: "TTT_ERR_CUDA",
     -7: "TTT_ERR_TIMEOUT", -8: "TTT_ERR_ALLOC", -9: "TTT_ERR_ARG", -10: "TTT_ERR_SCRATCH",
+    -11: "TTT_ERR_BOUNDS",
 }
+ERR_CODES = {name: code for code, name in STATUS.items()}
 
 
 class TTTError(RuntimeError):
@@ -80,6 +86,7 @@ SIGNATURES = {
     "ttt_version": ([], ctypes.c_int32),
     "ttt_test_fail_allocations": ([ctypes.c_int32], None),
     "ttt_selftest_wait_timeout": ([ctypes.c_void_p], ctypes.c_int32),
+    "ttt_selftest_bounds": ([ctypes.c_void_p], ctypes.c_int32),
 }
 
 
