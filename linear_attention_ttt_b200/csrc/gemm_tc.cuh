@@ -394,8 +394,33 @@ __device__ __forceinline__ void epilogue_body(const Problem& pr, const TileCoord
         a[u] = h1[u] * (SPLIT ? sigmoidf_(h1[u]) : sigmoid_fast(h1[u])) * h3[u];
     };
     const int64_t off = (((int64_t)z * e.orows + row0) * e.ocols + hid) * 2;
-    emit(static_cast<uint8_t*>(e.optr[0]) + off, ld, Hi{}, aq);
-    if constexpr (SPLIT) emit(static_cast<uint8_t*>(e.optr[3]) + off, ld, Lo{}, aq);
+    if constexpr (!SPLIT) {
+      // four 16-column steps; the TMEM reads of the next step are issued right
+      // after the wait for the current one and overlap its arithmetic
+      uint32_t rb[2][2][16];
+      auto issue = [&](int p) {
+        umma::tmem_ld16_async(tbase + c0 + 16 * p, rb[p & 1][0]);
+        umma::tmem_ld16_async(tbase + c0 + kHid + 16 * p, rb[p & 1][1]);
+      };
+      issue(0);
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        umma::tmem_wait_ld(rb[p & 1][0]);
+        umma::tmem_wait_ld(rb[p & 1][1]);
+        if (p + 1 < 4) issue(p + 1);
+        float a[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const float h1 = __uint_as_float(rb[p & 1][0][u]), h3 = __uint_as_float(rb[p & 1][1][u]);
+          a[u] = h1 * sigmoid_fast(h1) * h3;
+        }
+        put_bf16<false>(buf, lane, p, a);
+      }
+      flush_rows(buf, lane, static_cast<uint8_t*>(e.optr[0]) + off, ld, nrows);
+    } else {
+      emit(static_cast<uint8_t*>(e.optr[0]) + off, ld, Hi{}, aq);
+      emit(static_cast<uint8_t*>(e.optr[3]) + off, ld, Lo{}, aq);
+    }
   } else if constexpr (EPI == EPI_HKG) {
     // columns [0, 64) h1, [64, 128) h3, [128, 192) u of hidden units
     // hid .. hid + 63; this warp takes units [32ch, 32ch + 32). The sigmoid of
@@ -413,73 +438,80 @@ __device__ __forceinline__ void epilogue_body(const Problem& pr, const TileCoord
     };
     uint8_t* const bA = buf;
     uint8_t* const bB = buf + 2048;
-    auto load3 = [&](int p, float (&h1)[16], float (&h3)[16], float (&gz)[16]) {
-      uint32_t r1[16], r3[16], rg[16];
-      umma::tmem_ld16_async(tbase + cw + 16 * p, r1);
-      umma::tmem_ld16_async(tbase + kHid + cw + 16 * p, r3);
-      umma::tmem_ld16_async(tbase + 2 * kHid + cw + 16 * p, rg);
-      umma::tmem_wait_ld(r1);
-      umma::tmem_wait_ld(r3);
-      umma::tmem_wait_ld(rg);
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        h1[u] = __uint_as_float(r1[u]);
-        h3[u] = __uint_as_float(r3[u]);
-        gz[u] = -eta_i * __uint_as_float(rg[u]);
-      }
+    // Passes over the warp's 32 units in two 16-column steps each: ak (and, not
+    // split, dh3), then dh3 (split), then dh1. Each step reads h1, h3 and u
+    // from TMEM; the reads of the next step are issued right after the wait
+    // for the current one, so their latency overlaps this step's arithmetic
+    // (a wait covers every read of the thread issued before it).
+    constexpr int kSteps = SPLIT ? 6 : 4;
+    uint32_t rb[2][3][16];
+    auto issue = [&](int st) {
+      const int p = st & 1;
+      umma::tmem_ld16_async(tbase + cw + 16 * p, rb[st & 1][0]);
+      umma::tmem_ld16_async(tbase + kHid + cw + 16 * p, rb[st & 1][1]);
+      umma::tmem_ld16_async(tbase + 2 * kHid + cw + 16 * p, rb[st & 1][2]);
     };
     float sgm[2][16];
-    // pass 1: ak = eta silu(h1) h3 (+ dh3 = gz silu(h1) when not split)
+    issue(0);
 #pragma unroll
-    for (int p = 0; p < 2; ++p) {
-      float h1[16], h3[16], gz[16], a[16], d[16];
-      load3(p, h1, h3, gz);
+    for (int st = 0; st < kSteps; ++st) {
+      const int p = st & 1;
+      const int pass = SPLIT ? (st >> 1) : 2 * (st >> 1);  // 0: ak (+dh3), 1: dh3, 2: dh1
+      umma::tmem_wait_ld(rb[st & 1][0]);
+      umma::tmem_wait_ld(rb[st & 1][1]);
+      umma::tmem_wait_ld(rb[st & 1][2]);
+      if (st + 1 < kSteps) issue(st + 1);
+      float h1[16], h3[16], gz[16], d[16];
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
-        sgm[p][u] = SPLIT ? sigmoidf_(h1[u]) : sigmoid_fast(h1[u]);
-        const float s1 = h1[u] * sgm[p][u];
-        a[u] = eta_i * s1 * h3[u];
-        d[u] = gz[u] * s1;
+        h1[u] = __uint_as_float(rb[st & 1][0][u]);
+        h3[u] = __uint_as_float(rb[st & 1][1][u]);
+        gz[u] = -eta_i * __uint_as_float(rb[st & 1][2][u]);
       }
-      if constexpr (SPLIT) {
-        put_split_64(bA, bB, lane, p, a);
-      } else {
-        put_bf16_64<false>(bA, lane, p, a);
-        put_bf16_64<false>(bB, lane, p, d);
-      }
-    }
-    flush_rows64(bA, lane, dst(0), ld, nrows);
-    flush_rows64(bB, lane, dst(SPLIT ? 3 : 2), ld, nrows);
-    if constexpr (SPLIT) {
-      // pass 2: dh3 hi / lo
+      if (pass == 0) {
+        float a[16];
 #pragma unroll
-      for (int p = 0; p < 2; ++p) {
-        float h1[16], h3[16], gz[16], d[16];
-        load3(p, h1, h3, gz);
+        for (int u = 0; u < 16; ++u) {
+          sgm[p][u] = SPLIT ? sigmoidf_(h1[u]) : sigmoid_fast(h1[u]);
+          const float s1 = h1[u] * sgm[p][u];
+          a[u] = eta_i * s1 * h3[u];
+          d[u] = gz[u] * s1;
+        }
+        if constexpr (SPLIT) {
+          put_split_64(bA, bB, lane, p, a);
+        } else {
+          put_bf16_64<false>(bA, lane, p, a);
+          put_bf16_64<false>(bB, lane, p, d);
+        }
+      } else if (pass == 1) {
 #pragma unroll
         for (int u = 0; u < 16; ++u) d[u] = gz[u] * h1[u] * sgm[p][u];
         put_split_64(bA, bB, lane, p, d);
-      }
-      flush_rows64(bA, lane, dst(2), ld, nrows);
-      flush_rows64(bB, lane, dst(5), ld, nrows);
-    }
-    // last pass: dh1 = gz h3 silu'(h1),  silu'(x) = sigmoid(x) (1 + x (1 - sigmoid(x)))
+      } else {
+        // dh1 = gz h3 silu'(h1),  silu'(x) = sigmoid(x) (1 + x (1 - sigmoid(x)))
 #pragma unroll
-    for (int p = 0; p < 2; ++p) {
-      float h1[16], h3[16], gz[16], d[16];
-      load3(p, h1, h3, gz);
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const float sg1 = sgm[p][u];
-        d[u] = gz[u] * h3[u] * sg1 * (1.f + h1[u] * (1.f - sg1));
+        for (int u = 0; u < 16; ++u) {
+          const float sg1 = sgm[p][u];
+          d[u] = gz[u] * h3[u] * sg1 * (1.f + h1[u] * (1.f - sg1));
+        }
+        if constexpr (SPLIT)
+          put_split_64(bA, bB, lane, p, d);
+        else
+          put_bf16_64<false>(bA, lane, p, d);
       }
-      if constexpr (SPLIT)
-        put_split_64(bA, bB, lane, p, d);
-      else
-        put_bf16_64<false>(bA, lane, p, d);
+      if (p == 1) {  // the pass's 32 units are staged
+        if (pass == 0) {
+          flush_rows64(bA, lane, dst(0), ld, nrows);
+          flush_rows64(bB, lane, dst(SPLIT ? 3 : 2), ld, nrows);
+        } else if (pass == 1) {
+          flush_rows64(bA, lane, dst(2), ld, nrows);
+          flush_rows64(bB, lane, dst(5), ld, nrows);
+        } else {
+          flush_rows64(bA, lane, dst(1), ld, nrows);
+          if constexpr (SPLIT) flush_rows64(bB, lane, dst(4), ld, nrows);
+        }
+      }
     }
-    flush_rows64(bA, lane, dst(1), ld, nrows);
-    if constexpr (SPLIT) flush_rows64(bB, lane, dst(4), ld, nrows);
   } else if constexpr (EPI == EPI_GRAD) {
     const int oz2 = z % e.ozdiv, oz3 = z / e.ozdiv;
     for (int gi = 0; gi < pr.tn / 64; ++gi) {   // 32 fp32 columns per group
