@@ -17,22 +17,33 @@
 // and dL/dW_s becomes G of the previous chunk; after the first chunk it is
 // dL/dW0.
 //
+// In matrix form over a chunk (rows = tokens, N = diag(eta), E the rows e_t,
+// masks inclusive of the diagonal) these are
+//   dQ = dY W_s^T - tril(dY E^T) N K,
+//   kR = K G + triu(K Q^T) dY,   Rx = E G^T + triu(E dY^T) Q   (rows k_t R_t, R_t e_t^T),
+//   dL/dW_s = G + Q^T dY (+ K^T dE for MSE),
+// so only G links one chunk to the one before it.
+//
 // Layout: one CTA of 256 threads per (batch, head), fp32 arithmetic on the
-// CUDA cores. A forward pass stores the start weights of every chunk (MSE)
-// in a workspace, or only runs to the final weights (inner product, whose
-// token gradients do not depend on W). The backward then walks the chunks in
-// reverse and, inside each chunk, the tokens in reverse, carrying W_t
-// (recovered from the chunk-end weights by adding each token's update back),
-// R and the chunk's dL/dW_s contributions. Shared memory holds W_s, W_t and
-// R; the per-thread part of sum_t k_t^T de_t stays in registers.
+// CUDA cores, 16-token blocks staged in shared memory. Pass 1 walks the
+// chunks forward: it stores the chunk-start weights (MSE) in a workspace and
+// computes dQ with the running sum of the chunk's updates. Pass 2 walks the
+// chunks, and the blocks inside each chunk, in reverse, carrying R (G plus
+// the q^T dy of the later tokens of the chunk) in shared memory and the
+// chunk's sum_t k_t^T de_t in registers. Weight-shaped arrays in shared
+// memory have a row stride of dv + 1 floats and token tiles of d + 1, so that
+// walks along either index are free of bank conflicts.
 #include "common.cuh"
 
 namespace ttt {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kMaxElems = 128 * 128;                  // dk * dv
-constexpr int kRegs = kMaxElems / kThreads;           // per-thread dW_s part
+constexpr int kTB = 16;                                // tokens per block
+constexpr int kMaxD = 128;                             // dk, dv <= 128
+constexpr int kRegs = kMaxD * kMaxD / kThreads;        // weight elements per thread
+constexpr int kOut = kTB * kMaxD / kThreads;           // token-tile elements per thread
+constexpr int kLdS = kTB + 1;                          // row stride of the 16 x 16 tiles
 
 template <typename T>
 __device__ __forceinline__ float ld(const TokView& v, int b, int h, int64_t t, int c) {
@@ -43,177 +54,366 @@ __device__ __forceinline__ void st(const TokViewMut& v, int b, int h, int64_t t,
   (static_cast<T*>(v.p) + b * v.sb + h * v.sh + t * v.st)[c] = T(x);
 }
 
-template <typename T>
-__global__ void __launch_bounds__(kThreads) ttt_linear_bwd_kernel(LinearBwdArgs a) {
+// 4-byte asynchronous copy global -> shared (no register round trip)
+__device__ __forceinline__ void cp_async4(float* dst, const float* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(
+                   static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+               "l"(src)
+               : "memory");
+}
+// waits for this thread's copies; a barrier after it publishes them to the CTA
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+__host__ __device__ constexpr size_t bwd_smem_floats(int dk, int dv) {
+  return 2 * (size_t)dk * (dv + 1) + 3 * (size_t)kTB * (dk + 1) + 4 * (size_t)kTB * (dv + 1) +
+         2 * kTB * kLdS + kTB;
+}
+
+// kDiv: dk and dv divide the thread count, so that the element a thread owns
+// in pass u of a flat walk keeps its column: (tid + u * kThreads) % d = tid % d.
+// The index helpers then give the same elements with a column the compiler
+// sees as fixed, and loads along that column are shared across the passes.
+template <typename T, bool kDiv>
+__global__ void __launch_bounds__(kThreads, 1) ttt_linear_bwd_kernel(LinearBwdArgs a) {
   extern __shared__ float smem[];
   const int dk = a.dk, dv = a.dv, n = dk * dv;
+  const int ldw = dv + 1, ldk = dk + 1, ldv = dv + 1;
   const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool mse = a.loss == TTT_LOSS_MSE;
+  if (!TTT_BOUNDS(dk <= kMaxD && dv <= kMaxD && a.chunk > 0 &&
+                      (!kDiv || (kThreads % dk == 0 && kThreads % dv == 0)),
+                  a.status))
+    return;
+  // row and column of element tid + u * kThreads of a flat [.][d] walk
+  auto row_of = [&](int u, int d) {
+    return kDiv ? tid / d + (kThreads / d) * u : (tid + u * kThreads) / d;
+  };
+  auto col_of = [&](int u, int d) { return kDiv ? tid % d : (tid + u * kThreads) % d; };
 
-  float* Ws = smem;            // [dk][dv] chunk-start weights
-  float* Wt = Ws + n;          // [dk][dv] weights after the current token
-  float* R = Wt + n;           // [dk][dv]
-  float* qv = R + n;           // [dk]
-  float* kv = qv + dk;         // [dk]
-  float* vv = kv + dk;         // [dv]
-  float* dyv = vv + dv;        // [dv]
-  float* ev = dyv + dv;        // [dv] e_t (MSE) or v_t (inner product)
-  float* kR = ev + dv;         // [dv]
-  float* Rx = kR + dv;         // [dk] R_t e_t^T or R_t v_t^T
-  float* red = Rx + dk;        // [8] warp partials
-  float* etas = red + 8;       // [1]
+  float* Ws = smem;              // [dk][ldw] chunk-start weights
+  float* Acc = Ws + dk * ldw;    // [dk][ldw] pass 1: the chunk's updates so far; pass 2: R
+  float* Qs = Acc + dk * ldw;    // [kTB][ldk]
+  float* Ks = Qs + kTB * ldk;    // [kTB][ldk]
+  float* Zs = Ks + kTB * ldk;    // [kTB][ldk]  R_t e_t^T
+  float* Vs = Zs + kTB * ldk;    // [kTB][ldv]  v, then de (pass 2)
+  float* Ys = Vs + kTB * ldv;    // [kTB][ldv]  dy
+  float* Es = Ys + kTB * ldv;    // [kTB][ldv]  e
+  float* Xs = Es + kTB * ldv;    // [kTB][ldv]  k_t R_t
+  float* S1 = Xs + kTB * ldv;    // [kTB][kLdS]
+  float* S2 = S1 + kTB * kLdS;   // [kTB][kLdS]
+  float* etas = S2 + kTB * kLdS; // [kTB]
 
   const float* eta = a.eta.p + b * a.eta.sb + h * a.eta.sh;
-  auto load_tok = [&](int t, bool with_q) {
-    for (int c = tid; c < dk; c += kThreads) {
-      kv[c] = ld<T>(a.k, b, h, t, c);
-      if (with_q) qv[c] = ld<T>(a.q, b, h, t, c);
+  // tokens [t0, t0 + nt) into the tiles, zero rows after nt: every load is
+  // issued before the first shared-memory store, so that the block waits for
+  // one round trip
+  auto load_block = [&](int t0, int nt) {
+    float qv[kOut], kv[kOut], vv[kOut], yv[kOut];
+#pragma unroll
+    for (int u = 0; u < kOut; ++u) {
+      const int t = row_of(u, dk), r = col_of(u, dk);
+      const bool ok = t < kTB && t < nt;
+      qv[u] = ok ? ld<T>(a.q, b, h, t0 + t, r) : 0.f;
+      kv[u] = ok ? ld<T>(a.k, b, h, t0 + t, r) : 0.f;
     }
-    for (int c = tid; c < dv; c += kThreads) {
-      vv[c] = ld<T>(a.v, b, h, t, c);
-      if (with_q) dyv[c] = ld<T>(a.dy, b, h, t, c);
+#pragma unroll
+    for (int u = 0; u < kOut; ++u) {
+      const int t = row_of(u, dv), j = col_of(u, dv);
+      const bool ok = t < kTB && t < nt;
+      vv[u] = ok ? ld<T>(a.v, b, h, t0 + t, j) : 0.f;
+      yv[u] = ok ? ld<T>(a.dy, b, h, t0 + t, j) : 0.f;
     }
-    if (tid == 0) etas[0] = eta[(int64_t)t * a.eta.st];
+    const float ev = tid < nt ? eta[(int64_t)(t0 + tid) * a.eta.st] : 0.f;
+#pragma unroll
+    for (int u = 0; u < kOut; ++u) {
+      const int t = row_of(u, dk), r = col_of(u, dk);
+      if (t < kTB) Qs[t * ldk + r] = qv[u], Ks[t * ldk + r] = kv[u];
+    }
+#pragma unroll
+    for (int u = 0; u < kOut; ++u) {
+      const int t = row_of(u, dv), j = col_of(u, dv);
+      if (t < kTB) Vs[t * ldv + j] = vv[u], Ys[t * ldv + j] = yv[u];
+    }
+    if (tid < kTB) etas[tid] = ev;
   };
-  // ev = k W_s - v (MSE) or v (inner product), one thread per column
+  // a dense [dk][dv] fp32 matrix into a weight-shaped array (asynchronous;
+  // cp_async_wait_all and a barrier before use)
+  auto fetch_weights = [&](float* dst, const float* src) {
+    for (int x = tid; x < n; x += kThreads) cp_async4(dst + (x / dv) * ldw + x % dv, src + x);
+  };
+  // E = K W_s - V (MSE) or -V (inner product)
   auto make_e = [&]() {
-    for (int c = tid; c < dv; c += kThreads) {
-      if (mse) {
-        float acc = 0.f;
-        for (int r = 0; r < dk; ++r) acc = fmaf(kv[r], Ws[r * dv + c], acc);
-        ev[c] = acc - vv[c];
-      } else {
-        ev[c] = vv[c];
-      }
+    float acc[kOut];
+    int ti[kOut], ji[kOut];
+#pragma unroll
+    for (int u = 0; u < kOut; ++u) {
+      ti[u] = row_of(u, dv), ji[u] = col_of(u, dv), acc[u] = 0.f;
     }
+    if (mse)
+      #pragma unroll 4
+      for (int r = 0; r < dk; ++r) {
+#pragma unroll
+        for (int u = 0; u < kOut; ++u)
+          if (ti[u] < kTB) acc[u] = fmaf(Ks[ti[u] * ldk + r], Ws[r * ldw + ji[u]], acc[u]);
+      }
+#pragma unroll
+    for (int u = 0; u < kOut; ++u)
+      if (ti[u] < kTB) Es[ti[u] * ldv + ji[u]] = acc[u] - Vs[ti[u] * ldv + ji[u]];
   };
 
-  // ---- forward: chunk-start weights (MSE) and the final weights ----
+  // ---- pass 1: chunk-start weights (MSE) and dQ ----
   const float* W0 = a.W0 + b * a.w0_sb + (int64_t)h * n;
-  for (int x = tid; x < n; x += kThreads) Ws[x] = Wt[x] = W0[x];
-  __syncthreads();
+  fetch_weights(Ws, W0);
+  cp_async_wait_all();
   float* ck = a.ckpt ? a.ckpt + (int64_t)bh * a.nchunks * n : nullptr;
   for (int c = 0; c < a.nchunks; ++c) {
     const int s0 = c * a.chunk, e0 = min(s0 + a.chunk, a.T);
-    if (mse)
-      for (int x = tid; x < n; x += kThreads) ck[(int64_t)c * n + x] = Ws[x];
-    for (int t = s0; t < e0; ++t) {
-      load_tok(t, false);
+    for (int x = tid; x < n; x += kThreads) {
+      const int r = x / dv, j = x % dv;
+      if (mse) ck[(int64_t)c * n + x] = Ws[r * ldw + j];
+      Acc[r * ldw + j] = 0.f;
+    }
+    for (int t0 = s0; t0 < e0; t0 += kTB) {
+      const int nt = min(kTB, e0 - t0);
+      __syncthreads();  // the previous block is done with the tiles
+      load_block(t0, nt);
       __syncthreads();
       make_e();
       __syncthreads();
-      // W_t = W_{t-1} - eta_t k_t^T e_t (MSE) or + eta_t k_t^T v_t
-      const float sc = mse ? -etas[0] : etas[0];
-      for (int x = tid; x < n; x += kThreads) Wt[x] = fmaf(sc * kv[x / dv], ev[x % dv], Wt[x]);
+      // S1[t][i] = eta_i (dy_t . e_i) for i <= t
+      {
+        const int t = tid / kTB, i = tid % kTB;
+        float acc = 0.f;
+        if (i <= t && t < nt)
+          #pragma unroll 4
+          for (int j = 0; j < dv; ++j) acc = fmaf(Ys[t * ldv + j], Es[i * ldv + j], acc);
+        S1[t * kLdS + i] = etas[i] * acc;
+      }
       __syncthreads();
+      // dq_t = dy_t (W_s - Acc)^T - sum_{i <= t} S1[t][i] k_i
+      {
+        float acc[kOut];
+        int ti[kOut], ri[kOut];
+#pragma unroll
+        for (int u = 0; u < kOut; ++u) {
+          ti[u] = row_of(u, dk), ri[u] = col_of(u, dk), acc[u] = 0.f;
+        }
+        #pragma unroll 4
+        for (int j = 0; j < dv; ++j) {
+#pragma unroll
+          for (int u = 0; u < kOut; ++u)
+            if (ti[u] < kTB)
+              acc[u] = fmaf(Ys[ti[u] * ldv + j], Ws[ri[u] * ldw + j] - Acc[ri[u] * ldw + j], acc[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < kOut; ++u) {
+          if (ti[u] >= nt) continue;
+          for (int i = 0; i <= ti[u]; ++i)
+            acc[u] = fmaf(-S1[ti[u] * kLdS + i], Ks[i * ldk + ri[u]], acc[u]);
+          st<T>(a.gq, b, h, t0 + ti[u], ri[u], acc[u]);
+        }
+      }
+      __syncthreads();
+      // Acc += K^T N E
+      for (int x0 = 0; x0 < n; x0 += 8 * kThreads) {
+        float acc[8];
+        int ri[8], ji[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          ri[u] = row_of(x0 / kThreads + u, dv), ji[u] = col_of(x0 / kThreads + u, dv);
+          acc[u] = ri[u] < dk ? Acc[ri[u] * ldw + ji[u]] : 0.f;
+        }
+        for (int i = 0; i < nt; ++i) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            if (ri[u] < dk) acc[u] = fmaf(etas[i] * Ks[i * ldk + ri[u]], Es[i * ldv + ji[u]], acc[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (ri[u] < dk) Acc[ri[u] * ldw + ji[u]] = acc[u];
+      }
     }
-    for (int x = tid; x < n; x += kThreads) Ws[x] = Wt[x];
+    __syncthreads();
+    for (int x = tid; x < n; x += kThreads) {
+      const int r = x / dv, j = x % dv;
+      Ws[r * ldw + j] -= Acc[r * ldw + j];
+    }
     __syncthreads();
   }
-  // Wt = W_final now.
 
-  // ---- backward ----
+  // ---- pass 2: reverse ----
   const float* G0 = a.dWf ? a.dWf + (int64_t)bh * n : nullptr;
-  for (int x = tid; x < n; x += kThreads) R[x] = G0 ? G0[x] : 0.f;
-  float acc[kRegs];
+  if (G0) {
+    fetch_weights(Acc, G0);
+    cp_async_wait_all();
+  } else {
+    for (int x = tid; x < n; x += kThreads) Acc[(x / dv) * ldw + x % dv] = 0.f;
+  }
+  float kde[kRegs];  // this thread's part of sum_t k_t^T de_t over the chunk
 #pragma unroll
-  for (int i = 0; i < kRegs; ++i) acc[i] = 0.f;
-  float* dq_eta = a.deta + (int64_t)bh * a.T;
+  for (int u = 0; u < kRegs; ++u) kde[u] = 0.f;
+  float* deta_out = a.deta + (int64_t)bh * a.T;
   for (int c = a.nchunks - 1; c >= 0; --c) {
     const int s0 = c * a.chunk, e0 = min(s0 + a.chunk, a.T);
-    if (mse)
-      for (int x = tid; x < n; x += kThreads) Ws[x] = ck[(int64_t)c * n + x];
-    __syncthreads();
-    for (int t = e0 - 1; t >= s0; --t) {
-      load_tok(t, true);
+    __syncthreads();  // every thread is done with the later chunk's weights
+    if (mse) fetch_weights(Ws, ck + (int64_t)c * n);  // waited for below, with the tokens
+    const int nb = (e0 - s0 + kTB - 1) / kTB;
+    for (int bi = nb - 1; bi >= 0; --bi) {
+      const int t0 = s0 + bi * kTB, nt = min(kTB, e0 - t0);
+      __syncthreads();  // the previous block is done with the tiles
+      load_block(t0, nt);
+      cp_async_wait_all();  // the chunk's weights, at its first block
       __syncthreads();
       make_e();
-      // dq_t = dy_t W_t^T (reads shared memory only, like make_e)
-      for (int r = tid; r < dk; r += kThreads) {
-        float s = 0.f;
-        for (int j = 0; j < dv; ++j) s = fmaf(dyv[j], Wt[r * dv + j], s);
-        st<T>(a.gq, b, h, t, r, s);
-      }
-      __syncthreads();
-      // R += q_t^T dy_t; W_{t-1} = W_t + eta_t k_t^T e_t (MSE) or - eta_t k_t^T v_t
-      const float et = etas[0];
-      const float sc = mse ? et : -et;
-      for (int x = tid; x < n; x += kThreads) {
-        const int r = x / dv, j = x % dv;
-        R[x] = fmaf(qv[r], dyv[j], R[x]);
-        Wt[x] = fmaf(sc * kv[r], ev[j], Wt[x]);
-      }
-      __syncthreads();
-      // kR = k_t R_t (per column), Rx = R_t e_t^T (per row)
-      for (int j = tid; j < dv; j += kThreads) {
-        float s = 0.f;
-        for (int r = 0; r < dk; ++r) s = fmaf(kv[r], R[r * dv + j], s);
-        kR[j] = s;
-      }
-      for (int r = tid; r < dk; r += kThreads) {
-        float s = 0.f;
-        for (int j = 0; j < dv; ++j) s = fmaf(R[r * dv + j], ev[j], s);
-        Rx[r] = s;
-      }
-      __syncthreads();
-      // deta_t = -<R_t, g_t>: MSE -(k R) . e, inner product (k R) . v
+      // S1[t][t'] = k_t . q_t' for t <= t'
       {
+        const int t = tid / kTB, tp = tid % kTB;
+        float acc = 0.f;
+        if (t <= tp && tp < nt)
+          #pragma unroll 4
+          for (int r = 0; r < dk; ++r) acc = fmaf(Ks[t * ldk + r], Qs[tp * ldk + r], acc);
+        S1[t * kLdS + tp] = acc;
+      }
+      __syncthreads();
+      // S2[t][t'] = e_t . dy_t' for t <= t'
+      {
+        const int t = tid / kTB, tp = tid % kTB;
+        float acc = 0.f;
+        if (t <= tp && tp < nt)
+          #pragma unroll 4
+          for (int j = 0; j < dv; ++j) acc = fmaf(Es[t * ldv + j], Ys[tp * ldv + j], acc);
+        S2[t * kLdS + tp] = acc;
+      }
+      __syncthreads();
+      // kR = K R + S1 dY,  Rx = E R^T + S2 Q
+      {
+        float acc[kOut];
+        int ti[kOut], ji[kOut];
+#pragma unroll
+        for (int u = 0; u < kOut; ++u) {
+          ti[u] = row_of(u, dv), ji[u] = col_of(u, dv), acc[u] = 0.f;
+        }
+        #pragma unroll 4
+        for (int r = 0; r < dk; ++r) {
+#pragma unroll
+          for (int u = 0; u < kOut; ++u)
+            if (ti[u] < kTB) acc[u] = fmaf(Ks[ti[u] * ldk + r], Acc[r * ldw + ji[u]], acc[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < kOut; ++u) {
+          if (ti[u] >= kTB) continue;
+          for (int tp = ti[u]; tp < kTB; ++tp)
+            acc[u] = fmaf(S1[ti[u] * kLdS + tp], Ys[tp * ldv + ji[u]], acc[u]);
+          Xs[ti[u] * ldv + ji[u]] = acc[u];
+        }
+      }
+      {
+        float acc[kOut];
+        int ti[kOut], ri[kOut];
+#pragma unroll
+        for (int u = 0; u < kOut; ++u) {
+          ti[u] = row_of(u, dk), ri[u] = col_of(u, dk), acc[u] = 0.f;
+        }
+        #pragma unroll 4
+        for (int j = 0; j < dv; ++j) {
+#pragma unroll
+          for (int u = 0; u < kOut; ++u)
+            if (ti[u] < kTB) acc[u] = fmaf(Es[ti[u] * ldv + j], Acc[ri[u] * ldw + j], acc[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < kOut; ++u) {
+          if (ti[u] >= kTB) continue;
+          for (int tp = ti[u]; tp < kTB; ++tp)
+            acc[u] = fmaf(S2[ti[u] * kLdS + tp], Qs[tp * ldk + ri[u]], acc[u]);
+          Zs[ti[u] * ldk + ri[u]] = acc[u];
+        }
+      }
+      __syncthreads();
+      // deta_t = -(k_t R_t) . e_t; dv_t = eta_t k_t R_t; de_t = -dv_t (into Vs)
+      for (int t = warp; t < kTB; t += kThreads / 32) {
         float p = 0.f;
-        for (int j = tid; j < dv; j += kThreads) p = fmaf(kR[j], ev[j], p);
+        for (int j = lane; j < dv; j += 32) p = fmaf(Xs[t * ldv + j], Es[t * ldv + j], p);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
-        if ((tid & 31) == 0) red[tid >> 5] = p;
+        if (lane == 0 && t < nt) deta_out[t0 + t] = -p;
       }
-      __syncthreads();
-      if (tid == 0) {
-        float s = 0.f;
-        for (int w = 0; w < kThreads / 32; ++w) s += red[w];
-        dq_eta[t] = mse ? -s : s;
-      }
-      // dv_t and (MSE) de_t = -dv_t, kept in kR
-      for (int j = tid; j < dv; j += kThreads) {
-        const float dvj = et * kR[j];
-        st<T>(a.gv, b, h, t, j, dvj);
-        kR[j] = -dvj;
-      }
-      __syncthreads();
-      // dk_t; MSE: dL/dW_s += k_t^T de_t
-      for (int r = tid; r < dk; r += kThreads) {
-        float s;
-        if (mse) {
-          s = -et * Rx[r];
-          for (int j = 0; j < dv; ++j) s = fmaf(kR[j], Ws[r * dv + j], s);
-        } else {
-          s = et * Rx[r];
-        }
-        st<T>(a.gk, b, h, t, r, s);
-      }
-      if (mse) {
 #pragma unroll
-        for (int i = 0; i < kRegs; ++i) {
-          const int x = tid + i * kThreads;
-          if (x < n) acc[i] = fmaf(kv[x / dv], kR[x % dv], acc[i]);
+      for (int u = 0; u < kOut; ++u) {
+        const int t = row_of(u, dv), j = col_of(u, dv);
+        if (t < kTB) {
+          const float dvj = etas[t] * Xs[t * ldv + j];
+          if (t < nt) st<T>(a.gv, b, h, t0 + t, j, dvj);
+          Vs[t * ldv + j] = -dvj;
         }
       }
       __syncthreads();
-    }
-    // chunk start: G = R + sum_t k_t^T de_t carries into the previous chunk,
-    // whose end weights are this chunk's start weights
+      // dk_t = -eta_t R_t e_t^T (+ de_t W_s^T for MSE)
+      {
+        float acc[kOut];
+        int ti[kOut], ri[kOut];
 #pragma unroll
-    for (int i = 0; i < kRegs; ++i) {
-      const int x = tid + i * kThreads;
-      if (x < n) {
-        R[x] += acc[i];
-        acc[i] = 0.f;
+        for (int u = 0; u < kOut; ++u) {
+          ti[u] = row_of(u, dk), ri[u] = col_of(u, dk), acc[u] = 0.f;
+        }
+        if (mse)
+          #pragma unroll 4
+          for (int j = 0; j < dv; ++j) {
+#pragma unroll
+            for (int u = 0; u < kOut; ++u)
+              if (ti[u] < kTB) acc[u] = fmaf(Vs[ti[u] * ldv + j], Ws[ri[u] * ldw + j], acc[u]);
+          }
+#pragma unroll
+        for (int u = 0; u < kOut; ++u)
+          if (ti[u] < nt)
+            st<T>(a.gk, b, h, t0 + ti[u], ri[u],
+                  acc[u] - etas[ti[u]] * Zs[ti[u] * ldk + ri[u]]);
+      }
+      // R += Q^T dY (R is read above only before the last barrier);
+      // MSE: the chunk's sum_t k_t^T de_t
+      {
+        float yc[kTB], dc[kTB];  // this thread's column of dY and dE (kDiv)
+        if constexpr (kDiv) {
+#pragma unroll
+          for (int t = 0; t < kTB; ++t) {
+            yc[t] = Ys[t * ldv + tid % dv];
+            dc[t] = Vs[t * ldv + tid % dv];
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kRegs; ++u) {
+          const int r = row_of(u, dv), j = col_of(u, dv);
+          if (r < dk) {
+            float rr = Acc[r * ldw + j];
+#pragma unroll
+            for (int t = 0; t < kTB; ++t)
+              rr = fmaf(Qs[t * ldk + r], kDiv ? yc[t] : Ys[t * ldv + j], rr);
+            Acc[r * ldw + j] = rr;
+            if (mse) {
+#pragma unroll
+              for (int t = 0; t < kTB; ++t)
+                kde[u] = fmaf(Ks[t * ldk + r], kDiv ? dc[t] : Vs[t * ldv + j], kde[u]);
+            }
+          }
+        }
       }
     }
-    if (mse)
-      for (int x = tid; x < n; x += kThreads) Wt[x] = Ws[x];
-    __syncthreads();
+    // chunk start: dL/dW_s = R + sum_t k_t^T de_t is the previous chunk's G
+    // (each thread updates the elements it accumulated)
+#pragma unroll
+    for (int u = 0; u < kRegs; ++u) {
+      const int r = row_of(u, dv), j = col_of(u, dv);
+      if (r < dk) {
+        Acc[r * ldw + j] += kde[u];
+        kde[u] = 0.f;
+      }
+    }
   }
+  __syncthreads();
   float* dW = a.dW + (int64_t)bh * n;
-  for (int x = tid; x < n; x += kThreads) dW[x] = R[x];
+  for (int x = tid; x < n; x += kThreads) dW[x] = Acc[(x / dv) * ldw + x % dv];
 }
 
 // dL/dW0 of a weight shared over the batch: the sum over b in a fixed order.
@@ -228,7 +428,9 @@ __global__ void sum_over_batch_kernel(float* dst, const float* src, int B, int64
 
 }  // namespace
 
-bool ttt_linear_bwd_supported(int dk, int dv) { return dk <= 128 && dv <= 128 && dk * dv <= kMaxElems; }
+bool ttt_linear_bwd_supported(int dk, int dv) {
+  return dk >= 1 && dv >= 1 && dk <= kMaxD && dv <= kMaxD;
+}
 
 size_t ttt_linear_bwd_workspace(const LinearBwdArgs& a, bool w0_shared) {
   const int64_t n = (int64_t)a.dk * a.dv, Z = (int64_t)a.B * a.H;
@@ -250,19 +452,20 @@ cudaError_t launch_ttt_linear_bwd(LinearBwdArgs a, bool bf16, bool w0_shared, fl
     f += Z * a.nchunks * n;
   }
   a.dW = w0_shared ? f : dW0;
-  const size_t smem = sizeof(float) * (3 * n + 3 * a.dk + 4 * a.dv + 9);
+  const size_t smem = sizeof(float) * bwd_smem_floats(a.dk, a.dv);
+  const bool div = kThreads % a.dk == 0 && kThreads % a.dv == 0;
+  auto go = [&](auto kern) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess) kern<<<(int)Z, kThreads, smem, s>>>(a);
+    return e;
+  };
   cudaError_t e;
-  if (bf16) {
-    e = cudaFuncSetAttribute(ttt_linear_bwd_kernel<__nv_bfloat16>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    ttt_linear_bwd_kernel<__nv_bfloat16><<<(int)Z, kThreads, smem, s>>>(a);
-  } else {
-    e = cudaFuncSetAttribute(ttt_linear_bwd_kernel<float>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    ttt_linear_bwd_kernel<float><<<(int)Z, kThreads, smem, s>>>(a);
-  }
+  if (bf16)
+    e = div ? go(ttt_linear_bwd_kernel<__nv_bfloat16, true>)
+            : go(ttt_linear_bwd_kernel<__nv_bfloat16, false>);
+  else
+    e = div ? go(ttt_linear_bwd_kernel<float, true>) : go(ttt_linear_bwd_kernel<float, false>);
+  if (e != cudaSuccess) return e;
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (w0_shared) {
     const int64_t per_b = (int64_t)a.H * n;

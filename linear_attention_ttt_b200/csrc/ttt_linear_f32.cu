@@ -15,6 +15,8 @@
 //
 // Grid: (B*H, ceil(dv/32)); each CTA owns 32 output columns of one head. The
 // columns of W are independent in this rule, so no CTA talks to another.
+// The next block's tokens are fetched into registers while the current block
+// is computed, so that each block waits for at most one round of loads.
 #include "common.cuh"
 
 namespace ttt {
@@ -23,6 +25,10 @@ namespace {
 constexpr int kCols = 32;     // W columns per CTA
 constexpr int kTB = 16;       // tokens per block
 constexpr int kThreads = 256;
+constexpr int kMaxDk = 256;                        // the entry points reject larger heads
+constexpr int kQK = kTB * kMaxDk / kThreads;       // q and k values per thread and block
+constexpr int kV = kTB * kCols / kThreads;         // v values per thread and block
+static_assert(kV * kThreads == kTB * kCols, "v block split");
 
 template <typename T>
 __device__ __forceinline__ const T* tok_row(const TokView& v, int b, int h, int64_t t) {
@@ -30,7 +36,7 @@ __device__ __forceinline__ const T* tok_row(const TokView& v, int b, int h, int6
 }
 
 template <typename TT>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)
 ttt_linear_f32_kernel(LinearArgs a) {
   extern __shared__ float smem[];
   const int dk = a.dk, dv = a.dv;
@@ -58,61 +64,124 @@ ttt_linear_f32_kernel(LinearArgs a) {
   __syncthreads();
 
   const float* eta = a.eta.p + b * a.eta.sb + h * a.eta.sh;
+  if (!TTT_BOUNDS(dk <= kMaxDk && a.chunk > 0, a.status)) return;
+  // the block of tokens after the one at t0 (blocks never cross a chunk end)
+  auto block_len = [&](int t0) {
+    const int ce = min((t0 / a.chunk) * a.chunk + a.chunk, a.T);
+    return min(kTB, ce - t0);
+  };
+  float pq[kQK], pk[kQK], pv[kV], pe = 0.f;
+  auto fetch = [&](int t0, int nt) {
+#pragma unroll
+    for (int j = 0; j < kQK; ++j) {
+      const int x = tid + j * kThreads;
+      const int i = x / dk, c = x % dk;
+      const bool ok = x < kTB * dk && i < nt;
+      pq[j] = ok ? to_f32(tok_row<TT>(a.q, b, h, t0 + i)[c]) : 0.f;
+      pk[j] = ok ? to_f32(tok_row<TT>(a.k, b, h, t0 + i)[c]) : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < kV; ++j) {
+      const int x = tid + j * kThreads;
+      const int i = x / kCols, c = x % kCols;
+      pv[j] = (i < nt && c < ncol) ? to_f32(tok_row<TT>(a.v, b, h, t0 + i)[j0 + c]) : 0.f;
+    }
+    if (tid < kTB) pe = tid < nt ? eta[(int64_t)(t0 + tid) * a.eta.st] : 0.f;
+  };
+  if (a.T > 0) fetch(0, block_len(0));
   for (int cs = 0; cs < a.T; cs += a.chunk) {
     const int ce = min(cs + a.chunk, a.T);
     for (int t0 = cs; t0 < ce; t0 += kTB) {
       const int nt = min(kTB, ce - t0);
-      for (int x = tid; x < kTB * dk; x += kThreads) {
-        int i = x / dk, c = x % dk;
-        bool ok = i < nt;
-        Qs[x] = ok ? to_f32(tok_row<TT>(a.q, b, h, t0 + i)[c]) : 0.f;
-        Ks[x] = ok ? to_f32(tok_row<TT>(a.k, b, h, t0 + i)[c]) : 0.f;
+      // the previous block's last barrier has passed: the staging buffers are free
+#pragma unroll
+      for (int j = 0; j < kQK; ++j) {
+        const int x = tid + j * kThreads;
+        if (x < kTB * dk) Qs[x] = pq[j], Ks[x] = pk[j];
       }
-      for (int x = tid; x < kTB * kCols; x += kThreads) {
-        int i = x / kCols, c = x % kCols;
-        Vs[x] = (i < nt && c < ncol) ? to_f32(tok_row<TT>(a.v, b, h, t0 + i)[j0 + c]) : 0.f;
-      }
-      if (tid < kTB) etas[tid] = tid < nt ? eta[(int64_t)(t0 + tid) * a.eta.st] : 0.f;
+#pragma unroll
+      for (int j = 0; j < kV; ++j) Vs[tid + j * kThreads] = pv[j];
+      if (tid < kTB) etas[tid] = pe;
+      if (t0 + nt < a.T) fetch(t0 + nt, block_len(t0 + nt));
       __syncthreads();
 
-      // e_i at the chunk-start weights; scores q_t . k_i.
-      for (int x = tid; x < kTB * kCols; x += kThreads) {
-        int i = x / kCols, c = x % kCols;
-        float acc = 0.f;
+      // e_i at the chunk-start weights; scores q_t . k_i. Each thread owns
+      // kV outputs whose sums run side by side (each in its own fixed order).
+      {
+        float acc[kV] = {};
         if (a.loss == TTT_LOSS_MSE)
-          for (int r = 0; r < dk; ++r) acc = fmaf(Ks[i * dk + r], Wst[r * kCols + c], acc);
-        Es[x] = acc - Vs[x];
+          #pragma unroll 4
+          for (int r = 0; r < dk; ++r) {
+#pragma unroll
+            for (int j = 0; j < kV; ++j) {
+              const int x = tid + j * kThreads;
+              acc[j] = fmaf(Ks[(x / kCols) * dk + r], Wst[r * kCols + x % kCols], acc[j]);
+            }
+          }
+#pragma unroll
+        for (int j = 0; j < kV; ++j) Es[tid + j * kThreads] = acc[j] - Vs[tid + j * kThreads];
       }
       {
         int t = tid / kTB, i = tid % kTB;
         float acc = 0.f;
         if (i <= t)
+          #pragma unroll 4
           for (int r = 0; r < dk; ++r) acc = fmaf(Qs[t * dk + r], Ks[i * dk + r], acc);
         Ss[tid] = acc;
       }
       __syncthreads();
 
       // y_t = q_t (W_{t'} - dW) - sum_{i<=t} eta_i s_ti e_i
-      for (int x = tid; x < kTB * kCols; x += kThreads) {
-        int t = x / kCols, c = x % kCols;
-        if (t < nt && c < ncol) {
-          float acc = 0.f;
-          for (int r = 0; r < dk; ++r)
-            acc = fmaf(Qs[t * dk + r], Wst[r * kCols + c] - dW[r * kCols + c], acc);
-          for (int i = 0; i <= t; ++i) acc = fmaf(-etas[i] * Ss[t * kTB + i], Es[i * kCols + c], acc);
-          TT* o = static_cast<TT*>(a.out.p) + b * a.out.sb + h * a.out.sh +
-                  (int64_t)(t0 + t) * a.out.st;
-          o[j0 + c] = TT(acc);
+      {
+        float acc[kV] = {};
+        #pragma unroll 4
+        for (int r = 0; r < dk; ++r) {
+#pragma unroll
+          for (int j = 0; j < kV; ++j) {
+            const int x = tid + j * kThreads, t = x / kCols, c = x % kCols;
+            acc[j] = fmaf(Qs[t * dk + r], Wst[r * kCols + c] - dW[r * kCols + c], acc[j]);
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < kV; ++j) {
+          const int x = tid + j * kThreads, t = x / kCols, c = x % kCols;
+          if (t < nt && c < ncol) {
+            for (int i = 0; i <= t; ++i)
+              acc[j] = fmaf(-etas[i] * Ss[t * kTB + i], Es[i * kCols + c], acc[j]);
+            TT* o = static_cast<TT*>(a.out.p) + b * a.out.sb + h * a.out.sh +
+                    (int64_t)(t0 + t) * a.out.st;
+            o[j0 + c] = TT(acc[j]);
+          }
         }
       }
       __syncthreads();
 
-      // dW += sum_i eta_i k_i^T e_i
-      for (int x = tid; x < dk * kCols; x += kThreads) {
-        int r = x / kCols, c = x % kCols;
-        float acc = dW[x];
-        for (int i = 0; i < nt; ++i) acc = fmaf(etas[i] * Ks[i * dk + r], Es[i * kCols + c], acc);
-        dW[x] = acc;
+      // dW += sum_i eta_i k_i^T e_i: thread (r0 = tid / kCols, c = tid % kCols)
+      // owns rows r0, r0 + 8, ..., eight of them at a time
+      {
+        constexpr int kRowStep = kThreads / kCols, kU = 8;
+        const int c = tid % kCols, r0 = tid / kCols;
+        for (int rb = 0; rb < dk; rb += kU * kRowStep) {
+          float acc[kU];
+#pragma unroll
+          for (int u = 0; u < kU; ++u) {
+            const int r = rb + r0 + u * kRowStep;
+            acc[u] = r < dk ? dW[r * kCols + c] : 0.f;
+          }
+          for (int i = 0; i < nt; ++i) {
+            const float e = Es[i * kCols + c];
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+              const int r = rb + r0 + u * kRowStep;
+              if (r < dk) acc[u] = fmaf(etas[i] * Ks[i * dk + r], e, acc[u]);
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < kU; ++u) {
+            const int r = rb + r0 + u * kRowStep;
+            if (r < dk) dW[r * kCols + c] = acc[u];
+          }
+        }
       }
       __syncthreads();
     }
