@@ -44,6 +44,8 @@ from linear_attention_ttt_b200 import ops, synth  # noqa: E402
 METRIC = "TTT-layer tokens/s on 1 B200; % of bf16 tensor peak or HBM GB/s roofline"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# fp32 FMA peak from the unit counts: 148 SMs x 128 fp32 lanes x 2 FLOP x 1.965 GHz
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 def peaks():
@@ -67,6 +69,14 @@ def linear_bytes(w):
     per_head_token = (2 * w.dk + 2 * w.dv) * es + 4        # q, k, v in, y out, eta
     state = w.dk * w.dv * 4 * 2                             # W0 read + W_final write
     return w.B * w.H * (w.T * per_head_token + state)
+
+
+def linear_bwd_flops(w):
+    # The token-by-token chain rule: dq = dy W_t^T, the W_t update, R += q^T dy,
+    # k R and R e^T at 2 dk dv each, plus for MSE e = k W_s - v, de W_s^T and
+    # k^T de: 16 dk dv per head-token (MSE), 10 dk dv (inner product).
+    n = 16 if w.loss == synth.LOSS_MSE else 10
+    return w.B * w.H * w.T * n * w.dk * w.dv
 
 
 def linear_flops(w):
@@ -506,13 +516,15 @@ def measure_next_rows(runner, device):
             ach = work / (ms / 1e3) / (1e12 if unit == "TFLOP/s" else 1e9)
             item["roofline"] = {"bound": kind, "achieved": ach, "peak": peak, "unit": unit,
                                 "frac": ach / peak, "kernel": kernel,
-                                "peak_source": pk["_source"]}
+                                "peak_source": ("fp32 FMA lanes x max SM clock (derived)"
+                                                if kind == "alu" else pk["_source"])}
         out.append(item)
         torch.cuda.empty_cache()
 
-    # f1: TTT-Linear MSE / inner-product backward
-    for idx, T in ((3, 2048), (2, 1024)):
-        w = synth.config(idx, T=T)
+    # f1: TTT-Linear MSE / inner-product backward, at the forward workloads' sizes
+    for idx in (3, 2):
+        w = synth.config(idx)
+        T = w.T
         t = {n: dev(getattr(w, n), w.dtype if n in "qkv" else synth.F32)
              for n in ("q", "k", "v", "eta", "W0")}
         dy = torch.randn_like(t["v"])
@@ -520,7 +532,8 @@ def measure_next_rows(runner, device):
             {"workload": w.name, "batch": w.B, "heads": w.H, "seq_len": T, "d": w.dk,
              "chunk": w.chunk},
             lambda: ops.ttt_linear_bwd(t["q"], t["k"], t["v"], t["eta"], t["W0"], w.chunk,
-                                       w.loss, dy), w.B * T)
+                                       w.loss, dy), w.B * T,
+            roof=("alu", linear_bwd_flops(w), FP32_ALU_TFLOPS, "TFLOP/s", "ttt_linear_bwd"))
         del t, dy
     # f1: LaCT backward (GD), one shortened head pair of the d = 128 shape
     w = synth.make_lact(1, 2, 4096, 128, 512, 1024, synth.UPDATE_GD, seed=1090)

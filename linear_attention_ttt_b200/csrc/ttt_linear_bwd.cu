@@ -41,8 +41,6 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kTB = 16;                                // tokens per block
 constexpr int kMaxD = 128;                             // dk, dv <= 128
-constexpr int kRegs = kMaxD * kMaxD / kThreads;        // weight elements per thread
-constexpr int kOut = kTB * kMaxD / kThreads;           // token-tile elements per thread
 constexpr int kLdS = kTB + 1;                          // row stride of the 16 x 16 tiles
 
 template <typename T>
@@ -75,15 +73,19 @@ __host__ __device__ constexpr size_t bwd_smem_floats(int dk, int dv) {
 // in pass u of a flat walk keeps its column: (tid + u * kThreads) % d = tid % d.
 // The index helpers then give the same elements with a column the compiler
 // sees as fixed, and loads along that column are shared across the passes.
-template <typename T, bool kDiv>
+// D: the largest dk, dv the instance takes (64 or 128); it sizes the
+// per-thread register arrays, so that small heads run a smaller body.
+template <typename T, bool kDiv, int D>
 __global__ void __launch_bounds__(kThreads, 1) ttt_linear_bwd_kernel(LinearBwdArgs a) {
+  constexpr int kRegs = D * D / kThreads;   // weight elements per thread
+  constexpr int kOut = kTB * D / kThreads;  // token-tile elements per thread
   extern __shared__ float smem[];
   const int dk = a.dk, dv = a.dv, n = dk * dv;
   const int ldw = dv + 1, ldk = dk + 1, ldv = dv + 1;
   const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool mse = a.loss == TTT_LOSS_MSE;
-  if (!TTT_BOUNDS(dk <= kMaxD && dv <= kMaxD && a.chunk > 0 &&
+  if (!TTT_BOUNDS(dk <= D && dv <= D && a.chunk > 0 &&
                       (!kDiv || (kThreads % dk == 0 && kThreads % dv == 0)),
                   a.status))
     return;
@@ -459,12 +461,23 @@ cudaError_t launch_ttt_linear_bwd(LinearBwdArgs a, bool bf16, bool w0_shared, fl
     if (e == cudaSuccess) kern<<<(int)Z, kThreads, smem, s>>>(a);
     return e;
   };
+  const bool small = a.dk <= 64 && a.dv <= 64;
   cudaError_t e;
-  if (bf16)
-    e = div ? go(ttt_linear_bwd_kernel<__nv_bfloat16, true>)
-            : go(ttt_linear_bwd_kernel<__nv_bfloat16, false>);
-  else
-    e = div ? go(ttt_linear_bwd_kernel<float, true>) : go(ttt_linear_bwd_kernel<float, false>);
+  if (bf16) {
+    if (small)
+      e = div ? go(ttt_linear_bwd_kernel<__nv_bfloat16, true, 64>)
+              : go(ttt_linear_bwd_kernel<__nv_bfloat16, false, 64>);
+    else
+      e = div ? go(ttt_linear_bwd_kernel<__nv_bfloat16, true, 128>)
+              : go(ttt_linear_bwd_kernel<__nv_bfloat16, false, 128>);
+  } else {
+    if (small)
+      e = div ? go(ttt_linear_bwd_kernel<float, true, 64>)
+              : go(ttt_linear_bwd_kernel<float, false, 64>);
+    else
+      e = div ? go(ttt_linear_bwd_kernel<float, true, 128>)
+              : go(ttt_linear_bwd_kernel<float, false, 128>);
+  }
   if (e != cudaSuccess) return e;
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (w0_shared) {

@@ -27,6 +27,7 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kTB = 16;
 constexpr int kP = kTB + 1;   // padded token stride of the block buffers
+constexpr int kB = 8;         // global reads issued together per thread
 
 template <typename T>
 __device__ __forceinline__ float ldt(const TokView& v, int b, int h, int64_t t, int c) {
@@ -85,14 +86,33 @@ __global__ void __launch_bounds__(kThreads) ttt_mlp_kernel(MlpArgs a) {
     const int ce = min(cs + a.chunk, a.T);
     for (int t0 = cs; t0 < ce; t0 += kTB) {
       const int nt = min(kTB, ce - t0);
-      for (int x = tid; x < kTB * dk; x += kThreads) {
-        const int i = x / dk, c = x % dk;
-        Qs[c * kP + i] = i < nt ? ldt<T>(a.q, b, h, t0 + i, c) : 0.f;
-        Ks[c * kP + i] = i < nt ? ldt<T>(a.k, b, h, t0 + i, c) : 0.f;
+      for (int x0 = 0; x0 < kTB * dk; x0 += kB * kThreads) {
+        float qv[kB], kv[kB];
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+          const int x = x0 + tid + u * kThreads, i = x / dk, c = x % dk;
+          const bool ok = x < kTB * dk && i < nt;
+          qv[u] = ok ? ldt<T>(a.q, b, h, t0 + i, c) : 0.f;
+          kv[u] = ok ? ldt<T>(a.k, b, h, t0 + i, c) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+          const int x = x0 + tid + u * kThreads, i = x / dk, c = x % dk;
+          if (x < kTB * dk) Qs[c * kP + i] = qv[u], Ks[c * kP + i] = kv[u];
+        }
       }
-      for (int x = tid; x < kTB * dv; x += kThreads) {
-        const int i = x / dv, c = x % dv;
-        Vs[c * kP + i] = i < nt ? ldt<T>(a.v, b, h, t0 + i, c) : 0.f;
+      for (int x0 = 0; x0 < kTB * dv; x0 += kB * kThreads) {
+        float vv[kB];
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+          const int x = x0 + tid + u * kThreads, i = x / dv, c = x % dv;
+          vv[u] = x < kTB * dv && i < nt ? ldt<T>(a.v, b, h, t0 + i, c) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+          const int x = x0 + tid + u * kThreads, i = x / dv, c = x % dv;
+          if (x < kTB * dv) Vs[c * kP + i] = vv[u];
+        }
       }
       if (tid < kTB) et[tid] = tid < nt ? eta[(int64_t)(t0 + tid) * a.eta.st] : 0.f;
       __syncthreads();
@@ -102,6 +122,7 @@ __global__ void __launch_bounds__(kThreads) ttt_mlp_kernel(MlpArgs a) {
         float hk = sb1[j], zq = rb1[j];
         const float* w = sW1 + (int64_t)j * dk;
         const float* wr = rW1 + (int64_t)j * dk;
+        #pragma unroll 8
         for (int r = 0; r < dk; ++r) {
           hk = fmaf(w[r], Ks[r * kP + i], hk);
           zq = fmaf(wr[r], Qs[r * kP + i], zq);
@@ -126,6 +147,7 @@ __global__ void __launch_bounds__(kThreads) ttt_mlp_kernel(MlpArgs a) {
         const int c = x / kTB, i = x % kTB;
         float sv = sb2[c];
         const float* w = sW2 + (int64_t)c * dh;
+        #pragma unroll 8
         for (int j = 0; j < dh; ++j) sv = fmaf(w[j], Hs[j * kP + i], sv);
         Vs[c * kP + i] = sv - Vs[c * kP + i];
       }
@@ -134,6 +156,7 @@ __global__ void __launch_bounds__(kThreads) ttt_mlp_kernel(MlpArgs a) {
       for (int x = tid; x < kTB * dh; x += kThreads) {
         const int j = x / kTB, i = x % kTB;
         float sv = 0.f;
+        #pragma unroll 8
         for (int c = 0; c < dv; ++c) sv = fmaf(sW2[(int64_t)c * dh + j], Vs[c * kP + i], sv);
         Gs[j * kP + i] = sv * Hm[j * kP + i];
       }
@@ -163,6 +186,7 @@ __global__ void __launch_bounds__(kThreads) ttt_mlp_kernel(MlpArgs a) {
         if (t < nt) {
           float y = rb2[c];
           const float* w = rW2 + (int64_t)c * dh;
+          #pragma unroll 8
           for (int j = 0; j < dh; ++j) y = fmaf(w[j], Zs[j * kP + t], y);
           for (int i = 0; i <= t; ++i) y = fmaf(-et[i] * S2[t * kP + i], Vs[c * kP + i], y);
           T* o = static_cast<T*>(a.out.p) + b * a.out.sb + h * a.out.sh + (int64_t)(t0 + t) * a.out.st;
@@ -171,22 +195,46 @@ __global__ void __launch_bounds__(kThreads) ttt_mlp_kernel(MlpArgs a) {
       }
       __syncthreads();
       // running parameters: subtract this block's eta-weighted gradients
-      for (int64_t x = tid; x < (int64_t)dh * dk; x += kThreads) {
-        const int j = (int)(x / dk), r = (int)(x % dk);
-        float sv = 0.f;
-        for (int i = 0; i < nt; ++i) sv = fmaf(et[i] * Gs[j * kP + i], Ks[r * kP + i], sv);
-        rW1[x] -= sv;
+      // (the weight updates read and write the workspace in batches of kB
+      // elements per thread, so that each batch waits for one L2 round trip)
+      for (int64_t x0 = 0; x0 < (int64_t)dh * dk; x0 += kB * kThreads) {
+        float old[kB];
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+          const int64_t x = x0 + tid + u * kThreads;
+          old[u] = x < (int64_t)dh * dk ? rW1[x] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+          const int64_t x = x0 + tid + u * kThreads;
+          if (x >= (int64_t)dh * dk) continue;
+          const int j = (int)(x / dk), r = (int)(x % dk);
+          float sv = 0.f;
+          for (int i = 0; i < nt; ++i) sv = fmaf(et[i] * Gs[j * kP + i], Ks[r * kP + i], sv);
+          rW1[x] = old[u] - sv;
+        }
       }
       for (int j = tid; j < dh; j += kThreads) {
         float sv = 0.f;
         for (int i = 0; i < nt; ++i) sv = fmaf(et[i], Gs[j * kP + i], sv);
         rb1[j] -= sv;
       }
-      for (int64_t x = tid; x < (int64_t)dv * dh; x += kThreads) {
-        const int c = (int)(x / dh), j = (int)(x % dh);
-        float sv = 0.f;
-        for (int i = 0; i < nt; ++i) sv = fmaf(et[i] * Vs[c * kP + i], Hs[j * kP + i], sv);
-        rW2[x] -= sv;
+      for (int64_t x0 = 0; x0 < (int64_t)dv * dh; x0 += kB * kThreads) {
+        float old[kB];
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+          const int64_t x = x0 + tid + u * kThreads;
+          old[u] = x < (int64_t)dv * dh ? rW2[x] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+          const int64_t x = x0 + tid + u * kThreads;
+          if (x >= (int64_t)dv * dh) continue;
+          const int c = (int)(x / dh), j = (int)(x % dh);
+          float sv = 0.f;
+          for (int i = 0; i < nt; ++i) sv = fmaf(et[i] * Vs[c * kP + i], Hs[j * kP + i], sv);
+          rW2[x] = old[u] - sv;
+        }
       }
       for (int c = tid; c < dv; c += kThreads) {
         float sv = 0.f;
@@ -196,7 +244,19 @@ __global__ void __launch_bounds__(kThreads) ttt_mlp_kernel(MlpArgs a) {
       __syncthreads();
     }
     // chunk end: the running parameters start the next chunk
-    for (int64_t x = tid; x < nP; x += kThreads) ps[x] = ps[nP + x];
+    for (int64_t x0 = 0; x0 < nP; x0 += kB * kThreads) {
+      float v[kB];
+#pragma unroll
+      for (int u = 0; u < kB; ++u) {
+        const int64_t x = x0 + tid + u * kThreads;
+        v[u] = x < nP ? ps[nP + x] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kB; ++u) {
+        const int64_t x = x0 + tid + u * kThreads;
+        if (x < nP) ps[x] = v[u];
+      }
+    }
     __syncthreads();
   }
 
