@@ -7,7 +7,7 @@ Cases (synthetic inputs with the workloads' distributions, shortened):
   window       window attention, B1 H8 T16384 d128, window 4096
   lact_window  the LaCT Muon layer plus window attention, B1 H8 T16384 d128 dh512 b4096
   ttt_mlp      TTT-MLP, B4 H16 T2048 d64 dh256 chunk 16, bf16
-  linear_bwd   TTT-Linear MSE backward, B8 H16 T1024 d64 chunk 16, bf16
+  linear_bwd   TTT-Linear MSE backward, B8 H16 T2048 d64 chunk 16, bf16
   lact_bwd     LaCT GD backward, B1 H2 T2048 d128 dh512 chunk 1024, bf16
   momentum     LaCT with momentum (beta 0.9), B2 H4 T8192 d256 dh512 chunk 2048
 """
@@ -51,7 +51,7 @@ def make_case(name):
         Pd = [_dev(p, synth.F32) for p in P]
         return lambda: ops.ttt_mlp_fwd(*t, *Pd, 16)
     if name == "linear_bwd":
-        w = synth.config(3, T=1024)
+        w = synth.config(3, T=2048)
         t = [_dev(getattr(w, n), w.dtype if n in ("q", "k", "v") else synth.F32)
              for n in ("q", "k", "v", "eta", "W0")]
         dy = torch.randn_like(t[2])
