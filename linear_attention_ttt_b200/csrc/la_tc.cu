@@ -20,7 +20,8 @@
 // The A operands come from tensor memory, so the only shared-memory operands
 // are Q, K (from TMA) and P (written by the score warps).
 //
-// Each (batch, head) runs on two CTAs that split the sequence at tile `mid`.
+// Each (batch, head) runs on two CTAs that split the sequence at tile `mid`
+// (CTA 1 takes 7/16 of the tiles, rounded down).
 // CTA 0 handles tiles [0, mid). CTA 1 first builds the state after tile mid-1
 // with MMAs only: per tile, K scaled by eta in place and
 // S^T += V^T (diag(eta) K) with both operands in shared memory. It then
@@ -50,6 +51,10 @@ constexpr int kStages = 4;     // Q/K/V ring
 constexpr int kThreads = 512;
 constexpr int kVtWarp0 = 4, kScWarp0 = 8, kOutWarp0 = 12;
 constexpr int kL2Ahead = 4;    // tiles prefetched into L2 ahead of the smem ring
+// CTA 1's share of the tiles, in sixteenths (rounded down): it also rebuilds
+// the state over CTA 0's tiles, so an even split leaves CTA 0 idle at the end
+// (B4 H16 T4096: 7/16 111.5 us, 8/16 113.6 us, 6/16 114.1 us, 5/16 122.8 us).
+constexpr int kSeg1Sixteenths = 7;
 constexpr uint32_t kTileBytes = TT * D * 2;   // one bf16 [64 x 128] tile, 16 KB
 
 // TMEM columns
@@ -130,7 +135,7 @@ __global__ void __launch_bounds__(kThreads, 1) la_tc_kernel(const __grid_constan
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.x >> 1, seg = blockIdx.x & 1, b = bh / p.H, h = bh % p.H;
   if (!TTT_BOUNDS(bh < p.B * p.H, p.status)) return;  // uniform over both CTAs of the head
-  const int ntot = (p.T + TT - 1) / TT, mid = (ntot + 1) / 2;
+  const int ntot = (p.T + TT - 1) / TT, mid = ntot - (ntot * kSeg1Sixteenths) / 16;
   // tiles [0, p1) build the state only; tiles [p1, tend) run the full loop
   const int p1 = seg ? mid : 0, tend = seg ? ntot : mid, n2 = tend - p1;
   const int s0 = seg ? 1 : 0;  // s_ready phase of the first full tile
