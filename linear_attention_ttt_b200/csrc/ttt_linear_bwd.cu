@@ -24,7 +24,7 @@
 //   dL/dW_s = G + Q^T dY (+ K^T dE for MSE),
 // so only G links one chunk to the one before it.
 //
-// Layout: one CTA of 256 threads per (batch, head), fp32 arithmetic on the
+// Layout: one CTA of 256 (heads up to 64) or 512 threads per (batch, head), fp32 arithmetic on the
 // CUDA cores, 16-token blocks staged in shared memory. Pass 1 walks the
 // chunks forward: it stores the chunk-start weights (MSE) in a workspace and
 // computes dQ with the running sum of the chunk's updates. Pass 2 walks the
@@ -38,7 +38,9 @@
 namespace ttt {
 namespace {
 
-constexpr int kThreads = 256;
+// threads per CTA: 256 for heads up to 64, 512 for heads up to 128 (so that
+// the per-thread register arrays stay at 16-32 elements)
+__host__ __device__ constexpr int threads_for(int D) { return D == 128 ? 512 : 256; }
 constexpr int kTB = 16;                                // tokens per block
 constexpr int kMaxD = 128;                             // dk, dv <= 128
 constexpr int kLdS = kTB + 1;                          // row stride of the 16 x 16 tiles
@@ -70,15 +72,16 @@ __host__ __device__ constexpr size_t bwd_smem_floats(int dk, int dv) {
 }
 
 // kDiv: dk and dv divide the thread count, so that the element a thread owns
-// in pass u of a flat walk keeps its column: (tid + u * kThreads) % d = tid % d.
+// in pass u of a flat walk keeps its column: (tid + u * kNT) % d = tid % d.
 // The index helpers then give the same elements with a column the compiler
 // sees as fixed, and loads along that column are shared across the passes.
 // D: the largest dk, dv the instance takes (64 or 128); it sizes the
 // per-thread register arrays, so that small heads run a smaller body.
 template <typename T, bool kDiv, int D>
-__global__ void __launch_bounds__(kThreads, 1) ttt_linear_bwd_kernel(LinearBwdArgs a) {
-  constexpr int kRegs = D * D / kThreads;   // weight elements per thread
-  constexpr int kOut = kTB * D / kThreads;  // token-tile elements per thread
+__global__ void __launch_bounds__(threads_for(D), 1) ttt_linear_bwd_kernel(LinearBwdArgs a) {
+  constexpr int kNT = threads_for(D);
+  constexpr int kRegs = D * D / kNT;   // weight elements per thread
+  constexpr int kOut = kTB * D / kNT;  // token-tile elements per thread
   extern __shared__ float smem[];
   const int dk = a.dk, dv = a.dv, n = dk * dv;
   const int ldw = dv + 1, ldk = dk + 1, ldv = dv + 1;
@@ -86,14 +89,14 @@ __global__ void __launch_bounds__(kThreads, 1) ttt_linear_bwd_kernel(LinearBwdAr
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool mse = a.loss == TTT_LOSS_MSE;
   if (!TTT_BOUNDS(dk <= D && dv <= D && a.chunk > 0 &&
-                      (!kDiv || (kThreads % dk == 0 && kThreads % dv == 0)),
+                      (!kDiv || (kNT % dk == 0 && kNT % dv == 0)),
                   a.status))
     return;
-  // row and column of element tid + u * kThreads of a flat [.][d] walk
+  // row and column of element tid + u * kNT of a flat [.][d] walk
   auto row_of = [&](int u, int d) {
-    return kDiv ? tid / d + (kThreads / d) * u : (tid + u * kThreads) / d;
+    return kDiv ? tid / d + (kNT / d) * u : (tid + u * kNT) / d;
   };
-  auto col_of = [&](int u, int d) { return kDiv ? tid % d : (tid + u * kThreads) % d; };
+  auto col_of = [&](int u, int d) { return kDiv ? tid % d : (tid + u * kNT) % d; };
 
   float* Ws = smem;              // [dk][ldw] chunk-start weights
   float* Acc = Ws + dk * ldw;    // [dk][ldw] pass 1: the chunk's updates so far; pass 2: R
@@ -144,7 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1) ttt_linear_bwd_kernel(LinearBwdAr
   // a dense [dk][dv] fp32 matrix into a weight-shaped array (asynchronous;
   // cp_async_wait_all and a barrier before use)
   auto fetch_weights = [&](float* dst, const float* src) {
-    for (int x = tid; x < n; x += kThreads) cp_async4(dst + (x / dv) * ldw + x % dv, src + x);
+    for (int x = tid; x < n; x += kNT) cp_async4(dst + (x / dv) * ldw + x % dv, src + x);
   };
   // E = K W_s - V (MSE) or -V (inner product)
   auto make_e = [&]() {
@@ -173,7 +176,7 @@ __global__ void __launch_bounds__(kThreads, 1) ttt_linear_bwd_kernel(LinearBwdAr
   float* ck = a.ckpt ? a.ckpt + (int64_t)bh * a.nchunks * n : nullptr;
   for (int c = 0; c < a.nchunks; ++c) {
     const int s0 = c * a.chunk, e0 = min(s0 + a.chunk, a.T);
-    for (int x = tid; x < n; x += kThreads) {
+    for (int x = tid; x < n; x += kNT) {
       const int r = x / dv, j = x % dv;
       if (mse) ck[(int64_t)c * n + x] = Ws[r * ldw + j];
       Acc[r * ldw + j] = 0.f;
@@ -186,7 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1) ttt_linear_bwd_kernel(LinearBwdAr
       make_e();
       __syncthreads();
       // S1[t][i] = eta_i (dy_t . e_i) for i <= t
-      {
+      if (tid < kTB * kTB) {
         const int t = tid / kTB, i = tid % kTB;
         float acc = 0.f;
         if (i <= t && t < nt)
@@ -220,12 +223,12 @@ __global__ void __launch_bounds__(kThreads, 1) ttt_linear_bwd_kernel(LinearBwdAr
       }
       __syncthreads();
       // Acc += K^T N E
-      for (int x0 = 0; x0 < n; x0 += 8 * kThreads) {
+      for (int x0 = 0; x0 < n; x0 += 8 * kNT) {
         float acc[8];
         int ri[8], ji[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-          ri[u] = row_of(x0 / kThreads + u, dv), ji[u] = col_of(x0 / kThreads + u, dv);
+          ri[u] = row_of(x0 / kNT + u, dv), ji[u] = col_of(x0 / kNT + u, dv);
           acc[u] = ri[u] < dk ? Acc[ri[u] * ldw + ji[u]] : 0.f;
         }
         for (int i = 0; i < nt; ++i) {
@@ -239,7 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1) ttt_linear_bwd_kernel(LinearBwdAr
       }
     }
     __syncthreads();
-    for (int x = tid; x < n; x += kThreads) {
+    for (int x = tid; x < n; x += kNT) {
       const int r = x / dv, j = x % dv;
       Ws[r * ldw + j] -= Acc[r * ldw + j];
     }
@@ -252,7 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1) ttt_linear_bwd_kernel(LinearBwdAr
     fetch_weights(Acc, G0);
     cp_async_wait_all();
   } else {
-    for (int x = tid; x < n; x += kThreads) Acc[(x / dv) * ldw + x % dv] = 0.f;
+    for (int x = tid; x < n; x += kNT) Acc[(x / dv) * ldw + x % dv] = 0.f;
   }
   float kde[kRegs];  // this thread's part of sum_t k_t^T de_t over the chunk
 #pragma unroll
@@ -271,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1) ttt_linear_bwd_kernel(LinearBwdAr
       __syncthreads();
       make_e();
       // S1[t][t'] = k_t . q_t' for t <= t'
-      {
+      if (tid < kTB * kTB) {
         const int t = tid / kTB, tp = tid % kTB;
         float acc = 0.f;
         if (t <= tp && tp < nt)
@@ -281,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1) ttt_linear_bwd_kernel(LinearBwdAr
       }
       __syncthreads();
       // S2[t][t'] = e_t . dy_t' for t <= t'
-      {
+      if (tid < kTB * kTB) {
         const int t = tid / kTB, tp = tid % kTB;
         float acc = 0.f;
         if (t <= tp && tp < nt)
@@ -335,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1) ttt_linear_bwd_kernel(LinearBwdAr
       }
       __syncthreads();
       // deta_t = -(k_t R_t) . e_t; dv_t = eta_t k_t R_t; de_t = -dv_t (into Vs)
-      for (int t = warp; t < kTB; t += kThreads / 32) {
+      for (int t = warp; t < kTB; t += kNT / 32) {
         float p = 0.f;
         for (int j = lane; j < dv; j += 32) p = fmaf(Xs[t * ldv + j], Es[t * ldv + j], p);
 #pragma unroll
@@ -415,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1) ttt_linear_bwd_kernel(LinearBwdAr
   }
   __syncthreads();
   float* dW = a.dW + (int64_t)bh * n;
-  for (int x = tid; x < n; x += kThreads) dW[x] = Acc[(x / dv) * ldw + x % dv];
+  for (int x = tid; x < n; x += kNT) dW[x] = Acc[(x / dv) * ldw + x % dv];
 }
 
 // dL/dW0 of a weight shared over the batch: the sum over b in a fixed order.
@@ -455,28 +458,29 @@ cudaError_t launch_ttt_linear_bwd(LinearBwdArgs a, bool bf16, bool w0_shared, fl
   }
   a.dW = w0_shared ? f : dW0;
   const size_t smem = sizeof(float) * bwd_smem_floats(a.dk, a.dv);
-  const bool div = kThreads % a.dk == 0 && kThreads % a.dv == 0;
-  auto go = [&](auto kern) {
+  auto go = [&](auto kern, int nt) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e == cudaSuccess) kern<<<(int)Z, kThreads, smem, s>>>(a);
+    if (e == cudaSuccess) kern<<<(int)Z, nt, smem, s>>>(a);
     return e;
   };
   const bool small = a.dk <= 64 && a.dv <= 64;
+  const int nt = threads_for(small ? 64 : 128);
+  const bool div = nt % a.dk == 0 && nt % a.dv == 0;
   cudaError_t e;
   if (bf16) {
     if (small)
-      e = div ? go(ttt_linear_bwd_kernel<__nv_bfloat16, true, 64>)
-              : go(ttt_linear_bwd_kernel<__nv_bfloat16, false, 64>);
+      e = div ? go(ttt_linear_bwd_kernel<__nv_bfloat16, true, 64>, nt)
+              : go(ttt_linear_bwd_kernel<__nv_bfloat16, false, 64>, nt);
     else
-      e = div ? go(ttt_linear_bwd_kernel<__nv_bfloat16, true, 128>)
-              : go(ttt_linear_bwd_kernel<__nv_bfloat16, false, 128>);
+      e = div ? go(ttt_linear_bwd_kernel<__nv_bfloat16, true, 128>, nt)
+              : go(ttt_linear_bwd_kernel<__nv_bfloat16, false, 128>, nt);
   } else {
     if (small)
-      e = div ? go(ttt_linear_bwd_kernel<float, true, 64>)
-              : go(ttt_linear_bwd_kernel<float, false, 64>);
+      e = div ? go(ttt_linear_bwd_kernel<float, true, 64>, nt)
+              : go(ttt_linear_bwd_kernel<float, false, 64>, nt);
     else
-      e = div ? go(ttt_linear_bwd_kernel<float, true, 128>)
-              : go(ttt_linear_bwd_kernel<float, false, 128>);
+      e = div ? go(ttt_linear_bwd_kernel<float, true, 128>, nt)
+              : go(ttt_linear_bwd_kernel<float, false, 128>, nt);
   }
   if (e != cudaSuccess) return e;
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
