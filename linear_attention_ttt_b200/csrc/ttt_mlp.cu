@@ -29,12 +29,19 @@ constexpr int kTB = 16;
 constexpr int kP = kTB + 1;   // padded token stride of the block buffers
 constexpr int kB = 8;         // global reads issued together per thread
 
+// floats of the block buffers (before any shared-memory parameter copy)
+__host__ __device__ constexpr int64_t mlp_buf_floats(int dk, int dv, int dh) {
+  return (int64_t)(2 * dk + dv + 4 * dh) * kP + 2 * kTB * kP + kTB;
+}
+
 template <typename T>
 __device__ __forceinline__ float ldt(const TokView& v, int b, int h, int64_t t, int c) {
   return to_f32((static_cast<const T*>(v.p) + b * v.sb + h * v.sh + t * v.st)[c]);
 }
 
-template <typename T>
+// kSP: the chunk-start parameters live in shared memory (when they fit beside
+// the block buffers); the running copy stays in the workspace.
+template <typename T, bool kSP>
 __global__ void __launch_bounds__(kThreads) ttt_mlp_kernel(MlpArgs a) {
   extern __shared__ float smem[];
   const int dk = a.dk, dv = a.dv, dh = a.dh;
@@ -44,7 +51,7 @@ __global__ void __launch_bounds__(kThreads) ttt_mlp_kernel(MlpArgs a) {
 
   // workspace: start and running copies of (W1, b1, W2, b2)
   float* ps = a.ws + (int64_t)bh * 2 * nP;
-  float* sW1 = ps;
+  float* sW1 = kSP ? smem + mlp_buf_floats(dk, dv, dh) : ps;
   float* sb1 = sW1 + (int64_t)dh * dk;
   float* sW2 = sb1 + dh;
   float* sb2 = sW2 + (int64_t)dv * dh;
@@ -86,6 +93,14 @@ __global__ void __launch_bounds__(kThreads) ttt_mlp_kernel(MlpArgs a) {
     const int ce = min(cs + a.chunk, a.T);
     for (int t0 = cs; t0 < ce; t0 += kTB) {
       const int nt = min(kTB, ce - t0);
+      // the queries read the running parameters; at a chunk's first block they
+      // equal the start copy, which kSP keeps in shared memory
+      const bool first = t0 == cs, last = t0 + kTB >= ce;
+      const bool from_start = kSP && first;
+      const float* zW1 = from_start ? sW1 : rW1;
+      const float* zb1 = from_start ? sb1 : rb1;
+      const float* zW2 = from_start ? sW2 : rW2;
+      const float* zb2 = from_start ? sb2 : rb2;
       for (int x0 = 0; x0 < kTB * dk; x0 += kB * kThreads) {
         float qv[kB], kv[kB];
 #pragma unroll
@@ -119,9 +134,9 @@ __global__ void __launch_bounds__(kThreads) ttt_mlp_kernel(MlpArgs a) {
       // h = W1_s k + b1_s, and z0 = W1_run q + b1_run (running: earlier blocks applied)
       for (int x = tid; x < kTB * dh; x += kThreads) {
         const int j = x / kTB, i = x % kTB;
-        float hk = sb1[j], zq = rb1[j];
+        float hk = sb1[j], zq = zb1[j];
         const float* w = sW1 + (int64_t)j * dk;
-        const float* wr = rW1 + (int64_t)j * dk;
+        const float* wr = zW1 + (int64_t)j * dk;
         #pragma unroll 8
         for (int r = 0; r < dk; ++r) {
           hk = fmaf(w[r], Ks[r * kP + i], hk);
@@ -184,8 +199,8 @@ __global__ void __launch_bounds__(kThreads) ttt_mlp_kernel(MlpArgs a) {
       for (int x = tid; x < kTB * dv; x += kThreads) {
         const int c = x / kTB, t = x % kTB;
         if (t < nt) {
-          float y = rb2[c];
-          const float* w = rW2 + (int64_t)c * dh;
+          float y = zb2[c];
+          const float* w = zW2 + (int64_t)c * dh;
           #pragma unroll 8
           for (int j = 0; j < dh; ++j) y = fmaf(w[j], Zs[j * kP + t], y);
           for (int i = 0; i <= t; ++i) y = fmaf(-et[i] * S2[t * kP + i], Vs[c * kP + i], y);
@@ -212,12 +227,14 @@ __global__ void __launch_bounds__(kThreads) ttt_mlp_kernel(MlpArgs a) {
           float sv = 0.f;
           for (int i = 0; i < nt; ++i) sv = fmaf(et[i] * Gs[j * kP + i], Ks[r * kP + i], sv);
           rW1[x] = old[u] - sv;
+          if (kSP && last) sW1[x] = old[u] - sv;
         }
       }
       for (int j = tid; j < dh; j += kThreads) {
         float sv = 0.f;
         for (int i = 0; i < nt; ++i) sv = fmaf(et[i], Gs[j * kP + i], sv);
         rb1[j] -= sv;
+        if (kSP && last) sb1[j] = rb1[j];
       }
       for (int64_t x0 = 0; x0 < (int64_t)dv * dh; x0 += kB * kThreads) {
         float old[kB];
@@ -234,17 +251,20 @@ __global__ void __launch_bounds__(kThreads) ttt_mlp_kernel(MlpArgs a) {
           float sv = 0.f;
           for (int i = 0; i < nt; ++i) sv = fmaf(et[i] * Vs[c * kP + i], Hs[j * kP + i], sv);
           rW2[x] = old[u] - sv;
+          if (kSP && last) sW2[x] = old[u] - sv;
         }
       }
       for (int c = tid; c < dv; c += kThreads) {
         float sv = 0.f;
         for (int i = 0; i < nt; ++i) sv = fmaf(et[i], Vs[c * kP + i], sv);
         rb2[c] -= sv;
+        if (kSP && last) sb2[c] = rb2[c];
       }
       __syncthreads();
     }
-    // chunk end: the running parameters start the next chunk
-    for (int64_t x0 = 0; x0 < nP; x0 += kB * kThreads) {
+    // chunk end: the running parameters start the next chunk (kSP: the last
+    // block's update already wrote them into shared memory)
+    for (int64_t x0 = 0; x0 < (kSP ? 0 : nP); x0 += kB * kThreads) {
       float v[kB];
 #pragma unroll
       for (int u = 0; u < kB; ++u) {
@@ -278,19 +298,25 @@ size_t ttt_mlp_workspace(const MlpArgs& a) {
 }
 
 cudaError_t launch_ttt_mlp(const MlpArgs& a, bool bf16, cudaStream_t s) {
-  const size_t smem = sizeof(float) * ((2 * a.dk + a.dv + 4 * a.dh) * kP + 2 * kTB * kP + kTB);
-  cudaError_t e;
-  if (bf16) {
-    e = cudaFuncSetAttribute(ttt_mlp_kernel<__nv_bfloat16>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    ttt_mlp_kernel<__nv_bfloat16><<<a.B * a.H, kThreads, smem, s>>>(a);
-  } else {
-    e = cudaFuncSetAttribute(ttt_mlp_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
-    if (e != cudaSuccess) return e;
-    ttt_mlp_kernel<float><<<a.B * a.H, kThreads, smem, s>>>(a);
-  }
+  const int64_t nP = (int64_t)a.dh * a.dk + a.dh + (int64_t)a.dv * a.dh + a.dv;
+  const size_t buf = sizeof(float) * mlp_buf_floats(a.dk, a.dv, a.dh);
+  int dev = 0, optin = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess)
+    e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (e != cudaSuccess) return e;
+  const bool sp = buf + sizeof(float) * nP <= (size_t)optin;
+  const size_t smem = buf + (sp ? sizeof(float) * nP : 0);
+  auto go = [&](auto kern) {
+    cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (r == cudaSuccess) kern<<<a.B * a.H, kThreads, smem, s>>>(a);
+    return r;
+  };
+  if (bf16)
+    e = sp ? go(ttt_mlp_kernel<__nv_bfloat16, true>) : go(ttt_mlp_kernel<__nv_bfloat16, false>);
+  else
+    e = sp ? go(ttt_mlp_kernel<float, true>) : go(ttt_mlp_kernel<float, false>);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
