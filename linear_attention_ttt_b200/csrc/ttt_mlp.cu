@@ -42,7 +42,7 @@ __device__ __forceinline__ float ldt(const TokView& v, int b, int h, int64_t t, 
 // kSP: the chunk-start parameters live in shared memory (when they fit beside
 // the block buffers); the running copy stays in the workspace.
 template <typename T, bool kSP>
-__global__ void __launch_bounds__(kThreads) ttt_mlp_kernel(MlpArgs a) {
+__global__ void __launch_bounds__(kThreads, kSP ? 1 : 2) ttt_mlp_kernel(MlpArgs a) {
   extern __shared__ float smem[];
   const int dk = a.dk, dv = a.dv, dh = a.dh;
   const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
@@ -211,13 +211,21 @@ __global__ void __launch_bounds__(kThreads) ttt_mlp_kernel(MlpArgs a) {
       __syncthreads();
       // running parameters: subtract this block's eta-weighted gradients
       // (the weight updates read and write the workspace in batches of kB
-      // elements per thread, so that each batch waits for one L2 round trip)
+      // elements per thread, so that each batch waits for one L2 round trip).
+      // kSP: at a chunk's first block the running values are the start copy in
+      // shared memory, and the last block's result, the next start, goes there;
+      // the workspace copy is kept only between the blocks of one chunk.
+      const bool run_in = kSP && first, run_out = !kSP || !last;
+      auto put = [&](float* rp, float* sp, int64_t x, float val) {
+        if (run_out) rp[x] = val;
+        if (kSP && last) sp[x] = val;
+      };
       for (int64_t x0 = 0; x0 < (int64_t)dh * dk; x0 += kB * kThreads) {
         float old[kB];
 #pragma unroll
         for (int u = 0; u < kB; ++u) {
           const int64_t x = x0 + tid + u * kThreads;
-          old[u] = x < (int64_t)dh * dk ? rW1[x] : 0.f;
+          old[u] = x < (int64_t)dh * dk ? (run_in ? sW1[x] : rW1[x]) : 0.f;
         }
 #pragma unroll
         for (int u = 0; u < kB; ++u) {
@@ -226,22 +234,20 @@ __global__ void __launch_bounds__(kThreads) ttt_mlp_kernel(MlpArgs a) {
           const int j = (int)(x / dk), r = (int)(x % dk);
           float sv = 0.f;
           for (int i = 0; i < nt; ++i) sv = fmaf(et[i] * Gs[j * kP + i], Ks[r * kP + i], sv);
-          rW1[x] = old[u] - sv;
-          if (kSP && last) sW1[x] = old[u] - sv;
+          put(rW1, sW1, x, old[u] - sv);
         }
       }
       for (int j = tid; j < dh; j += kThreads) {
         float sv = 0.f;
         for (int i = 0; i < nt; ++i) sv = fmaf(et[i], Gs[j * kP + i], sv);
-        rb1[j] -= sv;
-        if (kSP && last) sb1[j] = rb1[j];
+        put(rb1, sb1, j, (run_in ? sb1[j] : rb1[j]) - sv);
       }
       for (int64_t x0 = 0; x0 < (int64_t)dv * dh; x0 += kB * kThreads) {
         float old[kB];
 #pragma unroll
         for (int u = 0; u < kB; ++u) {
           const int64_t x = x0 + tid + u * kThreads;
-          old[u] = x < (int64_t)dv * dh ? rW2[x] : 0.f;
+          old[u] = x < (int64_t)dv * dh ? (run_in ? sW2[x] : rW2[x]) : 0.f;
         }
 #pragma unroll
         for (int u = 0; u < kB; ++u) {
@@ -250,15 +256,13 @@ __global__ void __launch_bounds__(kThreads) ttt_mlp_kernel(MlpArgs a) {
           const int c = (int)(x / dh), j = (int)(x % dh);
           float sv = 0.f;
           for (int i = 0; i < nt; ++i) sv = fmaf(et[i] * Vs[c * kP + i], Hs[j * kP + i], sv);
-          rW2[x] = old[u] - sv;
-          if (kSP && last) sW2[x] = old[u] - sv;
+          put(rW2, sW2, x, old[u] - sv);
         }
       }
       for (int c = tid; c < dv; c += kThreads) {
         float sv = 0.f;
         for (int i = 0; i < nt; ++i) sv = fmaf(et[i], Vs[c * kP + i], sv);
-        rb2[c] -= sv;
-        if (kSP && last) sb2[c] = rb2[c];
+        put(rb2, sb2, c, (run_in ? sb2[c] : rb2[c]) - sv);
       }
       __syncthreads();
     }
@@ -282,7 +286,8 @@ __global__ void __launch_bounds__(kThreads) ttt_mlp_kernel(MlpArgs a) {
 
   float* fin[4] = {a.W1_final, a.b1_final, a.W2_final, a.b2_final};
   const int64_t len[4] = {(int64_t)dh * dk, dh, (int64_t)dv * dh, dv};
-  const float* run[4] = {rW1, rb1, rW2, rb2};
+  // kSP: the final parameters are the start copy the last block wrote
+  const float* run[4] = {kSP ? sW1 : rW1, kSP ? sb1 : rb1, kSP ? sW2 : rW2, kSP ? sb2 : rb2};
   for (int m = 0; m < 4; ++m)
     if (fin[m])
       for (int64_t x = tid; x < len[m]; x += kThreads) fin[m][(int64_t)bh * len[m] + x] = run[m][x];

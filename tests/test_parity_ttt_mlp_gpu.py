@@ -68,3 +68,11 @@ def test_per_sequence_parameters_and_uneven_sizes():
 def test_empty_sequence_copies_parameters():
     w, P = case(1, 2, 0, 32, 32, 64, 16, synth.F32, seed=13)
     compare(w, P, "T0")
+
+
+@pytest.mark.parametrize("chunk", [16, 32])
+def test_parameters_beyond_shared_memory(chunk):
+    """dk = dv = 128, dh = 512: the parameters (527 KB) do not fit in shared
+    memory, so both copies stay in the workspace."""
+    w, P = case(1, 1, 50, 128, 128, 512, chunk, synth.F32, seed=14 + chunk)
+    compare(w, P, f"f32 d128 dh512 b{chunk}")
