@@ -13,18 +13,21 @@
 //   y_t = W2_t a'_t + b2_t = W2_s a'_t + b2_s - sum_{i<=t} eta_i (a'_t . a_i + 1) r_i,
 // with a'_t = ReLU(z_t): the dual (attention-like) form of the chunk.
 //
-// Layout: one CTA of 256 threads per (batch, head), fp32 arithmetic on the
-// CUDA cores. A chunk is walked in blocks of 16 tokens; the parameters live in
-// an fp32 workspace (L2-resident) as the chunk-start copy P_s, used for the
-// keys' h, a, r, g, and the running copy, which already holds the updates of
-// the chunk's earlier blocks and serves the queries.
+// Layout: one CTA of 512 threads per (batch, head), fp32 arithmetic on the
+// CUDA cores. A chunk is walked in blocks of 16 tokens with two parameter
+// copies: the chunk-start copy P_s, used for the keys' h, a, r, g (and for the
+// queries of a chunk's first block), and the running copy, which holds the
+// updates of the chunk's earlier blocks and serves the other queries. P_s
+// sits in shared memory when it fits beside the block buffers (d 64, hidden
+// 256: 132 KB + 85 KB), else in an fp32 workspace (L2-resident) like the
+// running copy; with single-block chunks the running copy is never needed.
 #include "common.cuh"
 
 namespace ttt {
 
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;  // 16 warps: the product loops are latency-bound
 constexpr int kTB = 16;
 constexpr int kP = kTB + 1;   // padded token stride of the block buffers
 constexpr int kB = 8;         // global reads issued together per thread
@@ -42,7 +45,7 @@ __device__ __forceinline__ float ldt(const TokView& v, int b, int h, int64_t t, 
 // kSP: the chunk-start parameters live in shared memory (when they fit beside
 // the block buffers); the running copy stays in the workspace.
 template <typename T, bool kSP>
-__global__ void __launch_bounds__(kThreads, kSP ? 1 : 2) ttt_mlp_kernel(MlpArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) ttt_mlp_kernel(MlpArgs a) {
   extern __shared__ float smem[];
   const int dk = a.dk, dv = a.dv, dh = a.dh;
   const int bh = blockIdx.x, b = bh / a.H, h = bh % a.H;
@@ -147,7 +150,7 @@ __global__ void __launch_bounds__(kThreads, kSP ? 1 : 2) ttt_mlp_kernel(MlpArgs 
         Zs[j * kP + i] = zq;
       }
       // S1[t][i] = q_t . k_i + 1 (i <= t)
-      {
+      if (tid < kTB * kTB) {
         const int t = tid / kTB, i = tid % kTB;
         float sv = 0.f;
         if (i <= t) {
@@ -185,7 +188,7 @@ __global__ void __launch_bounds__(kThreads, kSP ? 1 : 2) ttt_mlp_kernel(MlpArgs 
       }
       __syncthreads();
       // S2[t][i] = a'_t . a_i + 1 (i <= t)
-      {
+      if (tid < kTB * kTB) {
         const int t = tid / kTB, i = tid % kTB;
         float sv = 0.f;
         if (i <= t) {
