@@ -157,13 +157,14 @@ __global__ void __launch_bounds__(threads_for(D), 1) ttt_linear_bwd_kernel(Linea
     for (int u = 0; u < kOut; ++u) {
       ti[u] = row_of(u, dv), ji[u] = col_of(u, dv), acc[u] = 0.f;
     }
-    if (mse)
-      #pragma unroll 4
+    if (mse) {
+#pragma unroll 4
       for (int r = 0; r < dk; ++r) {
 #pragma unroll
         for (int u = 0; u < kOut; ++u)
           if (ti[u] < kTB) acc[u] = fmaf(Ks[ti[u] * ldk + r], Ws[r * ldw + ji[u]], acc[u]);
       }
+    }
 #pragma unroll
     for (int u = 0; u < kOut; ++u)
       if (ti[u] < kTB) Es[ti[u] * ldv + ji[u]] = acc[u] - Vs[ti[u] * ldv + ji[u]];
@@ -192,9 +193,10 @@ __global__ void __launch_bounds__(threads_for(D), 1) ttt_linear_bwd_kernel(Linea
       if (tid < kTB * kTB) {
         const int t = tid / kTB, i = tid % kTB;
         float acc = 0.f;
-        if (i <= t && t < nt)
-          #pragma unroll 4
+        if (i <= t && t < nt) {
+#pragma unroll 4
           for (int j = 0; j < dv; ++j) acc = fmaf(Ys[t * ldv + j], Es[i * ldv + j], acc);
+        }
         S1[t * kLdS + i] = etas[i] * acc;
       }
       __syncthreads();
@@ -206,7 +208,7 @@ __global__ void __launch_bounds__(threads_for(D), 1) ttt_linear_bwd_kernel(Linea
         for (int u = 0; u < kOut; ++u) {
           ti[u] = row_of(u, dk), ri[u] = col_of(u, dk), acc[u] = 0.f;
         }
-        #pragma unroll 4
+#pragma unroll 4
         for (int j = 0; j < dv; ++j) {
 #pragma unroll
           for (int u = 0; u < kOut; ++u)
@@ -277,9 +279,10 @@ __global__ void __launch_bounds__(threads_for(D), 1) ttt_linear_bwd_kernel(Linea
       if (tid < kTB * kTB) {
         const int t = tid / kTB, tp = tid % kTB;
         float acc = 0.f;
-        if (t <= tp && tp < nt)
-          #pragma unroll 4
+        if (t <= tp && tp < nt) {
+#pragma unroll 4
           for (int r = 0; r < dk; ++r) acc = fmaf(Ks[t * ldk + r], Qs[tp * ldk + r], acc);
+        }
         S1[t * kLdS + tp] = acc;
       }
       __syncthreads();
@@ -287,9 +290,10 @@ __global__ void __launch_bounds__(threads_for(D), 1) ttt_linear_bwd_kernel(Linea
       if (tid < kTB * kTB) {
         const int t = tid / kTB, tp = tid % kTB;
         float acc = 0.f;
-        if (t <= tp && tp < nt)
-          #pragma unroll 4
+        if (t <= tp && tp < nt) {
+#pragma unroll 4
           for (int j = 0; j < dv; ++j) acc = fmaf(Es[t * ldv + j], Ys[tp * ldv + j], acc);
+        }
         S2[t * kLdS + tp] = acc;
       }
       __syncthreads();
@@ -301,7 +305,7 @@ __global__ void __launch_bounds__(threads_for(D), 1) ttt_linear_bwd_kernel(Linea
         for (int u = 0; u < kOut; ++u) {
           ti[u] = row_of(u, dv), ji[u] = col_of(u, dv), acc[u] = 0.f;
         }
-        #pragma unroll 4
+#pragma unroll 4
         for (int r = 0; r < dk; ++r) {
 #pragma unroll
           for (int u = 0; u < kOut; ++u)
@@ -322,7 +326,7 @@ __global__ void __launch_bounds__(threads_for(D), 1) ttt_linear_bwd_kernel(Linea
         for (int u = 0; u < kOut; ++u) {
           ti[u] = row_of(u, dk), ri[u] = col_of(u, dk), acc[u] = 0.f;
         }
-        #pragma unroll 4
+#pragma unroll 4
         for (int j = 0; j < dv; ++j) {
 #pragma unroll
           for (int u = 0; u < kOut; ++u)
@@ -363,13 +367,14 @@ __global__ void __launch_bounds__(threads_for(D), 1) ttt_linear_bwd_kernel(Linea
         for (int u = 0; u < kOut; ++u) {
           ti[u] = row_of(u, dk), ri[u] = col_of(u, dk), acc[u] = 0.f;
         }
-        if (mse)
-          #pragma unroll 4
+        if (mse) {
+#pragma unroll 4
           for (int j = 0; j < dv; ++j) {
 #pragma unroll
             for (int u = 0; u < kOut; ++u)
               if (ti[u] < kTB) acc[u] = fmaf(Vs[ti[u] * ldv + j], Ws[ri[u] * ldw + j], acc[u]);
           }
+        }
 #pragma unroll
         for (int u = 0; u < kOut; ++u)
           if (ti[u] < nt)

@@ -109,8 +109,8 @@ ttt_linear_f32_kernel(LinearArgs a) {
       // kV outputs whose sums run side by side (each in its own fixed order).
       {
         float acc[kV] = {};
-        if (a.loss == TTT_LOSS_MSE)
-          #pragma unroll 4
+        if (a.loss == TTT_LOSS_MSE) {
+#pragma unroll 4
           for (int r = 0; r < dk; ++r) {
 #pragma unroll
             for (int j = 0; j < kV; ++j) {
@@ -118,15 +118,17 @@ ttt_linear_f32_kernel(LinearArgs a) {
               acc[j] = fmaf(Ks[(x / kCols) * dk + r], Wst[r * kCols + x % kCols], acc[j]);
             }
           }
+        }
 #pragma unroll
         for (int j = 0; j < kV; ++j) Es[tid + j * kThreads] = acc[j] - Vs[tid + j * kThreads];
       }
-      {
+      if (tid < kTB * kTB) {
         int t = tid / kTB, i = tid % kTB;
         float acc = 0.f;
-        if (i <= t)
-          #pragma unroll 4
+        if (i <= t) {
+#pragma unroll 4
           for (int r = 0; r < dk; ++r) acc = fmaf(Qs[t * dk + r], Ks[i * dk + r], acc);
+        }
         Ss[tid] = acc;
       }
       __syncthreads();
@@ -134,7 +136,7 @@ ttt_linear_f32_kernel(LinearArgs a) {
       // y_t = q_t (W_{t'} - dW) - sum_{i<=t} eta_i s_ti e_i
       {
         float acc[kV] = {};
-        #pragma unroll 4
+#pragma unroll 4
         for (int r = 0; r < dk; ++r) {
 #pragma unroll
           for (int j = 0; j < kV; ++j) {
