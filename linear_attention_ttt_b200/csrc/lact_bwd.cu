@@ -71,24 +71,45 @@ __global__ void __launch_bounds__(256) bgemm_kernel(GemmArgs g) {
   const int m0 = blockIdx.y * kGT, n0 = blockIdx.x * kGT;
   const int tid = threadIdx.x, tm = tid / 16, tn = tid % 16;
   float acc[4][4] = {};
-  for (int k0 = 0; k0 < g.K; k0 += kGK) {
-    for (int e = tid; e < kGK * kGT; e += 256) {
+  // The next K step's operands are fetched into registers while the current
+  // step is computed (every load of a step is issued before its stores).
+  constexpr int kPer = kGK * kGT / 256;  // operand elements per thread and step
+  float ra[kPer], rb[kPer];
+  auto fetch = [&](int k0) {
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int e = tid + 256 * i;
       int kk, mm;
       if (g.tA) { mm = e % kGT; kk = e / kGT; } else { kk = e % kGK; mm = e / kGK; }
       const int gm = m0 + mm, gk = k0 + kk;
-      float x = 0.f;
-      if (gm < g.M && gk < g.K) x = g.tA ? A[(int64_t)gk * g.lda + gm] : A[(int64_t)gm * g.lda + gk];
-      As[kk][mm] = x;
+      ra[i] = (gm < g.M && gk < g.K)
+                  ? (g.tA ? A[(int64_t)gk * g.lda + gm] : A[(int64_t)gm * g.lda + gk])
+                  : 0.f;
     }
-    for (int e = tid; e < kGK * kGT; e += 256) {
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int e = tid + 256 * i;
       int kk, nn;
       if (g.tB) { kk = e % kGK; nn = e / kGK; } else { nn = e % kGT; kk = e / kGT; }
       const int gn = n0 + nn, gk = k0 + kk;
-      float x = 0.f;
-      if (gn < g.N && gk < g.K) x = g.tB ? B[(int64_t)gn * g.ldb + gk] : B[(int64_t)gk * g.ldb + gn];
-      Bs[kk][nn] = x;
+      rb[i] = (gn < g.N && gk < g.K)
+                  ? (g.tB ? B[(int64_t)gn * g.ldb + gk] : B[(int64_t)gk * g.ldb + gn])
+                  : 0.f;
     }
+  };
+  auto stage = [&]() {
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int e = tid + 256 * i;
+      if (g.tA) As[e / kGT][e % kGT] = ra[i]; else As[e % kGK][e / kGK] = ra[i];
+      if (g.tB) Bs[e % kGK][e / kGK] = rb[i]; else Bs[e / kGT][e % kGT] = rb[i];
+    }
+  };
+  if (g.K > 0) fetch(0);
+  for (int k0 = 0; k0 < g.K; k0 += kGK) {
+    stage();
     __syncthreads();
+    if (k0 + kGK < g.K) fetch(k0 + kGK);
 #pragma unroll
     for (int kk = 0; kk < kGK; ++kk) {
       float a[4], b[4];
