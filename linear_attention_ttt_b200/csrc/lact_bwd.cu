@@ -59,15 +59,17 @@ struct GemmArgs {
   int M, N, K, lda, ldb, ldc, tA, tB;
   int64_t sA, sB, sC;
   float alpha, beta;
+  int Z, kper;  // blockIdx.z = split * Z + z; split s covers K range [s kper, (s + 1) kper)
 };
 
 __global__ void __launch_bounds__(256) bgemm_kernel(GemmArgs g) {
   __shared__ float As[kGK][kGT + 4];
   __shared__ float Bs[kGK][kGT + 4];
-  const int z = blockIdx.z;
+  const int zz = blockIdx.z, z = zz % g.Z, sp = zz / g.Z;
   const float* A = g.A + z * g.sA;
   const float* B = g.B + z * g.sB;
-  float* C = g.C + z * g.sC;
+  float* C = g.C + zz * g.sC;  // split partials (sp > 0) go to consecutive slabs
+  const int kb = sp * g.kper, ke = min(g.K, kb + g.kper);
   const int m0 = blockIdx.y * kGT, n0 = blockIdx.x * kGT;
   const int tid = threadIdx.x, tm = tid / 16, tn = tid % 16;
   float acc[4][4] = {};
@@ -82,7 +84,7 @@ __global__ void __launch_bounds__(256) bgemm_kernel(GemmArgs g) {
       int kk, mm;
       if (g.tA) { mm = e % kGT; kk = e / kGT; } else { kk = e % kGK; mm = e / kGK; }
       const int gm = m0 + mm, gk = k0 + kk;
-      ra[i] = (gm < g.M && gk < g.K)
+      ra[i] = (gm < g.M && gk < ke)
                   ? (g.tA ? A[(int64_t)gk * g.lda + gm] : A[(int64_t)gm * g.lda + gk])
                   : 0.f;
     }
@@ -92,7 +94,7 @@ __global__ void __launch_bounds__(256) bgemm_kernel(GemmArgs g) {
       int kk, nn;
       if (g.tB) { kk = e % kGK; nn = e / kGK; } else { nn = e % kGT; kk = e / kGT; }
       const int gn = n0 + nn, gk = k0 + kk;
-      rb[i] = (gn < g.N && gk < g.K)
+      rb[i] = (gn < g.N && gk < ke)
                   ? (g.tB ? B[(int64_t)gn * g.ldb + gk] : B[(int64_t)gk * g.ldb + gn])
                   : 0.f;
     }
@@ -105,11 +107,11 @@ __global__ void __launch_bounds__(256) bgemm_kernel(GemmArgs g) {
       if (g.tB) Bs[e % kGK][e / kGK] = rb[i]; else Bs[e / kGT][e % kGT] = rb[i];
     }
   };
-  if (g.K > 0) fetch(0);
-  for (int k0 = 0; k0 < g.K; k0 += kGK) {
+  if (kb < ke) fetch(kb);
+  for (int k0 = kb; k0 < ke; k0 += kGK) {
     stage();
     __syncthreads();
-    if (k0 + kGK < g.K) fetch(k0 + kGK);
+    if (k0 + kGK < ke) fetch(k0 + kGK);
 #pragma unroll
     for (int kk = 0; kk < kGK; ++kk) {
       float a[4], b[4];
@@ -134,6 +136,23 @@ __global__ void __launch_bounds__(256) bgemm_kernel(GemmArgs g) {
         *c = g.alpha * acc[i][j] + (g.beta != 0.f ? g.beta * *c : 0.f);
       }
     }
+}
+
+// C[z] = alpha sum_s part[s][z] + beta C[z], the split-K partials summed in
+// split order (deterministic).
+__global__ void splitk_reduce_kernel(const float* part, float* C, int Z, int M, int N, int ldc,
+                                     int64_t sC, int splits, float alpha, float beta) {
+  const int64_t mn = (int64_t)M * N, n = (int64_t)Z * mn;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int z = (int)(i / mn);
+    const int64_t r = i % mn;
+    const int m = (int)(r / N), c = (int)(r % N);
+    float acc = 0.f;
+    for (int sp = 0; sp < splits; ++sp) acc += part[((int64_t)sp * Z + z) * mn + r];
+    float* o = C + z * sC + (int64_t)m * ldc + c;
+    *o = alpha * acc + (beta != 0.f ? beta * *o : 0.f);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -401,16 +420,44 @@ struct Ctx {
     const int64_t b = (n + per - 1) / per;
     return (int)(b < 4096 ? (b < 1 ? 1 : b) : 4096);
   }
-  // C = alpha op(A) op(B) + beta C for all z
+  // split-K scratch: room for kMaxSplit partial [M][N] slabs per z
+  float* sk = nullptr;
+  int64_t sk_mn = 0;
+  static constexpr int kMaxSplit = 8;
+  // C = alpha op(A) op(B) + beta C for all z. A product with few output tiles
+  // and a long K (the token reductions of the weight gradients) is split over
+  // K into partial slabs, summed by splitk_reduce_kernel in split order.
   void gemm(int Z, int M, int N, int K, const float* A, int lda, int64_t sA, bool tA,
             const float* B, int ldb, int64_t sB, bool tB, float* C, int ldc, int64_t sC,
             float alpha = 1.f, float beta = 0.f) {
     if (M == 0 || N == 0 || Z == 0) return;
-    GemmArgs g{A, B, C, M, N, K, lda, ldb, ldc, tA, tB, sA, sB, sC, alpha, beta};
-    dim3 grid((N + kGT - 1) / kGT, (M + kGT - 1) / kGT, Z);
+    const int tiles = Z * ((N + kGT - 1) / kGT) * ((M + kGT - 1) / kGT);
+    int splits = 1;
+    if (sk && (int64_t)M * N <= sk_mn && tiles < 148 && K >= 8 * kGK) {
+      splits = (2 * 148 + tiles - 1) / tiles;
+      const int by_k = K / (4 * kGK);  // at least four K steps per split
+      if (splits > by_k) splits = by_k;
+      if (splits > kMaxSplit) splits = kMaxSplit;
+    }
+    if (splits <= 1) {
+      GemmArgs g{A, B, C, M, N, K, lda, ldb, ldc, tA, tB, sA, sB, sC, alpha, beta, Z, K};
+      dim3 grid((N + kGT - 1) / kGT, (M + kGT - 1) / kGT, Z);
+      bgemm_kernel<<<grid, 256, 0, s>>>(g);
+      check(cudaGetLastError());
+      return;
+    }
+    const int ksteps = (K + kGK - 1) / kGK;
+    const int kper = (ksteps + splits - 1) / splits * kGK;
+    splits = (K + kper - 1) / kper;
+    GemmArgs g{A, B, sk, M, N, K, lda, ldb, N, tA, tB, sA, sB, (int64_t)M * N, 1.f, 0.f, Z, kper};
+    dim3 grid((N + kGT - 1) / kGT, (M + kGT - 1) / kGT, Z * splits);
     bgemm_kernel<<<grid, 256, 0, s>>>(g);
     check(cudaGetLastError());
+    splitk_reduce_kernel<<<grid1((int64_t)Z * M * N), 256, 0, s>>>(sk, C, Z, M, N, ldc, sC, splits,
+                                                                   alpha, beta);
+    check(cudaGetLastError());
   }
+  int grid1(int64_t n) { return grid(n); }
   void ew(int op, int Z, int64_t n, std::initializer_list<const float*> in,
           std::initializer_list<float*> out, int rows = 0, int cols = 0, float a = 0.f,
           float b = 0.f, float c = 0.f) {
@@ -502,11 +549,17 @@ ttt_status lact_backward(const LactArgs& a, const LactBwdArgs& g, cudaStream_t s
   }
   const size_t o_Xt = take(mn_max), o_dX = take(mn_max), o_dX2 = take(mn_max), o_dP = take(nn_max),
                o_dM = take(nn_max), o_tmp = take(nn_max), o_red = take(2);
+  // split-K slabs for the weight-shaped products; only small batches have
+  // fewer output tiles than SMs, so larger ones get no scratch and no split
+  const int64_t sk_mn = Z <= 16 ? mn_max : 0;
+  const size_t o_sk = take(Ctx::kMaxSplit * sk_mn);
   const size_t bytes = off * sizeof(float);
   void* base = nullptr;
   if (scratch_alloc(&base, bytes, st) != cudaSuccess) return TTT_ERR_ALLOC;
   float* F = static_cast<float*>(base);
   auto P = [&](size_t o) { return F + o; };
+  x.sk = sk_mn > 0 ? P(o_sk) : nullptr;
+  x.sk_mn = sk_mn;
 
   const float* Win[3] = {a.W1, a.W2, a.W3};
   // initial weights per z, row norms
