@@ -31,6 +31,7 @@ constexpr int kThreads = 512;  // 16 warps: the product loops are latency-bound
 constexpr int kTB = 16;
 constexpr int kP = kTB + 1;   // padded token stride of the block buffers
 constexpr int kB = 8;         // global reads issued together per thread
+static_assert(kThreads % kTB == 0, "paired outputs x, x + kThreads share their token");
 
 // floats of the block buffers (before any shared-memory parameter copy)
 __host__ __device__ constexpr int64_t mlp_buf_floats(int dk, int dv, int dh) {
@@ -134,20 +135,34 @@ __global__ void __launch_bounds__(kThreads, 1) ttt_mlp_kernel(MlpArgs a) {
       }
       if (tid < kTB) et[tid] = tid < nt ? eta[(int64_t)(t0 + tid) * a.eta.st] : 0.f;
       __syncthreads();
-      // h = W1_s k + b1_s, and z0 = W1_run q + b1_run (running: earlier blocks applied)
-      for (int x = tid; x < kTB * dh; x += kThreads) {
-        const int j = x / kTB, i = x % kTB;
-        float hk = sb1[j], zq = zb1[j];
+      // h = W1_s k + b1_s, and z0 = W1_run q + b1_run (running: earlier blocks
+      // applied). Each thread takes the outputs x and x + kThreads together (the
+      // same token i, since kThreads is a multiple of kTB): four sums side by
+      // side, each in its own fixed order, sharing the token loads.
+      for (int x = tid; x < kTB * dh; x += 2 * kThreads) {
+        const bool two = x + kThreads < kTB * dh;
+        const int j = x / kTB, i = x % kTB, j2 = two ? (x + kThreads) / kTB : j;
+        float hk = sb1[j], zq = zb1[j], hk2 = sb1[j2], zq2 = zb1[j2];
         const float* w = sW1 + (int64_t)j * dk;
         const float* wr = zW1 + (int64_t)j * dk;
-        #pragma unroll 8
+        const float* w2 = sW1 + (int64_t)j2 * dk;
+        const float* wr2 = zW1 + (int64_t)j2 * dk;
+#pragma unroll 4
         for (int r = 0; r < dk; ++r) {
-          hk = fmaf(w[r], Ks[r * kP + i], hk);
-          zq = fmaf(wr[r], Qs[r * kP + i], zq);
+          const float kr = Ks[r * kP + i], qr = Qs[r * kP + i];
+          hk = fmaf(w[r], kr, hk);
+          zq = fmaf(wr[r], qr, zq);
+          hk2 = fmaf(w2[r], kr, hk2);
+          zq2 = fmaf(wr2[r], qr, zq2);
         }
         Hs[j * kP + i] = fmaxf(hk, 0.f);
         Hm[j * kP + i] = hk > 0.f ? 1.f : 0.f;
         Zs[j * kP + i] = zq;
+        if (two) {
+          Hs[j2 * kP + i] = fmaxf(hk2, 0.f);
+          Hm[j2 * kP + i] = hk2 > 0.f ? 1.f : 0.f;
+          Zs[j2 * kP + i] = zq2;
+        }
       }
       // S1[t][i] = q_t . k_i + 1 (i <= t)
       if (tid < kTB * kTB) {
@@ -160,23 +175,36 @@ __global__ void __launch_bounds__(kThreads, 1) ttt_mlp_kernel(MlpArgs a) {
         S1[t * kP + i] = sv;
       }
       __syncthreads();
-      // r = W2_s a + b2_s - v
-      for (int x = tid; x < kTB * dv; x += kThreads) {
-        const int c = x / kTB, i = x % kTB;
-        float sv = sb2[c];
+      // r = W2_s a + b2_s - v (outputs x and x + kThreads together, as above)
+      for (int x = tid; x < kTB * dv; x += 2 * kThreads) {
+        const bool two = x + kThreads < kTB * dv;
+        const int c = x / kTB, i = x % kTB, c2 = two ? (x + kThreads) / kTB : c;
+        float sv = sb2[c], sv2 = sb2[c2];
         const float* w = sW2 + (int64_t)c * dh;
-        #pragma unroll 8
-        for (int j = 0; j < dh; ++j) sv = fmaf(w[j], Hs[j * kP + i], sv);
+        const float* w2 = sW2 + (int64_t)c2 * dh;
+#pragma unroll 4
+        for (int j = 0; j < dh; ++j) {
+          const float hj = Hs[j * kP + i];
+          sv = fmaf(w[j], hj, sv);
+          sv2 = fmaf(w2[j], hj, sv2);
+        }
         Vs[c * kP + i] = sv - Vs[c * kP + i];
+        if (two) Vs[c2 * kP + i] = sv2 - Vs[c2 * kP + i];
       }
       __syncthreads();
-      // g = (W2_s^T r) [h > 0]
-      for (int x = tid; x < kTB * dh; x += kThreads) {
-        const int j = x / kTB, i = x % kTB;
-        float sv = 0.f;
-        #pragma unroll 8
-        for (int c = 0; c < dv; ++c) sv = fmaf(sW2[(int64_t)c * dh + j], Vs[c * kP + i], sv);
+      // g = (W2_s^T r) [h > 0] (outputs x and x + kThreads together)
+      for (int x = tid; x < kTB * dh; x += 2 * kThreads) {
+        const bool two = x + kThreads < kTB * dh;
+        const int j = x / kTB, i = x % kTB, j2 = two ? (x + kThreads) / kTB : j;
+        float sv = 0.f, sv2 = 0.f;
+#pragma unroll 4
+        for (int c = 0; c < dv; ++c) {
+          const float rc = Vs[c * kP + i];
+          sv = fmaf(sW2[(int64_t)c * dh + j], rc, sv);
+          sv2 = fmaf(sW2[(int64_t)c * dh + j2], rc, sv2);
+        }
         Gs[j * kP + i] = sv * Hm[j * kP + i];
+        if (two) Gs[j2 * kP + i] = sv2 * Hm[j2 * kP + i];
       }
       __syncthreads();
       // z = z0 - sum_{i<=t} eta_i S1[t][i] g_i ; a' = ReLU(z)
@@ -199,16 +227,28 @@ __global__ void __launch_bounds__(kThreads, 1) ttt_mlp_kernel(MlpArgs a) {
       }
       __syncthreads();
       // y = W2_run a' + b2_run - sum_{i<=t} eta_i S2[t][i] r_i
-      for (int x = tid; x < kTB * dv; x += kThreads) {
-        const int c = x / kTB, t = x % kTB;
+      // (outputs x and x + kThreads together: the same token t)
+      for (int x = tid; x < kTB * dv; x += 2 * kThreads) {
+        const bool two = x + kThreads < kTB * dv;
+        const int c = x / kTB, t = x % kTB, c2 = two ? (x + kThreads) / kTB : c;
         if (t < nt) {
-          float y = zb2[c];
+          float y = zb2[c], y2 = zb2[c2];
           const float* w = zW2 + (int64_t)c * dh;
-          #pragma unroll 8
-          for (int j = 0; j < dh; ++j) y = fmaf(w[j], Zs[j * kP + t], y);
-          for (int i = 0; i <= t; ++i) y = fmaf(-et[i] * S2[t * kP + i], Vs[c * kP + i], y);
+          const float* w2 = zW2 + (int64_t)c2 * dh;
+#pragma unroll 4
+          for (int j = 0; j < dh; ++j) {
+            const float zj = Zs[j * kP + t];
+            y = fmaf(w[j], zj, y);
+            y2 = fmaf(w2[j], zj, y2);
+          }
+          for (int i = 0; i <= t; ++i) {
+            const float sti = -et[i] * S2[t * kP + i];
+            y = fmaf(sti, Vs[c * kP + i], y);
+            y2 = fmaf(sti, Vs[c2 * kP + i], y2);
+          }
           T* o = static_cast<T*>(a.out.p) + b * a.out.sb + h * a.out.sh + (int64_t)(t0 + t) * a.out.st;
           o[c] = T(y);
+          if (two) o[c2] = T(y2);
         }
       }
       __syncthreads();
