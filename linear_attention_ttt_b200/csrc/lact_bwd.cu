@@ -33,10 +33,10 @@
 // silu'(x) = s (1 + x (1 - s)) and silu''(x) = s (1 - s)(2 + x (1 - 2 s)),
 // s = sigmoid(x).
 //
-// Correctness first: fp32 arithmetic throughout (batched fp32 GEMMs on the
-// CUDA cores and elementwise / row kernels), orchestrated chunk by chunk from
-// the host over all (batch, head) pairs at once. A forward pass in the same
-// fp32 arithmetic stores the start weights of every chunk.
+// fp32 arithmetic throughout (batched fp32 GEMMs on the CUDA cores and
+// elementwise / row kernels), orchestrated chunk by chunk from the host over
+// all (batch, head) pairs at once. A forward pass in the same fp32 arithmetic
+// stores the start weights of every chunk.
 #include <cstring>
 #include <vector>
 
@@ -48,7 +48,10 @@ namespace {
 // ---------------------------------------------------------------------------
 // Batched fp32 GEMM: C[z] = alpha op(A[z]) op(B[z]) + beta C[z], op(A) M x K,
 // op(B) K x N; tA: A stored K x M (A[k * lda + m]); tB: B stored N x K.
-// 64 x 64 output tiles, 256 threads with 4 x 4 outputs each, K steps of 16.
+// 64 x 64 output tiles, 256 threads with 4 x 4 outputs each, K steps of 16,
+// the next step's operands fetched into registers during the current one.
+// With blockIdx.z = split * Z + z, split s covers one K range and writes its
+// partial tile to slab (split * Z + z) of C (see Ctx::gemm).
 // ---------------------------------------------------------------------------
 constexpr int kGT = 64, kGK = 16;
 
