@@ -79,6 +79,12 @@ def linear_bwd_flops(w):
     return w.B * w.H * w.T * n * w.dk * w.dv
 
 
+def ttt_mlp_flops(B, H, T, dk, dv, dh):
+    # The per-token rule: h = W1 k, z = W1 q and the W1 update at 2 dk dh each;
+    # r = W2 a, g = W2^T r, y = W2 a' and the W2 update at 2 dh dv each.
+    return B * H * T * (6 * dk * dh + 8 * dh * dv)
+
+
 def linear_flops(w):
     # qW, kW and K^T(NE) at 2 dk dv each (MSE) or qW and K^T(NV) (inner
     # product), plus the causal half of the intra-chunk products.
@@ -567,7 +573,9 @@ def measure_next_rows(runner, device):
     t = [dev(getattr(w, n), w.dtype) for n in ("q", "k", "v")] + [dev(w.eta, synth.F32)]
     Pd = [dev(p, synth.F32) for p in P]
     run("f3 ttt-mlp", {"workload": "ttt_mlp_bf16_B4_H16_T2048_d64_dh256_b16"},
-        lambda: ops.ttt_mlp_fwd(*t, *Pd, 16), w.B * w.T)
+        lambda: ops.ttt_mlp_fwd(*t, *Pd, 16), w.B * w.T,
+        roof=("alu", ttt_mlp_flops(w.B, w.H, w.T, w.dk, w.dv, 256), FP32_ALU_TFLOPS, "TFLOP/s",
+              "ttt_mlp"))
     del t, Pd
     # f4a: window attention (window 4096) and the LaCT + window block, Muon workload
     w = synth.config(5)
